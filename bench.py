@@ -1,0 +1,583 @@
+"""Paged decode benchmark: one step = KV append + paged decode attention for one
+synthetic batch, through the library's C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  ``value`` is decode tokens/s over all ranks
+(one new token per sequence per step), timed on the device with CUDA events
+over exactly K steps replayed from a CUDA graph, inputs resident in HBM.  L2
+is defeated by rotating over several copies of the KV pool whose total is a
+multiple of the L2 size.  ``roofline`` reports the decode launch's achieved
+HBM bandwidth on the algorithmic KV bytes; ``e2e`` repeats the measurement
+through the public Python API with the step's inputs copied from pinned host
+memory and the output copied back inside the timed region; ``cpu_baseline``
+times the fp64 CPU oracle on a bounded sample of the same workload.
+
+Multi-GPU (torchrun): every rank runs its own independent batch (different
+seed); there is no data-path collective.  Time = max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from paged_kv_cache_473_b200 import workloads as wl  # noqa: E402
+
+METRIC = "paged decode tokens/s and achieved HBM GB/s (% of B200 peak) per batch shape"
+HEADLINE = "tinyllama_1b"
+FALLBACK_HBM_GBS = 6650.0
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=HEADLINE, choices=list(wl.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--kernel", default="auto", choices=["auto", "cuda_core", "mma"])
+    ap.add_argument("--no-split", action="store_true", help="time pa_decode (one CTA per sequence, kv head)")
+    ap.add_argument("--partition", type=int, default=-1, help="split-K partition tokens (0 auto; -1 workload's)")
+    ap.add_argument("--shapes", default="auto", help="comma list of extra workloads to time, 'none', or 'auto'")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="bound on the CPU-oracle sample")
+    ap.add_argument("--no-cpu", action="store_true")
+    return ap.parse_args()
+
+
+# ---- distributed plumbing -----------------------------------------------------------
+
+
+def dist_init(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def rank_seed(w: wl.Workload, rank: int) -> int:
+    """Each rank draws an independent batch of the same shape."""
+    return w.seed + 7919 * rank
+
+
+# ---- clocks -------------------------------------------------------------------------
+
+_REASON_BITS = {
+    0x1: "gpu_idle",
+    0x2: "applications_clocks_setting",
+    0x4: "sw_power_cap",
+    0x8: "hw_slowdown",
+    0x10: "sync_boost",
+    0x20: "sw_thermal_slowdown",
+    0x40: "hw_thermal_slowdown",
+    0x80: "hw_power_brake_slowdown",
+    0x100: "display_clock_setting",
+}
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # noqa: BLE001
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        get_r = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(get_r(self._h))
+            except Exception:  # noqa: BLE001
+                break
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"], "samples": 0}
+        s = sorted(self.samples)
+        reasons = [n for bit, n in _REASON_BITS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": s[len(s) // 2], "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(s)}
+
+
+# ---- helpers --------------------------------------------------------------------------
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:  # noqa: BLE001
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "paged_kv_cache_473_b200", "csrc")
+    for n in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, n), "rb") as f:
+            h.update(n.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str, kernel_key: str):
+    """dram bytes per launch from a committed ncu summary, if taken on the current sources."""
+    try:
+        with open(PROFILE_TRAFFIC) as f:
+            d = json.load(f)
+        e = d[workload][kernel_key]
+        if e.get("source_hash") != kernel_source_hash():
+            return None
+        return int(e["dram_bytes_per_launch"])
+    except Exception:  # noqa: BLE001
+        return None
+
+
+def pool_copies(pool_bytes: int, l2_bytes: int) -> int:
+    """Rotate over enough pool copies that one pass over them is >= 4x L2."""
+    return max(1, min(16, math.ceil(4 * l2_bytes / max(1, pool_bytes))))
+
+
+# ---- our implementation ------------------------------------------------------------------
+
+
+class Runner:
+    """One workload on this GPU: rotating KV pools, persistent output/workspace."""
+
+    def __init__(self, w: wl.Workload, rank: int, kernel: str, split: bool, partition: int):
+        import paged_kv_cache_473_b200 as pa
+
+        self.pa = pa
+        self.w = w
+        self.kernel = kernel
+        self.split = split
+        self.batch = wl.make_batch(w, seed=rank_seed(w, rank), device="cuda")
+        b = self.batch
+        self.B = b.q.shape[0]
+        l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+        pool_bytes = 2 * b.k_cache.numel() * b.k_cache.element_size()
+        self.R = pool_copies(pool_bytes, l2)
+        self.pools = [(b.k_cache, b.v_cache)] + [(b.k_cache.clone(), b.v_cache.clone()) for _ in range(self.R - 1)]
+        self.pool_bytes_total = pool_bytes * self.R
+        self.max_ctx = max(1, b.max_context_len)
+        self.partition = pa.decode_splitk_partition(self.B, w.num_kv_heads, self.max_ctx,
+                                                    w.partition_tokens if partition < 0 else partition)
+        nbytes = pa.decode_splitk_workspace_size(self.B, w.num_q_heads, w.head_dim, self.max_ctx, self.partition,
+                                                 w.num_kv_heads)
+        self.ws = torch.empty(max(16, nbytes), dtype=torch.uint8, device="cuda")
+        self.out = torch.empty_like(b.q)
+        self.kv_bytes = wl.kv_bytes(b)
+        self.kv_bytes_unique = wl.kv_bytes(b, unique=True)
+        self.decode_launches = 0
+
+    def append(self, r, k_new=None, v_new=None, slots=None):
+        b = self.batch
+        kc, vc = self.pools[r]
+        self.pa.write_kv(b.k_new if k_new is None else k_new, b.v_new if v_new is None else v_new,
+                         b.slot_mapping if slots is None else slots, kc, vc)
+
+    def decode(self, r, q=None, tables=None, lens=None):
+        b, w = self.batch, self.w
+        kc, vc = self.pools[r]
+        q = b.q if q is None else q
+        tables = b.block_tables if tables is None else tables
+        lens = b.context_lens if lens is None else lens
+        if self.split:
+            self.pa.decode_splitk(q, kc, vc, tables, lens, w.scale, w.softcap, w.window,
+                                  max_context_len=self.max_ctx, partition_tokens=self.partition, out=self.out,
+                                  workspace=self.ws, kernel=self.kernel)
+        else:
+            self.pa.decode(q, kc, vc, tables, lens, w.scale, w.softcap, w.window, out=self.out, kernel=self.kernel)
+        self.decode_launches = self.pa.last_launch_count()
+
+    def step(self, r):
+        self.append(r)
+        self.decode(r)
+
+    def timed_graph(self, K: int):
+        """Capture K steps (pool i % R) with external timing events around each decode."""
+        ev = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
+              for _ in range(K)]
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                for i in range(K):
+                    r = i % self.R
+                    self.append(r)
+                    ev[i][0].record()
+                    self.decode(r)
+                    ev[i][1].record()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        return g, ev
+
+
+def run_timed(runner: Runner, K: int, W: int, world: int, device_index: int):
+    """Warm up W steps, then time exactly K graph-replayed steps."""
+    for i in range(W):
+        runner.step(i % runner.R)
+    torch.cuda.synchronize()
+    g, ev = runner.timed_graph(K)
+    # Warm the graph once (the replay itself is not counted).
+    g.replay()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(device_index) as clk:
+        start.record()
+        g.replay()
+        end.record()
+        torch.cuda.synchronize()
+    barrier(world)
+    total_ms = start.elapsed_time(end)
+    dec_ms = [a.elapsed_time(b) for a, b in ev]
+    del g
+    return total_ms, sum(dec_ms) / len(dec_ms), clk.summary()
+
+
+def run_e2e(runner: Runner, K: int, world: int):
+    """Public-API step with host inputs: H2D of the step's inputs, append, decode,
+    D2H of the output, all inside the timed region (eager launches)."""
+    b = runner.batch
+    host = {n: getattr(b, n).cpu().pin_memory() for n in ("q", "k_new", "v_new", "slot_mapping", "block_tables",
+                                                         "context_lens")}
+    dev = {n: torch.empty_like(getattr(b, n)) for n in host}
+    out_host = torch.empty(b.q.shape, dtype=b.q.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def one(i):
+        for n in host:
+            dev[n].copy_(host[n], non_blocking=True)
+        r = i % runner.R
+        runner.append(r, dev["k_new"], dev["v_new"], dev["slot_mapping"])
+        runner.decode(r, dev["q"], dev["block_tables"], dev["context_lens"])
+        out_host.copy_(runner.out, non_blocking=True)
+
+    for i in range(3):
+        one(i)
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    start.record()
+    for i in range(K):
+        one(i)
+    end.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    return start.elapsed_time(end), h2d, d2h
+
+
+class OracleSample:
+    """The CPU oracle as it stands, timed on a bounded sample of one workload
+    (the batch is copied to host memory once, outside any timing)."""
+
+    def __init__(self, w: wl.Workload, batch: wl.Batch):
+        import oracle
+
+        self.oracle = oracle
+        self.w = w
+        self.cpu = dict(q=batch.q.cpu(), k_new=batch.k_new.cpu(), v_new=batch.v_new.cpu(),
+                        slots=batch.slot_mapping.cpu(), kc=batch.k_cache.cpu(), vc=batch.v_cache.cpu(),
+                        tables=batch.block_tables.cpu(), lens=batch.context_lens.cpu())
+        oracle.build()
+        self.threads = oracle.num_threads()
+        c = self.cpu
+        self.B, self.hq = c["q"].shape[0], c["q"].shape[1]
+        t0 = time.perf_counter()
+        self._decode([(0, h) for h in range(self.hq)])
+        el = time.perf_counter() - t0
+        self.per_seq = max(1e-6, el * float(c["lens"].double().mean()) / max(1, int(c["lens"][0])))
+
+    def _decode(self, rows):
+        c, w = self.cpu, self.w
+        return self.oracle.decode(c["q"], c["kc"], c["vc"], c["tables"], c["lens"], w.scale, w.softcap, w.window,
+                                  rows=rows)
+
+    def run(self, seconds: float):
+        """Whole steps (append + decode of every sequence) until ``seconds`` of
+        work have run, or one step over the first n sequences when a whole step
+        would take longer than that."""
+        c = self.cpu
+        B, hq = self.B, self.hq
+        n_seq = B if self.per_seq * B <= seconds else max(1, int(seconds / self.per_seq))
+        rows = None if n_seq == B else [(i, h) for i in range(n_seq) for h in range(hq)]
+        steps = tokens = 0
+        t0 = time.perf_counter()
+        while True:
+            self.oracle.write_kv(c["k_new"][:n_seq], c["v_new"][:n_seq], c["slots"][:n_seq], c["kc"], c["vc"])
+            self._decode(rows)
+            steps += 1
+            tokens += n_seq
+            el = time.perf_counter() - t0
+            if el >= seconds or n_seq < B:
+                break
+        sample = (f"{steps} whole step(s): append + decode of all {B} sequences, fp64" if n_seq == B else
+                  f"append + decode of the first {n_seq} of {B} sequences (all {hq} query heads), fp64")
+        return {"value": tokens / el, "unit": "tokens/s", "cores": self.threads, "kind": "oracle", "sample": sample,
+                "seconds": round(el, 3)}
+
+
+def describe(w: wl.Workload, runner: Runner, args, l2_note: str):
+    return {
+        "workload": w.name,
+        "batch": runner.B,
+        "num_q_heads": w.num_q_heads,
+        "num_kv_heads": w.num_kv_heads,
+        "head_dim": w.head_dim,
+        "block_size": w.block_size,
+        "lengths": list(w.lengths),
+        "mean_context": round(float(runner.batch.context_lens.double().mean()), 1),
+        "softcap": w.softcap,
+        "window": w.window,
+        "prefix_share": w.prefix_share,
+        "path": "pa_decode" if not runner.split else f"pa_decode_splitk(partition={runner.partition})",
+        "kernel": args.kernel,
+        "l2": l2_note,
+        "seed": "workload seed + 7919 * rank",
+    }
+
+
+def shape_summary(w: wl.Workload, rank: int, kernel: str, K: int, W: int, world: int, dev_idx: int, peak: float):
+    runner = Runner(w, rank, kernel, True, -1)
+    total_ms, dec_ms, _ = run_timed(runner, K, W, world, dev_idx)
+    ms = total_ms / K
+    res = {
+        "tokens_per_s": round(runner.B / (ms * 1e-3), 1),
+        "ms_per_step": round(ms, 5),
+        "decode_ms": round(dec_ms, 5),
+        "decode_gbs": round(runner.kv_bytes / (dec_ms * 1e-3) / 1e9, 1),
+        "decode_frac": round(runner.kv_bytes / (dec_ms * 1e-3) / 1e9 / peak, 4),
+        "kv_bytes": runner.kv_bytes,
+        "kv_bytes_unique": runner.kv_bytes_unique,
+        "partition": runner.partition,
+    }
+    if runner.kv_bytes_unique != runner.kv_bytes:
+        res["decode_gbs_unique"] = round(runner.kv_bytes_unique / (dec_ms * 1e-3) / 1e9, 1)
+    del runner
+    torch.cuda.empty_cache()
+    return res
+
+
+def main_ours(args, world, rank, local):
+    w = wl.WORKLOADS[args.workload]
+    split = not args.no_split
+    runner = Runner(w, rank, args.kernel, split, args.partition)
+    l2 = torch.cuda.get_device_properties(local).L2_cache_size
+    l2_note = (f"rotating {runner.R} KV pool copies ({runner.pool_bytes_total / 1e6:.0f} MB, "
+               f"L2 {l2 / 1e6:.0f} MB)")
+    K, W = args.steps, args.warmup
+    total_ms, dec_ms, clocks = run_timed(runner, K, W, world, local)
+    total_ms = max_over_ranks(total_ms, world)
+    dec_ms = max_over_ranks(dec_ms, world)
+    tokens = sum_over_ranks(runner.B * K, world)
+    value = tokens / (total_ms * 1e-3)
+    e2e_ms, h2d, d2h = run_e2e(runner, K, world)
+    e2e_ms = max_over_ranks(e2e_ms, world)
+    peak, peak_kind = measured_peaks()
+    achieved = runner.kv_bytes / (dec_ms * 1e-3) / 1e9
+    kernel_key = "splitk" if split else "decode"
+    traffic = recorded_traffic(w.name, kernel_key)
+    launches_per_step = 1 + runner.decode_launches
+    line = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": round(total_ms / K, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.dtype,
+        "data": "synthetic (seeded; q/k/v ~ N(0,1), shuffled physical blocks, NaN canaries in dead slots)",
+        "config": describe(w, runner, args, l2_note),
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "decode (split-K partial + LSE combine)" if split else "decode",
+            "achieved": round(achieved, 1),
+            "peak": peak,
+            "peak_kind": peak_kind,
+            "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": traffic,
+            "algorithmic_bytes_per_launch": runner.kv_bytes,
+            "launch_ms": round(dec_ms, 5),
+        },
+        "e2e": {
+            "value": round(tokens / (e2e_ms * 1e-3), 1),
+            "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(e2e_ms / K, 5),
+        },
+        "gpu_launches": K * launches_per_step,
+        "clocks": clocks,
+    }
+    if world == 1 and rank == 0 and args.shapes != "none":
+        names = [n for n in wl.WORKLOADS if n not in (w.name, "tiny_fp32")] if args.shapes == "auto" else [
+            s for s in args.shapes.split(",") if s]
+        extra = {}
+        del runner
+        torch.cuda.empty_cache()
+        for n in names:
+            extra[n] = shape_summary(wl.WORKLOADS[n], rank, args.kernel, 50, 5, world, local, peak)
+        line["per_shape"] = extra
+        runner = None
+    if world == 1 and rank == 0 and not args.no_cpu:
+        b = wl.make_batch(w, seed=rank_seed(w, rank), device="cuda")
+        info = OracleSample(w, b).run(args.cpu_seconds)
+        info["value"] = round(info["value"], 2)
+        line["cpu_baseline"] = info
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main_reference(args, rank):
+    """The CPU oracle as the reference arm, on this run's workload and metric.
+    Under torchrun only rank 0 works; the other ranks return at once."""
+    if rank != 0:
+        return
+    w = wl.WORKLOADS[args.workload]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    b = wl.make_batch(w, seed=rank_seed(w, 0), device=dev)
+    sampler = OracleSample(w, b)
+    del b
+    K, W = args.steps, args.warmup
+    budget = max(0.05, 120.0 / max(1, K + W))  # keep the whole run within a few minutes
+    for _ in range(W):
+        sampler.run(budget)
+    t_tokens = t_secs = 0.0
+    info = None
+    for _ in range(K):
+        info = sampler.run(budget)
+        t_tokens += info["value"] * info["seconds"]
+        t_secs += info["seconds"]
+    value = t_tokens / t_secs
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": round(1e3 * t_secs / K, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded)",
+        "impl": "reference",
+        "config": {"workload": w.name, "batch": sampler.B, "path": "fp64 CPU oracle (C, OpenMP)"},
+        "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": info["cores"], "kind": "oracle",
+                         "sample": f"each step: {info['sample']}"},
+        "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        main_reference(args, int(os.environ.get("RANK", "0")))
+        return
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py --impl ours needs a CUDA device")
+    world, rank, local = dist_init(args)
+    try:
+        main_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,171 @@
+/*
+ * pagedattn.h -- C ABI of the B200 (sm_100a) paged KV cache library.
+ *
+ * Decode-phase attention over a block-structured KV cache, as used by
+ * nano-vLLM-style engines: a batch of sequences each brings one new query
+ * token; each sequence's keys and values live in fixed-size physical blocks of
+ * one shared pool and are reached through a per-sequence block table.
+ *
+ * Passages this interface follows (the pages print no kernel interface):
+ *   - nano-vllm (ovshake) README, "Key Concepts Explained: PagedAttention":
+ *     KV storage is a pool of fixed-size blocks handed to sequences on demand,
+ *     in any physical order; each sequence keeps the list of its blocks.
+ *   - same README, "Key Concepts Explained: KV Cache": a decode step computes
+ *     K and V for the new token only and attends over everything cached.
+ *   - same README, "X-Ray Mode", Steps 1-2: grouped-query attention (32 query
+ *     heads share 8 KV heads) and scores Q K^T / sqrt(head_dim).
+ *   - flex-nano-vllm README: paged attention with a page table serving
+ *     Gemma 2 (the source of the tanh logit softcap and sliding window).
+ *   - MinivLLM summary (sourcepulse), "How It Works": paging of the KV cache
+ *     for decoding, blockwise exact attention.
+ *
+ * Conventions common to every call
+ *   Cache layout ("HND"): k_cache and v_cache are row-major
+ *     [num_blocks][num_kv_heads][block_size][head_dim] of dtype elements, so
+ *     one (physical block, kv head) pair is one contiguous run of
+ *     block_size * head_dim elements.  slot s names row (s % block_size) of
+ *     block (s / block_size).
+ *   Tensors q, out: [batch][num_q_heads][head_dim]; k, v (new rows):
+ *     [num_tokens][num_kv_heads][head_dim]; block_tables:
+ *     [batch][max_blocks_per_seq] int32 (entries past a sequence's last block
+ *     are never read); context_lens: [batch] int32.
+ *   context_lens[b] counts every cached token of sequence b, including the one
+ *     appended this step (the query sits at position L-1).  L = 0 gives a zero
+ *     output row.
+ *   GQA: query head h reads kv head h / (num_q_heads / num_kv_heads).
+ *   scale multiplies q.k; softcap c > 0 and finite replaces a scaled score x by
+ *     c * tanh(x / c) (softcap <= 0 or +inf: no cap); window W > 0 keeps the
+ *     last W positions [max(0, L-W), L) (W <= 0: no window).
+ *   Supported: head_dim in {64, 128, 256}; block_size a power of two in
+ *     [16, 256]; 1 <= num_q_heads / num_kv_heads <= 8 (integral);
+ *     batch <= 65535; num_blocks * num_kv_heads * block_size < 2^31.
+ *   Memory: every pointer is caller-owned DEVICE memory of the current device
+ *     (q, caches, k, v, out, workspace 16-byte aligned; int32 arrays 4-byte;
+ *     slot_mapping 8-byte).  The library allocates nothing and keeps no state
+ *     beyond per-device constants and the device error word below.
+ *   Streams: every call is asynchronous on `stream` (NULL = the legacy
+ *     default stream); ordering follows stream order, so an append must be
+ *     issued before the decode that reads it on the same stream.
+ *   Errors: host checks run before anything is launched; a failed check
+ *     returns an error status and launches nothing.  Kernels never trap: bad
+ *     device-side values (a block id outside the pool, a slot outside the
+ *     pool, a context longer than its table) skip the access and set a bit in
+ *     the device error word, read back with pa_device_errors().
+ */
+#ifndef PAGEDATTN_H_
+#define PAGEDATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st; /* cudaStream_t is `struct CUstream_st *` */
+typedef struct CUstream_st* pa_stream_t;
+
+typedef enum { PA_F32 = 0, PA_BF16 = 1 } pa_dtype_t;
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID = 1,     /* an argument failed a host check; nothing was launched */
+  PA_ERR_UNSUPPORTED = 2, /* well-formed but outside what the kernels implement */
+  PA_ERR_WORKSPACE = 3,   /* split-K workspace missing, misaligned or too small */
+  PA_ERR_CUDA = 4         /* a CUDA runtime call or a launch failed */
+} pa_status_t;
+
+/* Which decode kernel runs.  AUTO picks the tensor-core kernel for bf16 and the
+ * CUDA-core kernel for fp32.  MMA is bf16 only. */
+typedef enum { PA_KERNEL_AUTO = 0, PA_KERNEL_CUDA_CORE = 1, PA_KERNEL_MMA = 2 } pa_kernel_t;
+
+/* Bits of the device error word. */
+enum {
+  PA_DEVERR_SLOT = 1u,       /* write_kv: slot >= num_blocks * block_size (row skipped) */
+  PA_DEVERR_BLOCK = 2u,      /* decode: block id outside [0, num_blocks) (tile skipped) */
+  PA_DEVERR_CONTEXT = 4u,    /* decode: context_lens[b] < 0 or > max_blocks_per_seq * block_size,
+                                or > max_context_len in split-K (length clamped) */
+  PA_DEVERR_TIMEOUT = 8u     /* a bounded wait on a tile load gave up (output row not written) */
+};
+
+/*
+ * pa_write_kv -- append one step's new key/value rows into the paged cache.
+ *   For every i < num_tokens with slot_mapping[i] >= 0 and every kv head h:
+ *     k_cache[s / bs][h][s % bs][:] = k[i][h][:]   (and the same for v)
+ *   The copy is bit-exact.  slot_mapping[i] < 0 marks a padding token (skipped).
+ *   A slot >= num_blocks * block_size sets PA_DEVERR_SLOT and is skipped.
+ *   Two tokens with the same slot in one call: which one lands is undefined.
+ *   Passage: nano-vllm README, "Key Concepts Explained: KV Cache" (only the new
+ *   token's K and V are computed; the rest are reused from the cache).
+ *   Returns PA_ERR_INVALID for null/misaligned pointers or bad sizes.
+ */
+pa_status_t pa_write_kv(const void* k, const void* v, const int64_t* slot_mapping, int32_t num_tokens,
+                        void* k_cache, void* v_cache, int32_t num_blocks, int32_t block_size,
+                        int32_t num_kv_heads, int32_t head_dim, pa_dtype_t dtype, pa_stream_t stream);
+
+/*
+ * pa_decode -- paged decode attention, one CTA per (sequence, kv head).
+ *   out[b][h][:] = sum_t softmax_t(x) V[b][g][t][:],  t in [s0, L),
+ *   x_t = scale * q[b][h] . K[b][g][t]  (then the softcap), g = h / G,
+ *   where K[b][g][t] is row t % bs of block block_tables[b][t / bs].
+ *   Accumulation and the softmax state are fp32; out has the input dtype
+ *   (bf16 rounded to nearest even).  Needs no workspace.
+ *   Passages: see the file header (PagedAttention, KV Cache, X-Ray Mode).
+ */
+pa_status_t pa_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                      const int32_t* context_lens, int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                      int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq, int32_t num_blocks,
+                      float scale, float softcap, int32_t window, void* out, pa_dtype_t dtype,
+                      pa_kernel_t kernel, pa_stream_t stream);
+
+/*
+ * Split-K (flash-decoding) variant for long contexts and small batches.
+ *   Each sequence's attended range is cut at multiples of partition_tokens;
+ *   one CTA per (partition, kv head, sequence) writes its partial softmax state
+ *   (running max m, sum l, unnormalised output o, all fp32) to the workspace,
+ *   and a second kernel merges the partials with a log-sum-exp combine:
+ *     M = max_p m_p,  out = sum_p e^(m_p - M) o_p / sum_p e^(m_p - M) l_p.
+ *   A sequence whose range falls in one partition is written directly by that
+ *   partition's CTA; its result is then bit-identical to pa_decode's.
+ *   partition_tokens: a multiple of 64, or 0 to let the library choose (see
+ *   pa_decode_splitk_partition).  max_context_len: an upper bound on every
+ *   context_lens[b] (a larger length sets PA_DEVERR_CONTEXT and is clamped);
+ *   it sizes the grid and the workspace.
+ *   workspace: device memory of at least pa_decode_splitk_workspace_size()
+ *   bytes, 16-byte aligned; its contents need no initialisation and are
+ *   scratch between the two kernels of one call.  Calls that share a workspace
+ *   must be ordered on one stream.
+ *   Returns PA_ERR_WORKSPACE when the workspace is null, misaligned or small.
+ */
+int32_t pa_decode_splitk_partition(int32_t batch, int32_t num_kv_heads, int32_t max_context_len,
+                                   int32_t partition_tokens);
+size_t pa_decode_splitk_workspace_size(int32_t batch, int32_t num_q_heads, int32_t head_dim,
+                                       int32_t max_context_len, int32_t partition_tokens,
+                                       int32_t num_kv_heads);
+pa_status_t pa_decode_splitk(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                             const int32_t* context_lens, int32_t batch, int32_t num_q_heads,
+                             int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                             int32_t max_blocks_per_seq, int32_t num_blocks, float scale, float softcap,
+                             int32_t window, void* out, pa_dtype_t dtype, int32_t partition_tokens,
+                             int32_t max_context_len, void* workspace, size_t workspace_bytes,
+                             pa_kernel_t kernel, pa_stream_t stream);
+
+/*
+ * pa_device_errors -- read (and with clear != 0, reset) the device error word
+ * of the current device.  Synchronises with the device.  *bits receives the
+ * OR of every PA_DEVERR_* raised since the last clear.
+ */
+pa_status_t pa_device_errors(uint32_t* bits, int32_t clear);
+
+/* Static description of a status code. */
+const char* pa_error_string(pa_status_t status);
+
+/* Number of kernels the last successful call on this host thread launched
+ * (0 after a failed call).  For accounting in benchmarks. */
+int32_t pa_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDATTN_H_ */

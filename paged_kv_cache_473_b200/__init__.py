@@ -1,1 +1,36 @@
+"""B200 (sm_100a) paged KV cache: KV append and paged decode attention.
 
+The compute lives in ``libpagedattn.so`` (C ABI, include/pagedattn.h); this
+package is its Python binding plus seeded synthetic batch generators
+(``workloads``) and the in-tree build step (``build``).
+"""
+
+from ._binding import (  # noqa: F401
+    DEVERR_BLOCK,
+    DEVERR_CONTEXT,
+    DEVERR_SLOT,
+    DEVERR_TIMEOUT,
+    KERNELS,
+    PagedAttnError,
+    decode,
+    decode_splitk,
+    decode_splitk_partition,
+    decode_splitk_workspace_size,
+    device_errors,
+    error_string,
+    last_launch_count,
+    lib,
+    write_kv,
+)
+
+__all__ = [
+    "write_kv",
+    "decode",
+    "decode_splitk",
+    "decode_splitk_partition",
+    "decode_splitk_workspace_size",
+    "device_errors",
+    "error_string",
+    "last_launch_count",
+    "PagedAttnError",
+]

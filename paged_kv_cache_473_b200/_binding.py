@@ -1,0 +1,168 @@
+"""ctypes binding of ``libpagedattn.so`` (include/pagedattn.h).
+
+Argument marshalling only: shapes, raw device pointers and the current CUDA
+stream go to the C ABI; every step of the computation runs in the library's
+kernels.  torch provides device memory (the optional ``out`` tensors and the
+split-K workspace) and streams.  The binding refuses to run if the library is
+missing or cannot be built; there is no fallback path.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+from . import build as _build
+
+PA_F32, PA_BF16 = 0, 1
+PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_CUDA = 0, 1, 2, 3, 4
+KERNELS = {"auto": 0, "cuda_core": 1, "mma": 2}
+DEVERR_SLOT, DEVERR_BLOCK, DEVERR_CONTEXT, DEVERR_TIMEOUT = 1, 2, 4, 8
+
+_c_i32, _c_i64, _c_f32, _c_sz, _c_vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t, ctypes.c_void_p
+
+
+class PagedAttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: status {status} ({error_string(status)})")
+
+
+def _load_library() -> ctypes.CDLL:
+    path = _build.LIB
+    if not _build.up_to_date():
+        try:
+            path = _build.build()
+        except Exception as e:  # noqa: BLE001
+            if not os.path.exists(path):
+                raise ImportError(f"libpagedattn.so is missing and could not be built: {e}") from e
+    lib = ctypes.CDLL(path)
+    lib.pa_write_kv.argtypes = [_c_vp, _c_vp, _c_vp, _c_i32, _c_vp, _c_vp, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32,
+                                _c_vp]
+    lib.pa_write_kv.restype = _c_i32
+    dec = [_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_f32, _c_f32,
+           _c_i32, _c_vp, _c_i32]
+    lib.pa_decode.argtypes = dec + [_c_i32, _c_vp]
+    lib.pa_decode.restype = _c_i32
+    lib.pa_decode_splitk.argtypes = dec + [_c_i32, _c_i32, _c_vp, _c_sz, _c_i32, _c_vp]
+    lib.pa_decode_splitk.restype = _c_i32
+    lib.pa_decode_splitk_partition.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32]
+    lib.pa_decode_splitk_partition.restype = _c_i32
+    lib.pa_decode_splitk_workspace_size.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32]
+    lib.pa_decode_splitk_workspace_size.restype = _c_sz
+    lib.pa_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint32), _c_i32]
+    lib.pa_device_errors.restype = _c_i32
+    lib.pa_error_string.argtypes = [_c_i32]
+    lib.pa_error_string.restype = ctypes.c_char_p
+    lib.pa_last_launch_count.argtypes = []
+    lib.pa_last_launch_count.restype = _c_i32
+    return lib
+
+
+lib = _load_library()
+
+
+def error_string(status: int) -> str:
+    return lib.pa_error_string(int(status)).decode()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return PA_F32
+    if t.dtype == torch.bfloat16:
+        return PA_BF16
+    raise TypeError(f"paged attention takes float32 or bfloat16 tensors, got {t.dtype}")
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _check(status: int, what: str) -> None:
+    if status != PA_OK:
+        raise PagedAttnError(status, what)
+
+
+def write_kv(k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor, k_cache: torch.Tensor,
+             v_cache: torch.Tensor, stream=None) -> None:
+    """Append ``k``/``v`` rows ``[N, Hkv, D]`` into the caches at ``slot_mapping`` (int64)."""
+    nb, hkv, bs, d = k_cache.shape
+    st = lib.pa_write_kv(_ptr(k), _ptr(v), _ptr(slot_mapping), slot_mapping.numel(), _ptr(k_cache), _ptr(v_cache),
+                         nb, bs, hkv, d, _dtype_code(k_cache), _stream(stream))
+    _check(st, "pa_write_kv")
+
+
+def _decode_common(q, k_cache, block_tables, out):
+    B, hq, d = q.shape
+    nb, hkv, bs, d2 = k_cache.shape
+    if out is None:
+        out = torch.empty_like(q)
+    return B, hq, d, nb, hkv, bs, out
+
+
+def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_tables: torch.Tensor,
+           context_lens: torch.Tensor, scale: float, softcap: float = 0.0, window: int = 0,
+           out: Optional[torch.Tensor] = None, kernel: str = "auto", stream=None) -> torch.Tensor:
+    """Paged decode attention, one CTA per (sequence, kv head).  Returns ``out``."""
+    B, hq, d, nb, hkv, bs, out = _decode_common(q, k_cache, block_tables, out)
+    st = lib.pa_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens), B, hq, hkv, d,
+                       bs, block_tables.shape[1], nb, float(scale), float(softcap), int(window), _ptr(out),
+                       _dtype_code(q), KERNELS[kernel], _stream(stream))
+    _check(st, "pa_decode")
+    return out
+
+
+def decode_splitk_partition(batch: int, num_kv_heads: int, max_context_len: int, partition_tokens: int = 0) -> int:
+    return lib.pa_decode_splitk_partition(batch, num_kv_heads, max_context_len, partition_tokens)
+
+
+def decode_splitk_workspace_size(batch: int, num_q_heads: int, head_dim: int, max_context_len: int,
+                                 partition_tokens: int = 0, num_kv_heads: int = 1) -> int:
+    return lib.pa_decode_splitk_workspace_size(batch, num_q_heads, head_dim, max_context_len, partition_tokens,
+                                               num_kv_heads)
+
+
+def decode_splitk(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_tables: torch.Tensor,
+                  context_lens: torch.Tensor, scale: float, softcap: float = 0.0, window: int = 0, *,
+                  max_context_len: int, partition_tokens: int = 0, out: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None, kernel: str = "auto", stream=None) -> torch.Tensor:
+    """Split-K (flash-decoding) paged decode with the log-sum-exp combine.
+
+    ``max_context_len`` is a host-side bound on every ``context_lens[b]``.  The
+    workspace (any dtype, device memory) is allocated with torch if not given.
+    """
+    B, hq, d, nb, hkv, bs, out = _decode_common(q, k_cache, block_tables, out)
+    need = decode_splitk_workspace_size(B, hq, d, max_context_len, partition_tokens, hkv)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    wbytes = workspace.numel() * workspace.element_size()
+    st = lib.pa_decode_splitk(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens), B, hq,
+                              hkv, d, bs, block_tables.shape[1], nb, float(scale), float(softcap), int(window),
+                              _ptr(out), _dtype_code(q), int(partition_tokens), int(max_context_len),
+                              _ptr(workspace), wbytes, KERNELS[kernel], _stream(stream))
+    _check(st, "pa_decode_splitk")
+    return out
+
+
+def device_errors(clear: bool = True) -> int:
+    """OR of the PA_DEVERR_* bits raised on the current device (synchronises)."""
+    bits = ctypes.c_uint32(0)
+    _check(lib.pa_device_errors(ctypes.byref(bits), 1 if clear else 0), "pa_device_errors")
+    return bits.value
+
+
+def last_launch_count() -> int:
+    return lib.pa_last_launch_count()

@@ -1,0 +1,378 @@
+// C ABI of the paged KV cache library: host-side argument checks, tensor-map
+// set-up, kernel selection and launches.  See include/pagedattn.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/pagedattn.h"
+#include "combine_and_append.cuh"
+#include "decode_common.cuh"
+#include "decode_mma.cuh"
+#include "decode_simt.cuh"
+
+namespace {
+
+using pa::DecodeParams;
+
+thread_local int32_t t_last_launches = 0;
+
+constexpr int kNoSplitPartition = 1 << 30;
+constexpr int kMaxPartsPerSeq = 8192;
+constexpr int kMaxGridYZ = 65535;
+// Split-K auto partition: aim for at least this many (partition, kv head,
+// sequence) work units, i.e. several resident CTAs for each of B200's 148 SMs.
+constexpr long long kTargetWorkUnits = 8LL * 148;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+int ilog2(int x) {
+  int r = 0;
+  while ((1 << r) < x) ++r;
+  return r;
+}
+
+// ---- tensor maps ---------------------------------------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool tensor_map_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode != nullptr;
+}
+
+// The cache viewed as a 2-D bf16 tensor [rows = num_blocks*Hkv*bs][head_dim];
+// a box is 64 columns (128 B) x 16 rows, landed with 128-byte swizzle.
+bool encode_cache_map(CUtensorMap* map, const void* base, int head_dim, long long rows) {
+  cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)pa::kSliceTokens};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ---- argument checks -------------------------------------------------------------
+
+struct Shape {
+  int batch, hq, hkv, d, bs, max_blocks, num_blocks;
+};
+
+pa_status_t check_decode_args(const void* q, const void* kc, const void* vc, const int32_t* bt, const int32_t* cl,
+                              const Shape& s, float softcap, const void* out, pa_dtype_t dt, pa_kernel_t kernel) {
+  if (s.batch < 0 || s.hq <= 0 || s.hkv <= 0 || s.d <= 0 || s.bs <= 0 || s.max_blocks <= 0 || s.num_blocks <= 0)
+    return PA_ERR_INVALID;
+  if (s.hq % s.hkv != 0) return PA_ERR_INVALID;
+  if (dt != PA_F32 && dt != PA_BF16) return PA_ERR_INVALID;
+  if (kernel != PA_KERNEL_AUTO && kernel != PA_KERNEL_CUDA_CORE && kernel != PA_KERNEL_MMA) return PA_ERR_INVALID;
+  if (std::isnan(softcap)) return PA_ERR_INVALID;
+  if (s.batch > 0) {
+    if (!q || !kc || !vc || !bt || !cl || !out) return PA_ERR_INVALID;
+    if (!aligned(q, 16) || !aligned(kc, 16) || !aligned(vc, 16) || !aligned(out, 16) || !aligned(bt, 4) ||
+        !aligned(cl, 4))
+      return PA_ERR_INVALID;
+  }
+  if (s.d != 64 && s.d != 128 && s.d != 256) return PA_ERR_UNSUPPORTED;
+  if (!pow2(s.bs) || s.bs < 16 || s.bs > 256) return PA_ERR_UNSUPPORTED;
+  if (s.hq / s.hkv > pa::kMaxGroup) return PA_ERR_UNSUPPORTED;
+  if (s.batch > kMaxGridYZ || s.hkv > kMaxGridYZ) return PA_ERR_UNSUPPORTED;
+  if ((long long)s.num_blocks * s.hkv * s.bs >= (1LL << 31)) return PA_ERR_UNSUPPORTED;
+  if ((long long)s.max_blocks * s.bs >= (1LL << 30)) return PA_ERR_UNSUPPORTED;
+  if (kernel == PA_KERNEL_MMA && dt != PA_BF16) return PA_ERR_UNSUPPORTED;
+  return PA_OK;
+}
+
+DecodeParams make_params(const void* q, const void* kc, const void* vc, const int32_t* bt, const int32_t* cl,
+                         const Shape& s, float scale, float softcap, int32_t window, void* out) {
+  DecodeParams p{};
+  p.q = q;
+  p.out = out;
+  p.k_cache = kc;
+  p.v_cache = vc;
+  p.block_tables = bt;
+  p.context_lens = cl;
+  p.batch = s.batch;
+  p.hq = s.hq;
+  p.hkv = s.hkv;
+  p.group = s.hq / s.hkv;
+  p.head_dim = s.d;
+  p.block_size = s.bs;
+  p.log2_bs = ilog2(s.bs);
+  p.max_blocks = s.max_blocks;
+  p.num_blocks = s.num_blocks;
+  p.window = window;
+  p.partition = kNoSplitPartition;
+  p.max_parts = 1;
+  p.max_context = s.max_blocks * s.bs;
+  p.scale = scale;
+  p.use_softcap = (softcap > 0.f && std::isfinite(softcap)) ? 1 : 0;
+  p.softcap = p.use_softcap ? softcap : 0.f;
+  p.inv_softcap = p.use_softcap ? 1.f / softcap : 0.f;
+  return p;
+}
+
+// ---- launches ---------------------------------------------------------------------
+
+// Opt a kernel in to more than 48 KB of dynamic shared memory, once per device
+// (the flag word is per kernel instantiation: one bit per device ordinal < 64).
+template <typename Kernel>
+cudaError_t set_smem(Kernel k, int bytes, std::atomic<uint64_t>& done) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
+template <int D, int NW, int ST, bool SPLIT>
+cudaError_t launch_mma_t(const DecodeParams& p, dim3 grid, cudaStream_t st) {
+  using Cfg = pa::MmaCfg<D, NW, ST>;
+  CUtensorMap kmap, vmap;
+  const long long rows = (long long)p.num_blocks * p.hkv * p.block_size;
+  if (!tensor_map_encoder()) return cudaErrorNotSupported;
+  if (!encode_cache_map(&kmap, p.k_cache, D, rows) || !encode_cache_map(&vmap, p.v_cache, D, rows))
+    return cudaErrorInvalidValue;
+  auto kern = pa::decode_mma_kernel<D, NW, ST, SPLIT>;
+  static std::atomic<uint64_t> smem_done{0};
+  cudaError_t e = set_smem(kern, Cfg::kSmemBytes, smem_done);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, NW * 32, Cfg::kSmemBytes, st>>>(kmap, vmap, p);
+  return cudaGetLastError();
+}
+
+template <bool SPLIT>
+cudaError_t launch_mma(const DecodeParams& p, dim3 grid, cudaStream_t st) {
+  switch (p.head_dim) {
+    case 64:
+      return launch_mma_t<64, 4, 4, SPLIT>(p, grid, st);
+    case 128:
+      return launch_mma_t<128, 4, 3, SPLIT>(p, grid, st);
+    default:
+      return launch_mma_t<256, 2, 3, SPLIT>(p, grid, st);
+  }
+}
+
+template <typename T, int D, int GP, bool SPLIT>
+cudaError_t launch_simt_t(const DecodeParams& p, dim3 grid, cudaStream_t st) {
+  constexpr int NW = 4;
+  const int smem = pa::merge_smem_bytes<NW>(D);
+  auto kern = pa::decode_simt_kernel<T, D, GP, NW, SPLIT>;
+  static std::atomic<uint64_t> smem_done{0};
+  cudaError_t e = set_smem(kern, smem, smem_done);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, NW * 32, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <typename T, int D, bool SPLIT>
+cudaError_t launch_simt_d(const DecodeParams& p, dim3 grid, cudaStream_t st) {
+  const int G = p.group;
+  if (G <= 1) return launch_simt_t<T, D, 1, SPLIT>(p, grid, st);
+  if (G <= 2) return launch_simt_t<T, D, 2, SPLIT>(p, grid, st);
+  if (G <= 4) return launch_simt_t<T, D, 4, SPLIT>(p, grid, st);
+  return launch_simt_t<T, D, 8, SPLIT>(p, grid, st);
+}
+
+template <typename T, bool SPLIT>
+cudaError_t launch_simt(const DecodeParams& p, dim3 grid, cudaStream_t st) {
+  switch (p.head_dim) {
+    case 64:
+      return launch_simt_d<T, 64, SPLIT>(p, grid, st);
+    case 128:
+      return launch_simt_d<T, 128, SPLIT>(p, grid, st);
+    default:
+      return launch_simt_d<T, 256, SPLIT>(p, grid, st);
+  }
+}
+
+template <bool SPLIT>
+cudaError_t launch_decode(const DecodeParams& p, pa_dtype_t dt, pa_kernel_t kernel, dim3 grid, cudaStream_t st) {
+  const bool use_mma = (kernel == PA_KERNEL_MMA) || (kernel == PA_KERNEL_AUTO && dt == PA_BF16);
+  if (use_mma) return launch_mma<SPLIT>(p, grid, st);
+  if (dt == PA_BF16) return launch_simt<__nv_bfloat16, SPLIT>(p, grid, st);
+  return launch_simt<float, SPLIT>(p, grid, st);
+}
+
+template <typename OutT>
+cudaError_t launch_combine(const DecodeParams& p, cudaStream_t st) {
+  const int smem = (((p.max_parts + 3) & ~3) + pa::kCombineWarps * p.head_dim) * 4;
+  dim3 grid(p.hq, p.batch);
+  switch (p.head_dim) {
+    case 64:
+      pa::combine_kernel<OutT, 64><<<grid, pa::kCombineWarps * 32, smem, st>>>(p);
+      break;
+    case 128:
+      pa::combine_kernel<OutT, 128><<<grid, pa::kCombineWarps * 32, smem, st>>>(p);
+      break;
+    default:
+      pa::combine_kernel<OutT, 256><<<grid, pa::kCombineWarps * 32, smem, st>>>(p);
+      break;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status_t pa_write_kv(const void* k, const void* v, const int64_t* slot_mapping, int32_t num_tokens,
+                        void* k_cache, void* v_cache, int32_t num_blocks, int32_t block_size,
+                        int32_t num_kv_heads, int32_t head_dim, pa_dtype_t dtype, pa_stream_t stream) {
+  t_last_launches = 0;
+  if (num_tokens < 0 || num_blocks <= 0 || block_size <= 0 || num_kv_heads <= 0 || head_dim <= 0)
+    return PA_ERR_INVALID;
+  if (dtype != PA_F32 && dtype != PA_BF16) return PA_ERR_INVALID;
+  const int elt = dtype == PA_F32 ? 4 : 2;
+  if ((head_dim * elt) % 16 != 0) return PA_ERR_UNSUPPORTED;
+  if (num_tokens == 0) return PA_OK;
+  if (!k || !v || !slot_mapping || !k_cache || !v_cache) return PA_ERR_INVALID;
+  if (!aligned(k, 16) || !aligned(v, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(slot_mapping, 8))
+    return PA_ERR_INVALID;
+  const int chunks = head_dim * elt / 16;
+  const long long total = (long long)num_tokens * num_kv_heads * chunks;
+  const long long blocks = (total + 255) / 256;
+  if (blocks > INT_MAX) return PA_ERR_UNSUPPORTED;
+  pa::write_kv_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
+      static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping, num_tokens,
+      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), (int64_t)num_blocks * block_size, block_size,
+      num_kv_heads, chunks);
+  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  t_last_launches = 1;
+  return PA_OK;
+}
+
+pa_status_t pa_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                      const int32_t* context_lens, int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                      int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq, int32_t num_blocks,
+                      float scale, float softcap, int32_t window, void* out, pa_dtype_t dtype,
+                      pa_kernel_t kernel, pa_stream_t stream) {
+  t_last_launches = 0;
+  const Shape s{batch, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks};
+  pa_status_t st = check_decode_args(q, k_cache, v_cache, block_tables, context_lens, s, softcap, out, dtype, kernel);
+  if (st != PA_OK) return st;
+  if (batch == 0) return PA_OK;
+  DecodeParams p = make_params(q, k_cache, v_cache, block_tables, context_lens, s, scale, softcap, window, out);
+  dim3 grid(1, num_kv_heads, batch);
+  if (launch_decode<false>(p, dtype, kernel, grid, stream) != cudaSuccess) return PA_ERR_CUDA;
+  t_last_launches = 1;
+  return PA_OK;
+}
+
+int32_t pa_decode_splitk_partition(int32_t batch, int32_t num_kv_heads, int32_t max_context_len,
+                                   int32_t partition_tokens) {
+  if (partition_tokens > 0) return partition_tokens;
+  const long long work = (long long)(batch > 0 ? batch : 1) * (num_kv_heads > 0 ? num_kv_heads : 1) *
+                         (max_context_len > 0 ? max_context_len : 1);
+  int P = 512;
+  while (P > 64 && work / P < kTargetWorkUnits) P >>= 1;
+  return P;
+}
+
+static long long splitk_parts(int32_t max_context_len, int32_t P) {
+  return ((long long)(max_context_len > 0 ? max_context_len : 1) + P - 1) / P;
+}
+
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+size_t pa_decode_splitk_workspace_size(int32_t batch, int32_t num_q_heads, int32_t head_dim,
+                                       int32_t max_context_len, int32_t partition_tokens,
+                                       int32_t num_kv_heads) {
+  if (batch <= 0 || num_q_heads <= 0 || head_dim <= 0) return 0;
+  const int P = pa_decode_splitk_partition(batch, num_kv_heads, max_context_len, partition_tokens);
+  if (P <= 0) return 0;
+  const size_t rows = (size_t)batch * num_q_heads * (size_t)splitk_parts(max_context_len, P);
+  return align256(rows * head_dim * 4) + align256(rows * 2 * 4);
+}
+
+pa_status_t pa_decode_splitk(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                             const int32_t* context_lens, int32_t batch, int32_t num_q_heads,
+                             int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                             int32_t max_blocks_per_seq, int32_t num_blocks, float scale, float softcap,
+                             int32_t window, void* out, pa_dtype_t dtype, int32_t partition_tokens,
+                             int32_t max_context_len, void* workspace, size_t workspace_bytes,
+                             pa_kernel_t kernel, pa_stream_t stream) {
+  t_last_launches = 0;
+  const Shape s{batch, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks};
+  pa_status_t st = check_decode_args(q, k_cache, v_cache, block_tables, context_lens, s, softcap, out, dtype, kernel);
+  if (st != PA_OK) return st;
+  if (partition_tokens < 0 || (partition_tokens > 0 && partition_tokens % 64 != 0)) return PA_ERR_INVALID;
+  if (max_context_len <= 0) return PA_ERR_INVALID;
+  if (batch == 0) return PA_OK;
+  const int P = pa_decode_splitk_partition(batch, num_kv_heads, max_context_len, partition_tokens);
+  const long long parts = splitk_parts(max_context_len, P);
+  if (parts > kMaxPartsPerSeq) return PA_ERR_UNSUPPORTED;
+  const size_t need = pa_decode_splitk_workspace_size(batch, num_q_heads, head_dim, max_context_len, P, num_kv_heads);
+  if (!workspace || !aligned(workspace, 16) || workspace_bytes < need) return PA_ERR_WORKSPACE;
+
+  DecodeParams p = make_params(q, k_cache, v_cache, block_tables, context_lens, s, scale, softcap, window, out);
+  p.partition = P;
+  p.max_parts = (int)parts;
+  p.max_context = max_context_len < p.max_context ? max_context_len : p.max_context;
+  const size_t rows = (size_t)batch * num_q_heads * parts;
+  p.ws_o = static_cast<float*>(workspace);
+  p.ws_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(rows * head_dim * 4));
+
+  dim3 grid((unsigned)parts, num_kv_heads, batch);
+  if (launch_decode<true>(p, dtype, kernel, grid, stream) != cudaSuccess) return PA_ERR_CUDA;
+  if (parts > 1) {
+    cudaError_t e = dtype == PA_BF16 ? launch_combine<__nv_bfloat16>(p, stream) : launch_combine<float>(p, stream);
+    if (e != cudaSuccess) return PA_ERR_CUDA;
+    t_last_launches = 2;
+  } else {
+    t_last_launches = 1;
+  }
+  return PA_OK;
+}
+
+pa_status_t pa_device_errors(uint32_t* bits, int32_t clear) {
+  if (!bits) return PA_ERR_INVALID;
+  unsigned int v = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return PA_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&v, pa::g_device_errors, sizeof v) != cudaSuccess) return PA_ERR_CUDA;
+  *bits = v;
+  if (clear) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(pa::g_device_errors, &zero, sizeof zero) != cudaSuccess) return PA_ERR_CUDA;
+  }
+  return PA_OK;
+}
+
+const char* pa_error_string(pa_status_t status) {
+  switch (status) {
+    case PA_OK:
+      return "ok";
+    case PA_ERR_INVALID:
+      return "invalid argument (null or misaligned pointer, or a bad size)";
+    case PA_ERR_UNSUPPORTED:
+      return "unsupported shape or dtype (head_dim, block_size, group size, or pool too large)";
+    case PA_ERR_WORKSPACE:
+      return "split-K workspace missing, misaligned or too small";
+    case PA_ERR_CUDA:
+      return "CUDA runtime error or failed launch";
+  }
+  return "unknown status";
+}
+
+int32_t pa_last_launch_count(void) { return t_last_launches; }
+
+}  // extern "C"

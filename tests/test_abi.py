@@ -1,0 +1,139 @@
+"""The C ABI on a machine without a GPU: the library loads, exports every
+function the header declares, and its host-side checks reject bad arguments
+before anything touches the device."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import paged_kv_cache_473_b200 as pa
+from paged_kv_cache_473_b200 import _binding as bnd
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "pagedattn.h")
+
+# 16-byte aligned fake device addresses: never dereferenced, because every call
+# below fails its host checks first.
+A = 0x10000
+MIS = 0x10004
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ["pa_write_kv", "pa_decode", "pa_decode_splitk", "pa_decode_splitk_workspace_size",
+              "pa_decode_splitk_partition", "pa_device_errors", "pa_error_string", "pa_last_launch_count"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(bnd._build.LIB)
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+
+
+def test_error_strings():
+    for s in range(5):
+        assert pa.error_string(s)
+    assert pa.error_string(99) == "unknown status"
+
+
+def _decode(**kw):
+    a = dict(q=A, k=A, v=A, bt=A, cl=A, B=2, hq=8, hkv=2, d=128, bs=16, mb=4, nb=8, scale=0.1, cap=0.0, win=0,
+             out=A, dt=bnd.PA_BF16, kern=0)
+    a.update(kw)
+    return bnd.lib.pa_decode(a["q"], a["k"], a["v"], a["bt"], a["cl"], a["B"], a["hq"], a["hkv"], a["d"], a["bs"],
+                             a["mb"], a["nb"], a["scale"], a["cap"], a["win"], a["out"], a["dt"], a["kern"], None)
+
+
+@pytest.mark.parametrize(
+    "kw,status",
+    [
+        (dict(q=None), bnd.PA_ERR_INVALID),
+        (dict(out=None), bnd.PA_ERR_INVALID),
+        (dict(q=MIS), bnd.PA_ERR_INVALID),
+        (dict(k=MIS), bnd.PA_ERR_INVALID),
+        (dict(bt=A + 2), bnd.PA_ERR_INVALID),
+        (dict(hq=6, hkv=4), bnd.PA_ERR_INVALID),
+        (dict(hkv=0), bnd.PA_ERR_INVALID),
+        (dict(B=-1), bnd.PA_ERR_INVALID),
+        (dict(dt=7), bnd.PA_ERR_INVALID),
+        (dict(kern=9), bnd.PA_ERR_INVALID),
+        (dict(cap=float("nan")), bnd.PA_ERR_INVALID),
+        (dict(d=96), bnd.PA_ERR_UNSUPPORTED),
+        (dict(bs=8), bnd.PA_ERR_UNSUPPORTED),
+        (dict(bs=48), bnd.PA_ERR_UNSUPPORTED),
+        (dict(hq=32, hkv=2), bnd.PA_ERR_UNSUPPORTED),
+        (dict(B=70000), bnd.PA_ERR_UNSUPPORTED),
+        (dict(nb=1 << 26, hkv=8, hq=8, bs=16), bnd.PA_ERR_UNSUPPORTED),
+        (dict(dt=bnd.PA_F32, kern=2), bnd.PA_ERR_UNSUPPORTED),
+    ],
+)
+def test_decode_host_checks(kw, status):
+    assert _decode(**kw) == status
+    assert pa.last_launch_count() == 0
+
+
+def test_empty_batch_is_a_no_op():
+    assert _decode(B=0, q=None, out=None) == bnd.PA_OK
+    assert pa.last_launch_count() == 0
+
+
+def _splitk(**kw):
+    a = dict(q=A, k=A, v=A, bt=A, cl=A, B=2, hq=8, hkv=2, d=128, bs=16, mb=4, nb=8, scale=0.1, cap=0.0, win=0,
+             out=A, dt=bnd.PA_BF16, P=64, maxL=64, ws=A, wsb=1 << 30, kern=0)
+    a.update(kw)
+    return bnd.lib.pa_decode_splitk(a["q"], a["k"], a["v"], a["bt"], a["cl"], a["B"], a["hq"], a["hkv"], a["d"],
+                                    a["bs"], a["mb"], a["nb"], a["scale"], a["cap"], a["win"], a["out"], a["dt"],
+                                    a["P"], a["maxL"], a["ws"], a["wsb"], a["kern"], None)
+
+
+@pytest.mark.parametrize(
+    "kw,status",
+    [
+        (dict(P=100), bnd.PA_ERR_INVALID),
+        (dict(P=-64), bnd.PA_ERR_INVALID),
+        (dict(maxL=0), bnd.PA_ERR_INVALID),
+        (dict(ws=None), bnd.PA_ERR_WORKSPACE),
+        (dict(ws=MIS), bnd.PA_ERR_WORKSPACE),
+        (dict(wsb=100), bnd.PA_ERR_WORKSPACE),
+        (dict(P=64, maxL=64 * 8193), bnd.PA_ERR_UNSUPPORTED),
+        (dict(d=32), bnd.PA_ERR_UNSUPPORTED),
+    ],
+)
+def test_splitk_host_checks(kw, status):
+    assert _splitk(**kw) == status
+
+
+def test_workspace_size_formula():
+    B, hq, d, maxL, P = 8, 32, 128, 131072, 512
+    parts = -(-maxL // P)
+    rows = B * hq * parts
+    al = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    assert pa.decode_splitk_workspace_size(B, hq, d, maxL, P, 8) == al(rows * d * 4) + al(rows * 2 * 4)
+    assert pa.decode_splitk_workspace_size(0, hq, d, maxL, P, 8) == 0
+
+
+def test_auto_partition_heuristic():
+    # Explicit sizes pass through; auto picks 512 unless that leaves fewer than
+    # 8 * 148 work units, halving down to 64.
+    assert pa.decode_splitk_partition(8, 8, 131072, 1024) == 1024
+    assert pa.decode_splitk_partition(8, 8, 131072, 0) == 512
+    assert pa.decode_splitk_partition(128, 8, 8192, 0) == 512
+    assert pa.decode_splitk_partition(64, 4, 2048, 0) == 256
+    assert pa.decode_splitk_partition(4, 2, 100, 0) == 64
+
+
+def test_write_kv_host_checks():
+    f = bnd.lib.pa_write_kv
+    assert f(None, A, A, 4, A, A, 8, 16, 2, 64, bnd.PA_BF16, None) == bnd.PA_ERR_INVALID
+    assert f(A, A, A + 4, 4, A, A, 8, 16, 2, 64, bnd.PA_BF16, None) == bnd.PA_ERR_INVALID
+    assert f(A, A, A, -1, A, A, 8, 16, 2, 64, bnd.PA_BF16, None) == bnd.PA_ERR_INVALID
+    assert f(A, A, A, 4, A, A, 8, 16, 2, 4, bnd.PA_BF16, None) == bnd.PA_ERR_UNSUPPORTED
+    assert f(A, A, A, 0, A, A, 8, 16, 2, 64, bnd.PA_BF16, None) == bnd.PA_OK

@@ -1,0 +1,286 @@
+"""GPU parity: the CUDA path, called through the C ABI, against the CPU oracle
+on the same seeded inputs.
+
+Append: bit-exact.  Decode: within max-abs / mean-abs 2e-2 / 2e-3 (bf16 inputs,
+fp32 accumulation) or 1e-4 / 1e-5 (fp32), of the fp64 oracle.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_473_b200 as pa
+from paged_kv_cache_473_b200 import workloads as wl
+from tests.gpu_helpers import TOL, assert_close, bits, errors, gpu_step, oracle_step, to_dev
+from tests.paging_helpers import scatter_to_pool
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # collected on CPU machines, never run there
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+# Sizes the oracle finishes in seconds that still span many 16-token slices,
+# several partitions and ragged tails.
+REDUCED = {
+    "tiny_fp32": dict(),
+    "tinyllama_1b": dict(batch=8),
+    "gemma2_2b": dict(batch=12),
+    "llama3_8b": dict(batch=16, max_len=3000),
+    "long_splitk": dict(lengths=[16384 + 37, 19999, 1, 1000]),
+}
+
+
+@pytest.fixture(autouse=True)
+def _clear_device_errors():
+    pa.device_errors(clear=True)
+    yield
+
+
+def _reduced(name, **extra):
+    w = wl.WORKLOADS[name]
+    kw = dict(REDUCED[name])
+    kw.update(extra)
+    b_cpu = wl.make_batch(w, **kw)
+    return w, b_cpu, to_dev(b_cpu)
+
+
+@pytest.mark.parametrize("name", list(wl.WORKLOADS))
+def test_write_kv_is_bit_exact(name):
+    w, b_cpu, b = _reduced(name)
+    _, kc, vc = gpu_step(b)
+    _, kc_ref, vc_ref = oracle_step(b_cpu)
+    assert torch.equal(bits(kc), bits(kc_ref))
+    assert torch.equal(bits(vc), bits(vc_ref))
+    assert pa.device_errors() == 0
+
+
+def test_write_kv_skips_padding_and_flags_bad_slots():
+    w = wl.WORKLOADS["tinyllama_1b"]
+    b_cpu = wl.make_batch(w, batch=4, max_len=300)
+    b = to_dev(b_cpu)
+    slots = b.slot_mapping.clone()
+    slots[1] = -1
+    kc, vc = b.k_cache.clone(), b.v_cache.clone()
+    pa.write_kv(b.k_new, b.v_new, slots, kc, vc)
+    kc_ref, vc_ref = b_cpu.k_cache.clone(), b_cpu.v_cache.clone()
+    oracle.write_kv(b_cpu.k_new, b_cpu.v_new, slots.cpu(), kc_ref, vc_ref)
+    assert torch.equal(bits(kc), bits(kc_ref)) and torch.equal(bits(vc), bits(vc_ref))
+    assert pa.device_errors() == 0
+    slots[2] = b.num_blocks * w.block_size  # one past the pool: skipped and reported
+    kc2 = b.k_cache.clone()
+    vc2 = b.v_cache.clone()
+    pa.write_kv(b.k_new, b.v_new, slots, kc2, vc2)
+    assert pa.device_errors() & pa.DEVERR_SLOT
+
+
+@pytest.mark.parametrize("name", list(wl.WORKLOADS))
+@pytest.mark.parametrize("split", [False, True])
+@pytest.mark.parametrize("kernel", ["auto", "cuda_core"])
+def test_step_parity(name, split, kernel):
+    w, b_cpu, b = _reduced(name)
+    out, _, _ = gpu_step(b, kernel=kernel, split=split, partition=w.partition_tokens)
+    ref, _, _ = oracle_step(b_cpu)
+    assert_close(out, ref, w.torch_dtype, f"{name} split={split} kernel={kernel}")
+    assert pa.device_errors() == 0
+
+
+@pytest.mark.parametrize("window", [4096, 1, 64, 200, 300, 511])
+@pytest.mark.parametrize("split", [False, True])
+def test_gemma_softcap_and_sliding_window(window, split):
+    w, b_cpu, b = _reduced("gemma2_2b")
+    out, _, _ = gpu_step(b, split=split, partition=128, window=window)
+    ref, _, _ = oracle_step(b_cpu, window=window)
+    assert_close(out, ref, w.torch_dtype, f"window={window}")
+
+
+@pytest.mark.parametrize("partition", [64, 256, 512, 1024])
+def test_splitk_is_invariant_to_partition_size(partition):
+    w, b_cpu, b = _reduced("long_splitk")
+    out, _, _ = gpu_step(b, split=True, partition=partition)
+    ref, _, _ = oracle_step(b_cpu)
+    assert_close(out, ref, w.torch_dtype, f"partition={partition}")
+
+
+@pytest.mark.parametrize("kernel", ["auto", "cuda_core"])
+def test_one_partition_splitk_is_bit_identical_to_decode(kernel):
+    w, b_cpu, b = _reduced("tinyllama_1b")
+    a, _, _ = gpu_step(b, kernel=kernel)
+    s, _, _ = gpu_step(b, kernel=kernel, split=True, partition=2048)
+    assert torch.equal(bits(a), bits(s))
+
+
+@pytest.mark.parametrize("kernel", ["auto", "cuda_core"])
+@pytest.mark.parametrize("split", [False, True])
+def test_block_permutation_invariance_is_bit_exact(kernel, split):
+    w, b_cpu, b = _reduced("llama3_8b")
+    base, kc, vc = gpu_step(b, kernel=kernel, split=split, partition=256)
+    nb = kc.shape[0]
+    perm = torch.randperm(nb, generator=torch.Generator().manual_seed(5)).cuda()
+    kc2, vc2 = torch.empty_like(kc), torch.empty_like(vc)
+    kc2[perm] = kc
+    vc2[perm] = vc
+    t2 = b.block_tables.clone()
+    m = t2 >= 0
+    t2[m] = perm[t2[m].long()].to(torch.int32)
+    if split:
+        out = pa.decode_splitk(b.q, kc2, vc2, t2, b.context_lens, w.scale, max_context_len=b.max_context_len,
+                               partition_tokens=256, kernel=kernel)
+    else:
+        out = pa.decode(b.q, kc2, vc2, t2, b.context_lens, w.scale, kernel=kernel)
+    torch.cuda.synchronize()
+    assert torch.equal(bits(out), bits(base))
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_context_of_length_one_returns_v_exactly(dtype, d):
+    gen = torch.Generator().manual_seed(d)
+    hkv, hq, B = 2, 8, 5
+    ks = [torch.randn((1, hkv, d), generator=gen).to(dtype) for _ in range(B)]
+    vs = [torch.randn((1, hkv, d), generator=gen).to(dtype) for _ in range(B)]
+    kc, vc, tables, cl = scatter_to_pool(ks, vs, 16, gen, dtype=dtype)
+    q = (torch.randn((B, hq, d), generator=gen) * 30).to(dtype)
+    kern = "auto"
+    out = pa.decode(q.cuda(), kc.cuda(), vc.cuda(), tables.cuda(), cl.cuda(), 1 / math.sqrt(d), 10.0, 0, kernel=kern)
+    torch.cuda.synchronize()
+    for i in range(B):
+        for h in range(hq):
+            assert torch.equal(bits(out[i, h]), bits(vs[i][0, h // 4]))
+
+
+def test_zero_length_context_gives_zero_rows():
+    w, b_cpu, b = _reduced("tinyllama_1b")
+    cl = b.context_lens.clone()
+    cl[3] = 0
+    for split in (False, True):
+        if split:
+            out = pa.decode_splitk(b.q, b.k_cache, b.v_cache, b.block_tables, cl, w.scale,
+                                   max_context_len=b.max_context_len, partition_tokens=64)
+        else:
+            out = pa.decode(b.q, b.k_cache, b.v_cache, b.block_tables, cl, w.scale)
+        torch.cuda.synchronize()
+        assert torch.count_nonzero(out[3]).item() == 0
+        assert torch.isfinite(out.float()).all()
+
+
+def test_infinite_softcap_is_bit_identical_to_no_softcap():
+    w, b_cpu, b = _reduced("gemma2_2b")
+    a, _, _ = gpu_step(b, softcap=0.0)
+    c, _, _ = gpu_step(b, softcap=float("inf"))
+    assert torch.equal(bits(a), bits(c))
+    ref, _, _ = oracle_step(b_cpu, softcap=0.0)
+    assert_close(a, ref, torch.bfloat16, "no softcap")
+
+
+@pytest.mark.parametrize("split", [False, True])
+def test_window_edges(split):
+    """W = L-1, L, L+1 around one sequence's length, and W >= L equal to no window."""
+    w, b_cpu, b = _reduced("tinyllama_1b")
+    L0 = int(b_cpu.context_lens[0])
+    base, _, _ = gpu_step(b, split=split, partition=64, window=0)
+    for W in (L0 - 1, L0, L0 + 1, 1):
+        out, _, _ = gpu_step(b, split=split, partition=64, window=W)
+        ref, _, _ = oracle_step(b_cpu, window=W)
+        assert_close(out, ref, torch.bfloat16, f"W={W}")
+    big, _, _ = gpu_step(b, split=split, partition=64, window=1 << 20)
+    assert torch.equal(bits(big), bits(base))
+
+
+def test_identical_keys_give_mean_of_v():
+    gen = torch.Generator().manual_seed(8)
+    L, hkv, d = 700, 4, 128
+    key = torch.randn((1, hkv, d), generator=gen)
+    ks = [key.expand(L, hkv, d).clone().to(torch.bfloat16)]
+    vs = [torch.randn((L, hkv, d), generator=gen).to(torch.bfloat16)]
+    kc, vc, tables, cl = scatter_to_pool(ks, vs, 16, gen, dtype=torch.bfloat16)
+    q = torch.randn((1, 16, d), generator=gen).to(torch.bfloat16)
+    out = pa.decode(q.cuda(), kc.cuda(), vc.cuda(), tables.cuda(), cl.cuda(), 0.09)
+    torch.cuda.synchronize()
+    for h in range(16):
+        mean = vs[0][:, h // 4].double().mean(0).numpy()
+        mx, _ = errors(out[0, h], mean)
+        assert mx <= 2e-2
+
+
+@pytest.mark.parametrize("hq,hkv", [(4, 4), (6, 2), (24, 3), (8, 1), (16, 2)])
+@pytest.mark.parametrize("kernel", ["auto", "cuda_core"])
+def test_group_sizes(hq, hkv, kernel):
+    w = wl.WORKLOADS["llama3_8b"].replace(num_q_heads=hq, num_kv_heads=hkv, prefix_share=0.0)
+    b_cpu = wl.make_batch(w, batch=6, max_len=900)
+    b = to_dev(b_cpu)
+    out, _, _ = gpu_step(b, kernel=kernel)
+    ref, _, _ = oracle_step(b_cpu)
+    assert_close(out, ref, torch.bfloat16, f"G={hq // hkv}")
+
+
+@pytest.mark.parametrize("bs,d", [(16, 256), (32, 64), (64, 128), (256, 256), (256, 64)])
+def test_block_sizes_and_head_dims(bs, d):
+    w = wl.WORKLOADS["gemma2_2b"].replace(block_size=bs, head_dim=d)
+    b_cpu = wl.make_batch(w, batch=5)
+    b = to_dev(b_cpu)
+    for split in (False, True):
+        out, _, _ = gpu_step(b, split=split, partition=256)
+        ref, _, _ = oracle_step(b_cpu)
+        assert_close(out, ref, torch.bfloat16, f"bs={bs} d={d} split={split}")
+
+
+def test_large_scores_stay_finite():
+    w = wl.WORKLOADS["llama3_8b"]
+    b_cpu = wl.make_batch(w, batch=6, max_len=1500, q_scale=100.0)
+    b = to_dev(b_cpu)
+    for split in (False, True):
+        out, _, _ = gpu_step(b, split=split, partition=128)
+        ref, _, _ = oracle_step(b_cpu)
+        assert_close(out, ref, torch.bfloat16, f"q x100 split={split}")
+
+
+def test_bad_block_id_and_long_context_are_reported_not_faulted():
+    w, b_cpu, b = _reduced("tinyllama_1b")
+    t = b.block_tables.clone()
+    t[0, 0] = b.num_blocks + 5  # outside the pool: the tile is skipped
+    pa.decode(b.q, b.k_cache, b.v_cache, t, b.context_lens, w.scale)
+    assert pa.device_errors() & pa.DEVERR_BLOCK
+    cl = b.context_lens.clone()
+    cl[1] = b.max_blocks_per_seq * w.block_size + 1  # longer than the table: clamped
+    pa.decode(b.q, b.k_cache, b.v_cache, b.block_tables, cl, w.scale)
+    assert pa.device_errors() & pa.DEVERR_CONTEXT
+    cl = b.context_lens.clone()
+    pa.decode_splitk(b.q, b.k_cache, b.v_cache, b.block_tables, cl, w.scale,
+                     max_context_len=int(cl.max().item()) - 1, partition_tokens=64)
+    assert pa.device_errors() & pa.DEVERR_CONTEXT
+    # The context stays usable.
+    out, _, _ = gpu_step(b)
+    ref, _, _ = oracle_step(b_cpu)
+    assert_close(out, ref, torch.bfloat16, "after errors")
+    assert pa.device_errors() == 0
+
+
+# ---- full sizes, bench launch configuration, sampled rows -----------------------
+
+FULL = ["tinyllama_1b", "gemma2_2b", "llama3_8b", "long_splitk"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_sampled_rows(name):
+    w = wl.WORKLOADS[name]
+    b = wl.make_batch(w, device="cuda")
+    cpu = dict(q=b.q.cpu(), k_new=b.k_new.cpu(), v_new=b.v_new.cpu(), slots=b.slot_mapping.cpu(),
+               kc=b.k_cache.cpu(), vc=b.v_cache.cpu(), tables=b.block_tables.cpu(), lens=b.context_lens.cpu())
+    out, _, _ = gpu_step(b, split=True, partition=w.partition_tokens)
+    assert torch.isfinite(out.float()).all()
+    assert pa.device_errors() == 0
+    oracle.write_kv(cpu["k_new"], cpu["v_new"], cpu["slots"], cpu["kc"], cpu["vc"])
+    g = torch.Generator().manual_seed(99)
+    B, hq = w.batch, w.num_q_heads
+    rows = [(int(i), int(h)) for i, h in zip(torch.randint(0, B, (48,), generator=g),
+                                             torch.randint(0, hq, (48,), generator=g))]
+    # Always include the longest and the shortest sequence.
+    L = cpu["lens"]
+    rows += [(int(L.argmax()), 0), (int(L.argmin()), hq - 1)]
+    ref = oracle.decode(cpu["q"], cpu["kc"], cpu["vc"], cpu["tables"], cpu["lens"], w.scale, w.softcap, w.window,
+                        rows=rows)
+    got = torch.stack([out[i, h] for i, h in rows])
+    assert_close(got, ref, w.torch_dtype, f"{name} full size, sampled rows")
