@@ -50,7 +50,8 @@ def parse():
     ap.add_argument("--workload", default=HEADLINE, choices=list(wl.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--kernel", default="auto", choices=["auto", "cuda_core", "mma"])
-    ap.add_argument("--no-split", action="store_true", help="time pa_decode (one CTA per sequence, kv head)")
+    ap.add_argument("--no-split", action="store_true", help="one CTA per (sequence, kv head), no split-K")
+    ap.add_argument("--unfused", action="store_true", help="separate append kernel (pa_write_kv) before the decode")
     ap.add_argument("--partition", type=int, default=-1, help="split-K partition tokens (0 auto; -1 workload's)")
     ap.add_argument("--shapes", default="auto", help="comma list of extra workloads to time, 'none', or 'auto'")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="bound on the CPU-oracle sample")
@@ -220,15 +221,21 @@ def pool_copies(pool_bytes: int, l2_bytes: int) -> int:
 
 
 class Runner:
-    """One workload on this GPU: rotating KV pools, persistent output/workspace."""
+    """One workload on this GPU: rotating KV pools, persistent output/workspace.
 
-    def __init__(self, w: wl.Workload, rank: int, kernel: str, split: bool, partition: int):
+    A step appends the batch's new key/value rows at position L-1 of every
+    sequence and runs the paged decode: fused in one call (pa_decode_step), or
+    as pa_write_kv followed by pa_decode / pa_decode_splitk (``fused=False``).
+    """
+
+    def __init__(self, w: wl.Workload, rank: int, kernel: str, split: bool, partition: int, fused: bool = True):
         import paged_kv_cache_473_b200 as pa
 
         self.pa = pa
         self.w = w
         self.kernel = kernel
         self.split = split
+        self.fused = fused
         self.batch = wl.make_batch(w, seed=rank_seed(w, rank), device="cuda")
         b = self.batch
         self.B = b.q.shape[0]
@@ -238,39 +245,52 @@ class Runner:
         self.pools = [(b.k_cache, b.v_cache)] + [(b.k_cache.clone(), b.v_cache.clone()) for _ in range(self.R - 1)]
         self.pool_bytes_total = pool_bytes * self.R
         self.max_ctx = max(1, b.max_context_len)
-        self.partition = pa.decode_splitk_partition(self.B, w.num_kv_heads, self.max_ctx,
-                                                    w.partition_tokens if partition < 0 else partition)
+        # 0: the library's schedule (balanced stream schedule on the tensor-core path)
+        self.partition = w.partition_tokens if partition < 0 else partition
         nbytes = pa.decode_splitk_workspace_size(self.B, w.num_q_heads, w.head_dim, self.max_ctx, self.partition,
                                                  w.num_kv_heads)
-        self.ws = torch.empty(max(16, nbytes), dtype=torch.uint8, device="cuda")
+        self.ws = torch.zeros(max(16, nbytes), dtype=torch.uint8, device="cuda")  # zero before first use
         self.out = torch.empty_like(b.q)
         self.kv_bytes = wl.kv_bytes(b)
         self.kv_bytes_unique = wl.kv_bytes(b, unique=True)
-        self.decode_launches = 0
+        self.launches_per_step = 0
 
-    def append(self, r, k_new=None, v_new=None, slots=None):
+    def inputs(self):
         b = self.batch
-        kc, vc = self.pools[r]
-        self.pa.write_kv(b.k_new if k_new is None else k_new, b.v_new if v_new is None else v_new,
-                         b.slot_mapping if slots is None else slots, kc, vc)
+        return dict(q=b.q, k_new=b.k_new, v_new=b.v_new, slot_mapping=b.slot_mapping, block_tables=b.block_tables,
+                    context_lens=b.context_lens)
 
-    def decode(self, r, q=None, tables=None, lens=None):
-        b, w = self.batch, self.w
+    def append(self, r, x):
         kc, vc = self.pools[r]
-        q = b.q if q is None else q
-        tables = b.block_tables if tables is None else tables
-        lens = b.context_lens if lens is None else lens
-        if self.split:
-            self.pa.decode_splitk(q, kc, vc, tables, lens, w.scale, w.softcap, w.window,
+        self.pa.write_kv(x["k_new"], x["v_new"], x["slot_mapping"], kc, vc)
+        return self.pa.last_launch_count()
+
+    def decode(self, r, x):
+        w = self.w
+        kc, vc = self.pools[r]
+        if self.fused:
+            self.pa.decode_step(x["q"], x["k_new"], x["v_new"], kc, vc, x["block_tables"], x["context_lens"], w.scale,
+                                w.softcap, w.window, split=self.split, max_context_len=self.max_ctx,
+                                partition_tokens=self.partition, out=self.out, workspace=self.ws, kernel=self.kernel)
+        elif self.split:
+            self.pa.decode_splitk(x["q"], kc, vc, x["block_tables"], x["context_lens"], w.scale, w.softcap, w.window,
                                   max_context_len=self.max_ctx, partition_tokens=self.partition, out=self.out,
                                   workspace=self.ws, kernel=self.kernel)
         else:
-            self.pa.decode(q, kc, vc, tables, lens, w.scale, w.softcap, w.window, out=self.out, kernel=self.kernel)
-        self.decode_launches = self.pa.last_launch_count()
+            self.pa.decode(x["q"], kc, vc, x["block_tables"], x["context_lens"], w.scale, w.softcap, w.window,
+                           out=self.out, kernel=self.kernel)
+        return self.pa.last_launch_count()
 
-    def step(self, r):
-        self.append(r)
-        self.decode(r)
+    def step(self, r, x=None, ev=None):
+        """One step on pool r.  ``ev``: (start, end) events around the decode launch(es)."""
+        x = self.inputs() if x is None else x
+        n = 0 if self.fused else self.append(r, x)
+        if ev is not None:
+            ev[0].record()
+        n += self.decode(r, x)
+        if ev is not None:
+            ev[1].record()
+        self.launches_per_step = n
 
     def timed_graph(self, K: int):
         """Capture K steps (pool i % R) with external timing events around each decode."""
@@ -282,11 +302,7 @@ class Runner:
         with torch.cuda.stream(s):
             with torch.cuda.graph(g, stream=s):
                 for i in range(K):
-                    r = i % self.R
-                    self.append(r)
-                    ev[i][0].record()
-                    self.decode(r)
-                    ev[i][1].record()
+                    self.step(i % self.R, ev=ev[i])
         torch.cuda.current_stream().wait_stream(s)
         torch.cuda.synchronize()
         return g, ev
@@ -321,8 +337,8 @@ def run_e2e(runner: Runner, K: int, world: int):
     """Public-API step with host inputs: H2D of the step's inputs, append, decode,
     D2H of the output, all inside the timed region (eager launches)."""
     b = runner.batch
-    host = {n: getattr(b, n).cpu().pin_memory() for n in ("q", "k_new", "v_new", "slot_mapping", "block_tables",
-                                                         "context_lens")}
+    names = ("q", "k_new", "v_new", "block_tables", "context_lens") + (() if runner.fused else ("slot_mapping",))
+    host = {n: getattr(b, n).cpu().pin_memory() for n in names}
     dev = {n: torch.empty_like(getattr(b, n)) for n in host}
     out_host = torch.empty(b.q.shape, dtype=b.q.dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host.values())
@@ -331,9 +347,7 @@ def run_e2e(runner: Runner, K: int, world: int):
     def one(i):
         for n in host:
             dev[n].copy_(host[n], non_blocking=True)
-        r = i % runner.R
-        runner.append(r, dev["k_new"], dev["v_new"], dev["slot_mapping"])
-        runner.decode(r, dev["q"], dev["block_tables"], dev["context_lens"])
+        runner.step(i % runner.R, dev)
         out_host.copy_(runner.out, non_blocking=True)
 
     for i in range(3):
@@ -415,15 +429,19 @@ def describe(w: wl.Workload, runner: Runner, args, l2_note: str):
         "softcap": w.softcap,
         "window": w.window,
         "prefix_share": w.prefix_share,
-        "path": "pa_decode" if not runner.split else f"pa_decode_splitk(partition={runner.partition})",
+        "path": ("pa_decode_step" if runner.fused else "pa_write_kv + " + ("pa_decode_splitk" if runner.split else
+                                                                          "pa_decode"))
+        + ((" (split-K, dynamic work queue)" if runner.partition == 0 else
+            f" (split-K, partition {runner.partition})") if runner.split else " (one CTA per sequence, kv head)"),
         "kernel": args.kernel,
         "l2": l2_note,
         "seed": "workload seed + 7919 * rank",
     }
 
 
-def shape_summary(w: wl.Workload, rank: int, kernel: str, K: int, W: int, world: int, dev_idx: int, peak: float):
-    runner = Runner(w, rank, kernel, True, -1)
+def shape_summary(w: wl.Workload, rank: int, kernel: str, K: int, W: int, world: int, dev_idx: int, peak: float,
+                  partition: int = -1):
+    runner = Runner(w, rank, kernel, True, partition)
     total_ms, dec_ms, _ = run_timed(runner, K, W, world, dev_idx)
     ms = total_ms / K
     res = {
@@ -446,7 +464,7 @@ def shape_summary(w: wl.Workload, rank: int, kernel: str, K: int, W: int, world:
 def main_ours(args, world, rank, local):
     w = wl.WORKLOADS[args.workload]
     split = not args.no_split
-    runner = Runner(w, rank, args.kernel, split, args.partition)
+    runner = Runner(w, rank, args.kernel, split, args.partition, fused=not args.unfused)
     l2 = torch.cuda.get_device_properties(local).L2_cache_size
     l2_note = (f"rotating {runner.R} KV pool copies ({runner.pool_bytes_total / 1e6:.0f} MB, "
                f"L2 {l2 / 1e6:.0f} MB)")
@@ -460,9 +478,9 @@ def main_ours(args, world, rank, local):
     e2e_ms = max_over_ranks(e2e_ms, world)
     peak, peak_kind = measured_peaks()
     achieved = runner.kv_bytes / (dec_ms * 1e-3) / 1e9
-    kernel_key = "splitk" if split else "decode"
+    kernel_key = ("step" if runner.fused else "decode") + ("_splitk" if split else "")
     traffic = recorded_traffic(w.name, kernel_key)
-    launches_per_step = 1 + runner.decode_launches
+    launches_per_step = runner.launches_per_step
     line = {
         "metric": METRIC,
         "value": round(value, 1),
@@ -479,7 +497,8 @@ def main_ours(args, world, rank, local):
         "config": describe(w, runner, args, l2_note),
         "roofline": {
             "bound": "hbm",
-            "kernel": "decode (split-K partial + LSE combine)" if split else "decode",
+            "kernel": ("fused append + " if runner.fused else "") + (
+                "split-K decode + LSE combine" if split else "decode"),
             "achieved": round(achieved, 1),
             "peak": peak,
             "peak_kind": peak_kind,
@@ -507,6 +526,8 @@ def main_ours(args, world, rank, local):
         torch.cuda.empty_cache()
         for n in names:
             extra[n] = shape_summary(wl.WORKLOADS[n], rank, args.kernel, 50, 5, world, local, peak)
+            if wl.WORKLOADS[n].partition_tokens:  # also the dynamic schedule
+                extra[n + "@dynamic"] = shape_summary(wl.WORKLOADS[n], rank, args.kernel, 50, 5, world, local, peak, 0)
         line["per_shape"] = extra
         runner = None
     if world == 1 and rank == 0 and not args.no_cpu:

@@ -127,14 +127,25 @@ pa_status_t pa_decode(const void* q, const void* k_cache, const void* v_cache, c
  *     M = max_p m_p,  out = sum_p e^(m_p - M) o_p / sum_p e^(m_p - M) l_p.
  *   A sequence whose range falls in one partition is written directly by that
  *   partition's CTA; its result is then bit-identical to pa_decode's.
+ *   The combine kernel is launched as a programmatic dependent of the first
+ *   (its launch overlaps the first kernel's tail; it reads nothing before the
+ *   first kernel has completed).
  *   partition_tokens: a multiple of 64, or 0 to let the library choose (see
  *   pa_decode_splitk_partition).  max_context_len: an upper bound on every
  *   context_lens[b] (a larger length sets PA_DEVERR_CONTEXT and is clamped);
  *   it sizes the grid and the workspace.
+ *   Schedules: partition_tokens > 0 launches one CTA per (partition, kv head,
+ *   sequence).  partition_tokens == 0 lets the library choose the partition
+ *   size and, on the tensor-core path (bf16) with batch <= 2048, runs the
+ *   dynamic schedule: a persistent grid whose CTAs claim (sequence, kv head,
+ *   partition) items from a counter kept in the workspace, so that SMs that
+ *   stream faster take more of the work.
  *   workspace: device memory of at least pa_decode_splitk_workspace_size()
- *   bytes, 16-byte aligned; its contents need no initialisation and are
- *   scratch between the two kernels of one call.  Calls that share a workspace
- *   must be ordered on one stream.
+ *   bytes, 16-byte aligned, zero-filled before its first use.  Each call
+ *   leaves it ready for the next one (the dynamic schedule's counter returns
+ *   to zero at the end of the call; the rest is scratch between the call's two
+ *   kernels).  After a call that failed or raised PA_DEVERR_TIMEOUT, zero it
+ *   again.  Calls that share a workspace must be ordered on one stream.
  *   Returns PA_ERR_WORKSPACE when the workspace is null, misaligned or small.
  */
 int32_t pa_decode_splitk_partition(int32_t batch, int32_t num_kv_heads, int32_t max_context_len,
@@ -149,6 +160,35 @@ pa_status_t pa_decode_splitk(const void* q, const void* k_cache, const void* v_c
                              int32_t window, void* out, pa_dtype_t dtype, int32_t partition_tokens,
                              int32_t max_context_len, void* workspace, size_t workspace_bytes,
                              pa_kernel_t kernel, pa_stream_t stream);
+
+/*
+ * pa_decode_step -- one decode step: append the step's new key/value rows and
+ * attend, in one pass over the cache.
+ *   Equivalent to pa_write_kv(k_new, v_new, slots) followed by the decode, where
+ *   slots[b] is the slot of position L-1 of sequence b, i.e.
+ *   block_tables[b][(L-1)/bs] * bs + (L-1) % bs with L = context_lens[b]
+ *   (nothing is appended for L == 0).  k_new, v_new: [batch][num_kv_heads]
+ *   [head_dim], device memory, 16-byte aligned.  The cache must not be read by
+ *   other work while the call runs; the block receiving position L-1 must not be
+ *   shared with another sequence (prefix-shared blocks are full and never the
+ *   one being appended to).
+ *   The attention uses the new rows from on-chip memory, and the CTA that
+ *   serves position L-1 of (sequence, kv head) writes them to the cache, so no
+ *   separate append kernel runs.  The outputs and the cache contents equal those
+ *   of pa_write_kv followed by pa_decode / pa_decode_splitk bit for bit.
+ *   partition_tokens < 0: one CTA per (sequence, kv head), like pa_decode (the
+ *   workspace may be NULL and max_context_len is ignored).  partition_tokens >= 0:
+ *   split-K exactly as pa_decode_splitk (0 = library's choice).
+ *   Passage: nano-vllm README, "Key Concepts Explained: KV Cache" (each decode
+ *   step processes only the new token and attends over the cache).
+ */
+pa_status_t pa_decode_step(const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                           const int32_t* block_tables, const int32_t* context_lens, int32_t batch,
+                           int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                           int32_t max_blocks_per_seq, int32_t num_blocks, float scale, float softcap,
+                           int32_t window, void* out, pa_dtype_t dtype, int32_t partition_tokens,
+                           int32_t max_context_len, void* workspace, size_t workspace_bytes, pa_kernel_t kernel,
+                           pa_stream_t stream);
 
 /*
  * pa_device_errors -- read (and with clear != 0, reset) the device error word

@@ -14,6 +14,7 @@ from ._binding import (  # noqa: F401
     PagedAttnError,
     decode,
     decode_splitk,
+    decode_step,
     decode_splitk_partition,
     decode_splitk_workspace_size,
     device_errors,
@@ -27,6 +28,7 @@ __all__ = [
     "write_kv",
     "decode",
     "decode_splitk",
+    "decode_step",
     "decode_splitk_partition",
     "decode_splitk_workspace_size",
     "device_errors",

@@ -49,6 +49,10 @@ def _load_library() -> ctypes.CDLL:
     lib.pa_decode.restype = _c_i32
     lib.pa_decode_splitk.argtypes = dec + [_c_i32, _c_i32, _c_vp, _c_sz, _c_i32, _c_vp]
     lib.pa_decode_splitk.restype = _c_i32
+    lib.pa_decode_step.argtypes = [_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_i32, _c_i32, _c_i32, _c_i32,
+                                   _c_i32, _c_i32, _c_i32, _c_f32, _c_f32, _c_i32, _c_vp, _c_i32, _c_i32, _c_i32,
+                                   _c_vp, _c_sz, _c_i32, _c_vp]
+    lib.pa_decode_step.restype = _c_i32
     lib.pa_decode_splitk_partition.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32]
     lib.pa_decode_splitk_partition.restype = _c_i32
     lib.pa_decode_splitk_workspace_size.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32]
@@ -141,19 +145,52 @@ def decode_splitk(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                   workspace: Optional[torch.Tensor] = None, kernel: str = "auto", stream=None) -> torch.Tensor:
     """Split-K (flash-decoding) paged decode with the log-sum-exp combine.
 
-    ``max_context_len`` is a host-side bound on every ``context_lens[b]``.  The
-    workspace (any dtype, device memory) is allocated with torch if not given.
+    ``max_context_len`` is a host-side bound on every ``context_lens[b]``.
+    ``partition_tokens=0`` lets the library schedule the work (the dynamic work
+    queue on the tensor-core path).  The workspace (device memory) must be
+    zero-filled before its first use; it is allocated zeroed with torch if not
+    given.
     """
     B, hq, d, nb, hkv, bs, out = _decode_common(q, k_cache, block_tables, out)
     need = decode_splitk_workspace_size(B, hq, d, max_context_len, partition_tokens, hkv)
     if workspace is None:
-        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+        workspace = torch.zeros(max(need, 16), dtype=torch.uint8, device=q.device)
     wbytes = workspace.numel() * workspace.element_size()
     st = lib.pa_decode_splitk(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens), B, hq,
                               hkv, d, bs, block_tables.shape[1], nb, float(scale), float(softcap), int(window),
                               _ptr(out), _dtype_code(q), int(partition_tokens), int(max_context_len),
                               _ptr(workspace), wbytes, KERNELS[kernel], _stream(stream))
     _check(st, "pa_decode_splitk")
+    return out
+
+
+def decode_step(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor,
+                v_cache: torch.Tensor, block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
+                softcap: float = 0.0, window: int = 0, *, split: bool = True, max_context_len: int = 0,
+                partition_tokens: int = 0, out: Optional[torch.Tensor] = None,
+                workspace: Optional[torch.Tensor] = None, kernel: str = "auto", stream=None) -> torch.Tensor:
+    """One decode step: append ``k_new``/``v_new`` ``[B, Hkv, D]`` at position
+    ``context_lens[b] - 1`` of each sequence and attend, in one pass.
+
+    ``split=False``: one CTA per (sequence, kv head).  ``split=True``: split-K
+    with the combine (``max_context_len`` required; workspace allocated with
+    torch if not given).
+    """
+    B, hq, d, nb, hkv, bs, out = _decode_common(q, k_cache, block_tables, out)
+    ptoks = int(partition_tokens) if split else -1
+    wptr, wbytes = None, 0
+    if split:
+        if max_context_len <= 0:
+            raise ValueError("decode_step(split=True) needs max_context_len")
+        need = decode_splitk_workspace_size(B, hq, d, max_context_len, partition_tokens, hkv)
+        if workspace is None:
+            workspace = torch.zeros(max(need, 16), dtype=torch.uint8, device=q.device)
+        wptr, wbytes = _ptr(workspace), workspace.numel() * workspace.element_size()
+    st = lib.pa_decode_step(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                            _ptr(context_lens), B, hq, hkv, d, bs, block_tables.shape[1], nb, float(scale),
+                            float(softcap), int(window), _ptr(out), _dtype_code(q), ptoks, int(max_context_len), wptr,
+                            wbytes, KERNELS[kernel], _stream(stream))
+    _check(st, "pa_decode_step")
     return out
 
 

@@ -2,95 +2,106 @@
 #pragma once
 
 #include "decode_common.cuh"
+#include "ptx.cuh"
 
 namespace pa {
 
 // ---- split-K combine ----------------------------------------------------------
 //
-// One CTA per (query head, sequence).  The partitions of the sequence's
-// attended range each left (m_p, l_p, o_p) in the workspace (log2 domain, o_p
-// unnormalised relative to m_p).  With M = max_p m_p:
+// NWR warps per output row (sequence b, query head h).  The partitions of the
+// sequence's attended range each left (m_p, l_p, o_p) in the workspace (log2
+// domain, o_p unnormalised relative to m_p).  With M = max_p m_p:
 //   out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p.
-// Sequences whose range fits one partition were written by the decode kernel.
+// Warp r of a row takes partitions r, r + NWR, ...; lane k computes the
+// weights of every 32nd of those and broadcasts them, and each lane
+// accumulates D/32 consecutive dims.  With NWR > 1 the row's warps add their
+// sums through shared memory.  Sequences whose range fits one partition were
+// written by the decode kernel and are skipped here.
 constexpr int kCombineWarps = 8;
 
-template <typename OutT, int D>
+template <typename OutT, int D, int NWR>
 __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const DecodeParams p) {
   constexpr int VEC = D / 32;
-  extern __shared__ __align__(16) float csm[];  // [max_parts] weights, then [kCombineWarps][D]
-  __shared__ float red[kCombineWarps];
-  __shared__ float s_M, s_den;
-
-  const int h = blockIdx.x, b = blockIdx.y;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int L = clamp_context(p, b, false);
-  const int s0 = window_start(L, p.window);
-  if (L <= s0) return;
-  const int P = p.partition;
-  const int pb = s0 / P, n = (L + P - 1) / P - pb;
-  if (n <= 1) return;
-
-  const size_t row = (size_t)b * p.hq + h;
-  const float* ml = p.ws_ml + (row * p.max_parts + pb) * 2;
-  const float* po = p.ws_o + (row * p.max_parts + pb) * D;
-  float* wts = csm;
-  float* acc_s = csm + ((p.max_parts + 3) & ~3);
-
-  float M = -CUDART_INF_F;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) M = fmaxf(M, ml[2 * i]);
+  constexpr int ROWS = kCombineWarps / NWR;  // rows per CTA
+  constexpr uint32_t FULL = 0xffffffffu;
+  __shared__ float red_o[NWR > 1 ? kCombineWarps : 1][NWR > 1 ? D : 1];
+  __shared__ float red_l[kCombineWarps];
+  pdl_wait();  // the partials come from the preceding decode kernel
+  if (p.dynamic && blockIdx.x == 0 && threadIdx.x == 0) *p.queue = 0;  // ready for the next call
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int r = warp % NWR;
+  const int row = blockIdx.x * ROWS + warp / NWR;
+  bool active = row < p.batch * p.hq;
+  int pb = 0, n = 0;
+  if (active) {
+    const int b = row / p.hq;
+    const int L = clamp_context(p, b, false);
+    const int s0 = window_start(L, p.window);
+    const int P = p.partition;
+    pb = s0 / P;
+    n = L > s0 ? (L + P - 1) / P - pb : 0;
+    if (p.dynamic && n == 0 && r == 0) {  // no work item covered this row
+      OutT* out = static_cast<OutT*>(p.out) + (size_t)row * D + lane * VEC;
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-  if (lane == 0) red[warp] = M;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float v = red[0];
-    for (int w = 1; w < kCombineWarps; ++w) v = fmaxf(v, red[w]);
-    s_M = v;
+      for (int v = 0; v < VEC; ++v) store_out<OutT>(out + v, 0.f);
+    }
+    active = n > 1;
   }
-  __syncthreads();
-  M = s_M;
-
-  float den = 0.f;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    const float w = exp2f(ml[2 * i] - M);
-    wts[i] = w;
-    den += w * ml[2 * i + 1];
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
-  __syncthreads();  // red[] reuse
-  if (lane == 0) red[warp] = den;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float v = 0.f;
-    for (int w = 0; w < kCombineWarps; ++w) v += red[w];
-    s_den = v;
-  }
-
   float acc[VEC];
 #pragma unroll
   for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
-  for (int i = warp; i < n; i += kCombineWarps) {
-    const float w = wts[i];
-    const float* src = po + (size_t)i * D + lane * VEC;
+  float den = 0.f;
+  if (active) {
+    const float* ml = p.ws_ml + ((size_t)row * p.max_parts + pb) * 2;
+    const float* po = p.ws_o + ((size_t)row * p.max_parts + pb) * D + lane * VEC;
+    float M = -CUDART_INF_F;
+    for (int i = lane; i < n; i += 32) M = fmaxf(M, ml[2 * i]);
 #pragma unroll
-    for (int v = 0; v < VEC; v += 2) {
-      const float2 x = *reinterpret_cast<const float2*>(src + v);
-      acc[v] = fmaf(w, x.x, acc[v]);
-      acc[v + 1] = fmaf(w, x.y, acc[v + 1]);
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, off));
+    // This warp's partitions: i = r + NWR * j.
+    const int nj = (n - r + NWR - 1) / NWR;
+    for (int c = 0; c < nj; c += 32) {
+      const int j = c + lane;
+      float w = 0.f;
+      if (j < nj) {
+        const int i = r + NWR * j;
+        w = exp2f(ml[2 * i] - M);
+        den = fmaf(w, ml[2 * i + 1], den);
+      }
+      const int cnt = min(32, nj - c);
+#pragma unroll 8
+      for (int e = 0; e < cnt; ++e) {
+        const float wj = __shfl_sync(FULL, w, e);
+        const float* src = po + (size_t)(r + NWR * (c + e)) * D;
+#pragma unroll
+        for (int v = 0; v < VEC; v += 2) {
+          const float2 x = *reinterpret_cast<const float2*>(src + v);
+          acc[v] = fmaf(wj, x.x, acc[v]);
+          acc[v + 1] = fmaf(wj, x.y, acc[v + 1]);
+        }
+      }
     }
-  }
 #pragma unroll
-  for (int v = 0; v < VEC; ++v) acc_s[warp * D + lane * VEC + v] = acc[v];
-  __syncthreads();
-  OutT* out = static_cast<OutT*>(p.out) + row * D;
-  const float inv = 1.f / s_den;
-  for (int d = threadIdx.x; d < D; d += blockDim.x) {
-    float s = 0.f;
-#pragma unroll
-    for (int w = 0; w < kCombineWarps; ++w) s += acc_s[w * D + d];
-    store_out<OutT>(out + d, s * inv);
+    for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(FULL, den, off);
   }
+  if (NWR > 1) {
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) red_o[warp][lane * VEC + v] = acc[v];
+    if (lane == 0) red_l[warp] = den;
+    __syncthreads();
+    if (!active || r != 0) return;
+    for (int w2 = 1; w2 < NWR; ++w2) {
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) acc[v] += red_o[warp + w2][lane * VEC + v];
+      den += red_l[warp + w2];
+    }
+  } else if (!active) {
+    return;
+  }
+  const float inv = 1.f / den;
+  OutT* out = static_cast<OutT*>(p.out) + (size_t)row * D + lane * VEC;
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) store_out<OutT>(out + v, acc[v] * inv);
 }
 
 // ---- KV append ------------------------------------------------------------------

@@ -29,8 +29,11 @@ struct DecodeParams {
   const void* v_cache;
   const int32_t* block_tables;  // [B][max_blocks]
   const int32_t* context_lens;  // [B]
+  const void* k_new;            // fused append: the step's new rows [B][Hkv][D] (else null)
+  const void* v_new;
   float* ws_o;                  // split-K partial outputs [B][Hq][max_parts][D]
   float* ws_ml;                 // split-K partial (m, l)  [B][Hq][max_parts][2]
+  int* queue;                   // dynamic schedule: the work-item counter (zero between calls)
   int batch, hq, hkv, group, head_dim;
   int block_size, log2_bs, max_blocks, num_blocks;
   int window;
@@ -41,6 +44,7 @@ struct DecodeParams {
   float softcap;    // > 0 and finite: cap enabled
   float inv_softcap;
   int use_softcap;
+  int dynamic;      // the dynamic schedule ran: the combine also resets `queue` and writes L == 0 rows
 };
 
 // Token range one CTA attends.
@@ -75,6 +79,12 @@ __device__ __forceinline__ CtaRange cta_range(const DecodeParams& p, int b, int 
   return r;
 }
 
+// Row (within the 2-D view [num_blocks*Hkv*bs][D] of the cache) holding token t
+// of kv head g, given the token's physical block.
+__device__ __forceinline__ int cache_row(const DecodeParams& p, int phys, int g, int t) {
+  return (phys * p.hkv + g) * p.block_size + (t & (p.block_size - 1));
+}
+
 template <typename T>
 __device__ __forceinline__ void store_out(T* dst, float v);
 template <>
@@ -89,62 +99,86 @@ __device__ void write_zero_rows(const DecodeParams& p, int b, int g) {
   for (int i = threadIdx.x; i < p.group * p.head_dim; i += blockDim.x) store_out<T>(out + i, 0.f);
 }
 
-// Cross-warp merge buffer: per warp, per head (max, sum) and the unnormalised
-// output row, all in the log2 domain.  Laid over the CTA's ring buffer once
-// every warp has finished with it.
+// Cross-warp merge buffer: per warp w and head h (slot w*gs + h) the running
+// max, the sum (log2 domain) and the unnormalised output row.
 struct MergeSmem {
-  float* m;  // [NW][kMaxGroup]
-  float* l;  // [NW][kMaxGroup]
-  float* o;  // [NW][kMaxGroup][D]
+  float* m;  // [NW][gs]
+  float* l;  // [NW][gs]
+  float* o;  // [NW][gs][D]
+  int gs;    // head stride
 };
 
 template <int NW>
-__device__ __forceinline__ MergeSmem merge_smem(void* base, int D) {
+__device__ __forceinline__ MergeSmem merge_smem(void* base, int D, int gs = kMaxGroup) {
   MergeSmem s;
   s.m = static_cast<float*>(base);
-  s.l = s.m + NW * kMaxGroup;
-  s.o = s.l + NW * kMaxGroup;
+  s.l = s.m + NW * gs;
+  s.o = s.l + NW * gs;
+  s.gs = gs;
   (void)D;
   return s;
 }
 
 template <int NW>
-__host__ __device__ constexpr int merge_smem_bytes(int D) {
-  return (2 * NW * kMaxGroup + NW * kMaxGroup * D) * 4;
+__host__ __device__ constexpr int merge_smem_bytes(int D, int gs = kMaxGroup) {
+  return (2 * NW * gs + NW * gs * D) * 4;
 }
 
-// Combine the NW warps' states and write either the final output (normalised,
-// input dtype) or the partition's partial state to the workspace.
+// Where a merged (sequence, kv head) group of G query heads goes: the
+// normalised rows (final) or the partial state (m, l in log2 domain, o
+// unnormalised), each with its own per-head stride in elements.
+template <typename OutT>
+struct MergeDest {
+  bool final_write;
+  OutT* out;  // head h at out + h * D
+  float* po;  // head h at po + h * po_stride
+  float* pml; // head h at pml + h * pml_stride
+  size_t po_stride, pml_stride;
+};
+
+// Combine the NW warps' states in `s` for the G heads, using threads
+// [tid0, tid0 + nthreads) of the CTA.
 template <int NW, typename OutT>
-__device__ void merge_and_store(const DecodeParams& p, const MergeSmem& s, int b, int g, int part,
-                                bool final_write) {
-  const int D = p.head_dim, G = p.group;
-  for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+__device__ void merge_warps(const MergeSmem& s, int G, int D, const MergeDest<OutT>& dst, int tid, int nthreads) {
+  for (int idx = tid; idx < G * D; idx += nthreads) {
     const int h = idx / D, d = idx - h * D;
     float M = -CUDART_INF_F;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) M = fmaxf(M, s.m[w * kMaxGroup + h]);
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, s.m[w * s.gs + h]);
     float num = 0.f, den = 0.f;
 #pragma unroll
     for (int w = 0; w < NW; ++w) {
-      const float mw = s.m[w * kMaxGroup + h];
+      const float mw = s.m[w * s.gs + h];
       if (mw == -CUDART_INF_F) continue;  // this warp saw no token
       const float c = exp2f(mw - M);
-      num += c * s.o[(w * kMaxGroup + h) * D + d];
-      den += c * s.l[w * kMaxGroup + h];
+      num += c * s.o[(w * s.gs + h) * D + d];
+      den += c * s.l[w * s.gs + h];
     }
-    const size_t row = (size_t)b * p.hq + (size_t)g * G + h;
-    if (final_write) {
-      store_out<OutT>(static_cast<OutT*>(p.out) + row * D + d, num / den);
+    if (dst.final_write) {
+      store_out<OutT>(dst.out + (size_t)h * D + d, num / den);
     } else {
-      const size_t slot = row * p.max_parts + part;
-      p.ws_o[slot * D + d] = num;
+      dst.po[h * dst.po_stride + d] = num;
       if (d == 0) {
-        p.ws_ml[slot * 2 + 0] = M;
-        p.ws_ml[slot * 2 + 1] = den;
+        dst.pml[h * dst.pml_stride + 0] = M;
+        dst.pml[h * dst.pml_stride + 1] = den;
       }
     }
   }
+}
+
+// The grid-scheduled kernels' destination: output rows of (b, g) or the
+// partition's slot in the [B][Hq][max_parts] workspace.
+template <typename OutT>
+__device__ __forceinline__ MergeDest<OutT> grid_dest(const DecodeParams& p, int b, int g, int part, bool final_write) {
+  MergeDest<OutT> d;
+  const size_t row = (size_t)b * p.hq + (size_t)g * p.group;
+  d.final_write = final_write;
+  d.out = static_cast<OutT*>(p.out) + row * p.head_dim;
+  d.po = p.ws_o + (row * p.max_parts + part) * p.head_dim;
+  d.pml = p.ws_ml + (row * p.max_parts + part) * 2;
+  d.po_stride = (size_t)p.max_parts * p.head_dim;
+  d.pml_stride = (size_t)p.max_parts * 2;
+  return d;
 }
 
 }  // namespace pa

@@ -7,9 +7,14 @@
 // vector load from global memory, and the warp sums the per-lane partial dot
 // products with shuffles.  Used for fp32 caches and as the CUDA-core baseline
 // the tensor-core kernel is measured against.
+//
+// APPEND (the fused decode step): the CTA whose range ends at the sequence's
+// last token takes position L-1's key/value from the step's new rows, and the
+// warp that meets it also writes them to the cache slot of that position.
 #pragma once
 
 #include "decode_common.cuh"
+#include "ptx.cuh"
 
 namespace pa {
 
@@ -65,11 +70,12 @@ struct VecLoad<__nv_bfloat16, VEC> {
 };
 
 // GP: group size rounded up to a power of two (heads >= G are padding).
-template <typename T, int D, int GP, int NW, bool SPLIT>
+template <typename T, int D, int GP, int NW, bool SPLIT, bool APPEND>
 __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams p) {
   constexpr int VEC = D / 32;
   constexpr int U = 4;  // tokens per inner step
   extern __shared__ __align__(16) uint8_t smem_raw[];
+  if (SPLIT) pdl_launch_dependents();  // the combine kernel may launch now and wait for this grid
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int part = SPLIT ? (int)blockIdx.x : 0;
@@ -108,6 +114,8 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams
   const int32_t* table = p.block_tables + (size_t)b * p.max_blocks;
   const T* kc = static_cast<const T*>(p.k_cache);
   const T* vc = static_cast<const T*>(p.v_cache);
+  const bool append_cta = APPEND && r.hi == r.L;
+  const size_t new_off = ((size_t)b * p.hkv + g) * D + lane * VEC;
 
   for (int j = j0 + warp; j < j1; j += NW) {
     const int t0 = j * kSliceTokens;
@@ -124,7 +132,20 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams
       for (int u = 0; u < U; ++u) {
         const int t = t0 + u0 + u;
         valid[u] = t >= r.lo && t < r.hi;
-        if (valid[u]) {
+        if (APPEND && append_cta && t == r.L - 1) {
+          // The appended token: read the new rows and store them in the cache.
+          const T* kn = static_cast<const T*>(p.k_new) + new_off;
+          const T* vn = static_cast<const T*>(p.v_new) + new_off;
+          VecLoad<T, VEC>::load(kn, kr[u]);
+          VecLoad<T, VEC>::load(vn, vr[u]);
+          T* kd = const_cast<T*>(kc) + (row0 + u0 + u) * D + lane * VEC;
+          T* vd = const_cast<T*>(vc) + (row0 + u0 + u) * D + lane * VEC;
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) {
+            kd[e] = kn[e];
+            vd[e] = vn[e];
+          }
+        } else if (valid[u]) {
           VecLoad<T, VEC>::load(kc + (row0 + u0 + u) * D + lane * VEC, kr[u]);
           VecLoad<T, VEC>::load(vc + (row0 + u0 + u) * D + lane * VEC, vr[u]);
         } else {
@@ -195,7 +216,7 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams
     }
   }
   __syncthreads();
-  merge_and_store<NW, T>(p, ms, b, g, part, !SPLIT || r.final_write);
+  merge_warps<NW, T>(ms, G, D, grid_dest<T>(p, b, g, part, !SPLIT || r.final_write), threadIdx.x, blockDim.x);
 }
 
 }  // namespace pa

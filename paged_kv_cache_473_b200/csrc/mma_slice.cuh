@@ -1,0 +1,226 @@
+// One warp's attention over one 16-token slice held in shared memory, on the
+// tensor cores (bf16 warp MMA, fp32 accumulation), and the per-warp online
+// softmax state it updates.  Shared by the decode kernels.
+//
+// Shared-memory slice layout (as landed by TMA with 128-byte swizzle): K then V,
+// each D/64 panels of [16 rows x 128 B]; 16-byte chunk c of row r sits at
+// chunk c ^ (r & 7).
+//
+// With G <= 8 query heads of the group padded to 8 MMA columns:
+//   S^T[16 tok x 8 heads] = K[16 x D] . Q^T[D x 8]          (D/16 MMAs)
+//   online softmax over the slice (fp32, log2 domain, warp shuffles)
+//   O^T[D x 8 heads]     += V^T[D x 16] . P^T[16 x 8]        (D/16 MMAs)
+// K feeds the A operand straight from shared memory (ldmatrix), V^T through
+// ldmatrix.trans, and P moves from the S accumulator layout to the B operand
+// layout with movmatrix.trans, so it never touches shared memory.
+#pragma once
+
+#include "decode_common.cuh"
+#include "ptx.cuh"
+
+namespace pa {
+
+constexpr int kPanelBytes = kSliceTokens * 128;  // 16 rows x 128 B
+
+template <int D>
+struct SliceBytes {
+  static constexpr int kSlice = (D / 64) * kPanelBytes;  // K (or V) of one slice
+  static constexpr int kStage = 2 * kSlice;             // K then V
+};
+
+// Lane n0 = 2*(lane%4) holds heads n0 and n0+1: running max (log2 domain), its
+// partial sum over the tokens it saw, and O^T rows d = mt*16 + lane/4 (+8).
+template <int D>
+struct WarpAttn {
+  float m0, m1, l0, l1;
+  float o[D / 16][4];
+
+  __device__ __forceinline__ void reset() {
+    m0 = m1 = -CUDART_INF_F;
+    l0 = l1 = 0.f;
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+  }
+
+  // Lane partial sums -> per-head sums (lanes with the same lane%4 share heads).
+  __device__ __forceinline__ void reduce_sums() {
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+    }
+  }
+
+  // Write this warp's state into the merge buffer: m[warp*gs + h], l[...],
+  // o[(warp*gs + h)*D + d] for the G real heads.  Call after reduce_sums().
+  __device__ __forceinline__ void dump(float* m, float* l, float* ob, int warp, int gs, int G, int lane) const {
+    const int n0 = 2 * (lane & 3);
+    if (lane < 4) {
+      if (n0 < G) {
+        m[warp * gs + n0] = m0;
+        l[warp * gs + n0] = l0;
+      }
+      if (n0 + 1 < G) {
+        m[warp * gs + n0 + 1] = m1;
+        l[warp * gs + n0 + 1] = l1;
+      }
+    }
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) {
+      const int d = mt * 16 + (lane >> 2);
+      if (n0 < G) {
+        ob[(warp * gs + n0) * D + d] = o[mt][0];
+        ob[(warp * gs + n0) * D + d + 8] = o[mt][2];
+      }
+      if (n0 + 1 < G) {
+        ob[(warp * gs + n0 + 1) * D + d] = o[mt][1];
+        ob[(warp * gs + n0 + 1) * D + d + 8] = o[mt][3];
+      }
+    }
+  }
+};
+
+// Q^T as the B operand of S^T = K Q^T: column n = lane / 4 is query head n of
+// the group; heads >= G are zero.
+template <int D>
+__device__ __forceinline__ void load_q_frags(uint32_t (&qf)[D / 16][2], const __nv_bfloat16* q_group, int G,
+                                             int lane) {
+  const int n = lane >> 2;
+  const __nv_bfloat16* qrow = q_group + (size_t)(n < G ? n : 0) * D;
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const int c = kk * 16 + 2 * (lane & 3);
+    qf[kk][0] = n < G ? *reinterpret_cast<const uint32_t*>(qrow + c) : 0u;
+    qf[kk][1] = n < G ? *reinterpret_cast<const uint32_t*>(qrow + c + 8) : 0u;
+  }
+}
+
+// Load one slice (cache rows [y, y+16) of K and of V) into the stage at `dst`
+// with 2-D TMA tile loads, one 64-column panel per instruction.  The warp
+// calls this together: lane 0 arms the stage's barrier with the byte count and
+// lanes 0 .. 2*D/64-1 each issue one panel (issuing from several lanes at once
+// costs about as much as one TMA instruction from one lane).  y < 0 (a bad
+// block id) arms the barrier with no bytes and raises PA_DEVERR_BLOCK.
+template <int D>
+__device__ __forceinline__ void issue_slice(uint32_t dst, uint32_t bar, const CUtensorMap* kmap,
+                                            const CUtensorMap* vmap, int y, int lane) {
+  constexpr int kPanels = D / 64;
+  if (y < 0) {
+    if (lane == 0) {
+      raise_error(PA_DEVERR_BLOCK);
+      mbar_arrive(bar);  // complete the phase with no data; the slice computes on stale tiles
+    }
+    return;
+  }
+  if (lane == 0) mbar_arrive_expect_tx(bar, SliceBytes<D>::kStage);
+  __syncwarp();
+  if (lane < 2 * kPanels) {
+    const int pn = lane % kPanels;
+    const bool is_v = lane >= kPanels;
+    tma_load_2d(dst + (is_v ? SliceBytes<D>::kSlice : 0) + pn * kPanelBytes, is_v ? vmap : kmap, bar, pn * 64, y);
+  }
+}
+
+// Overwrite row `row` (0..15) of the slice at kbase/vbase with the new key and
+// value rows; lane l < D/8 holds 16-byte chunk l of each.
+template <int D>
+__device__ __forceinline__ void overwrite_slice_row(uint32_t kbase, uint32_t vbase, int row, const uint4& knew,
+                                                    const uint4& vnew, int lane) {
+  if (lane < D / 8) {
+    const uint32_t off = (lane >> 3) * kPanelBytes + row * 128 + (((lane & 7) ^ (row & 7)) << 4);
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(kbase + off), "r"(knew.x), "r"(knew.y),
+                 "r"(knew.z), "r"(knew.w)
+                 : "memory");
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(vbase + off), "r"(vnew.x), "r"(vnew.y),
+                 "r"(vnew.z), "r"(vnew.w)
+                 : "memory");
+    fence_proxy_async_smem();  // before TMA writes this stage again
+  }
+  __syncwarp();
+}
+
+// Attend the slice of tokens [t0, t0+16) whose K/V rows sit at kbase/vbase;
+// only tokens in [lo, hi) count.
+template <int D>
+__device__ __forceinline__ void attend_slice(WarpAttn<D>& st, const uint32_t (&qf)[D / 16][2], uint32_t kbase,
+                                             uint32_t vbase, int t0, int lo, int hi, float qk_scale,
+                                             const DecodeParams& p, int lane) {
+  constexpr uint32_t FULL = 0xffffffffu;
+  const uint32_t k_lane = ((lane & 7) | (lane & 8)) * 128;          // row = lane%8 + 8*((lane/8)%2)
+  const uint32_t v_lane = ((lane & 7) | ((lane >> 4) << 3)) * 128;  // row = lane%8 + 8*(lane/16)
+  const uint32_t k_sub = lane >> 4, v_sub = (lane >> 3) & 1, swz = lane & 7;
+
+  // ---- S^T = K Q^T ---------------------------------------------------------
+  float sc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t chunk = ((kk & 3) << 1) | k_sub;
+    const uint32_t addr = kbase + (kk >> 2) * kPanelBytes + k_lane + ((chunk ^ swz) << 4);
+    uint32_t a0, a1, a2, a3;
+    ldsm_x4(addr, a0, a1, a2, a3);
+    mma_bf16_16816(sc, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+  }
+  // sc[0], sc[1]: token t0 + lane/4, heads n0, n0+1; sc[2], sc[3]: token + 8.
+  float x[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    float v = sc[e] * qk_scale;
+    if (p.use_softcap) v = p.softcap * tanhf(v * p.inv_softcap) * kLog2e;
+    x[e] = v;
+  }
+  const bool partial = (t0 < lo) || (t0 + kSliceTokens > hi);
+  uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;
+  if (partial) {
+    const int ta = t0 + (lane >> 2), tb = ta + 8;
+    if (!(ta >= lo && ta < hi)) x[0] = x[1] = -CUDART_INF_F;
+    if (!(tb >= lo && tb < hi)) x[2] = x[3] = -CUDART_INF_F;
+    // Tokens held by this lane in the V^T fragments: 2*(lane%4) (+1) and +8.
+    const int tc = t0 + 2 * (lane & 3);
+    auto ok = [&](int t) { return t >= lo && t < hi; };
+    keep_lo = (ok(tc) ? 0x0000ffffu : 0u) | (ok(tc + 1) ? 0xffff0000u : 0u);
+    keep_hi = (ok(tc + 8) ? 0x0000ffffu : 0u) | (ok(tc + 9) ? 0xffff0000u : 0u);
+  }
+
+  // ---- online softmax --------------------------------------------------------
+  float mx0 = fmaxf(x[0], x[2]), mx1 = fmaxf(x[1], x[3]);
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, off));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, off));
+  }
+  const float mn0 = fmaxf(st.m0, mx0), mn1 = fmaxf(st.m1, mx1);
+  const float al0 = exp2f(st.m0 - mn0), al1 = exp2f(st.m1 - mn1);
+  st.m0 = mn0;
+  st.m1 = mn1;
+  const uint32_t plo = pack_bf16x2(exp2f(x[0] - mn0), exp2f(x[1] - mn1));
+  const uint32_t phi = pack_bf16x2(exp2f(x[2] - mn0), exp2f(x[3] - mn1));
+  st.l0 = st.l0 * al0 + bf16_lo(plo) + bf16_lo(phi);
+  st.l1 = st.l1 * al1 + bf16_hi(plo) + bf16_hi(phi);
+#pragma unroll
+  for (int mt = 0; mt < D / 16; ++mt) {
+    st.o[mt][0] *= al0;
+    st.o[mt][1] *= al1;
+    st.o[mt][2] *= al0;
+    st.o[mt][3] *= al1;
+  }
+  const uint32_t pb0 = movmatrix_trans(plo);
+  const uint32_t pb1 = movmatrix_trans(phi);
+
+  // ---- O^T += V^T P^T ---------------------------------------------------------
+#pragma unroll
+  for (int mt = 0; mt < D / 16; ++mt) {
+    const uint32_t chunk = ((mt & 3) << 1) | v_sub;
+    const uint32_t addr = vbase + (mt >> 2) * kPanelBytes + v_lane + ((chunk ^ swz) << 4);
+    uint32_t a0, a1, a2, a3;
+    ldsm_x4_trans(addr, a0, a1, a2, a3);
+    if (partial) {
+      a0 &= keep_lo;
+      a1 &= keep_lo;
+      a2 &= keep_hi;
+      a3 &= keep_hi;
+    }
+    mma_bf16_16816(st.o[mt], a0, a1, a2, a3, pb0, pb1);
+  }
+}
+
+}  // namespace pa

@@ -9,12 +9,15 @@
 #include <cmath>
 #include <cstdint>
 #include <mutex>
+#include <algorithm>
+#include <utility>
 
 #include "../../include/pagedattn.h"
 #include "combine_and_append.cuh"
 #include "decode_common.cuh"
 #include "decode_mma.cuh"
 #include "decode_simt.cuh"
+#include "decode_dynamic.cuh"
 
 namespace {
 
@@ -25,9 +28,12 @@ thread_local int32_t t_last_launches = 0;
 constexpr int kNoSplitPartition = 1 << 30;
 constexpr int kMaxPartsPerSeq = 8192;
 constexpr int kMaxGridYZ = 65535;
+constexpr size_t kQueueBytes = 256;  // the dynamic schedule's work counter (after the partials)
 // Split-K auto partition: aim for at least this many (partition, kv head,
 // sequence) work units, i.e. several resident CTAs for each of B200's 148 SMs.
 constexpr long long kTargetWorkUnits = 8LL * 148;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
@@ -143,7 +149,28 @@ cudaError_t set_smem(Kernel k, int bytes, std::atomic<uint64_t>& done) {
   return e;
 }
 
-template <int D, int NW, int ST, bool SPLIT>
+// Launch `kern` with cudaLaunchKernelEx; `pdl` lets it start while the
+// preceding kernel on the stream finishes (it must call griddepcontrol.wait
+// before reading that kernel's output).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, int smem, cudaStream_t st, bool pdl,
+                      Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  if (pdl) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+template <int D, int NW, int ST, bool SPLIT, bool APPEND>
 cudaError_t launch_mma_t(const DecodeParams& p, dim3 grid, cudaStream_t st) {
   using Cfg = pa::MmaCfg<D, NW, ST>;
   CUtensorMap kmap, vmap;
@@ -151,83 +178,258 @@ cudaError_t launch_mma_t(const DecodeParams& p, dim3 grid, cudaStream_t st) {
   if (!tensor_map_encoder()) return cudaErrorNotSupported;
   if (!encode_cache_map(&kmap, p.k_cache, D, rows) || !encode_cache_map(&vmap, p.v_cache, D, rows))
     return cudaErrorInvalidValue;
-  auto kern = pa::decode_mma_kernel<D, NW, ST, SPLIT>;
+  auto kern = pa::decode_mma_kernel<D, NW, ST, SPLIT, APPEND>;
   static std::atomic<uint64_t> smem_done{0};
   cudaError_t e = set_smem(kern, Cfg::kSmemBytes, smem_done);
   if (e != cudaSuccess) return e;
-  kern<<<grid, NW * 32, Cfg::kSmemBytes, st>>>(kmap, vmap, p);
-  return cudaGetLastError();
+  return launch_ex(kern, grid, dim3(NW * 32), Cfg::kSmemBytes, st, false, kmap, vmap, p);
 }
 
-template <bool SPLIT>
+template <bool SPLIT, bool APPEND>
 cudaError_t launch_mma(const DecodeParams& p, dim3 grid, cudaStream_t st) {
   switch (p.head_dim) {
     case 64:
-      return launch_mma_t<64, 4, 4, SPLIT>(p, grid, st);
+      return launch_mma_t<64, 4, 4, SPLIT, APPEND>(p, grid, st);
     case 128:
-      return launch_mma_t<128, 4, 3, SPLIT>(p, grid, st);
+      return launch_mma_t<128, 4, 3, SPLIT, APPEND>(p, grid, st);
     default:
-      return launch_mma_t<256, 2, 3, SPLIT>(p, grid, st);
+      return launch_mma_t<256, 2, 3, SPLIT, APPEND>(p, grid, st);
   }
 }
 
-template <typename T, int D, int GP, bool SPLIT>
+template <typename T, int D, int GP, bool SPLIT, bool APPEND>
 cudaError_t launch_simt_t(const DecodeParams& p, dim3 grid, cudaStream_t st) {
   constexpr int NW = 4;
   const int smem = pa::merge_smem_bytes<NW>(D);
-  auto kern = pa::decode_simt_kernel<T, D, GP, NW, SPLIT>;
+  auto kern = pa::decode_simt_kernel<T, D, GP, NW, SPLIT, APPEND>;
   static std::atomic<uint64_t> smem_done{0};
   cudaError_t e = set_smem(kern, smem, smem_done);
   if (e != cudaSuccess) return e;
-  kern<<<grid, NW * 32, smem, st>>>(p);
-  return cudaGetLastError();
+  return launch_ex(kern, grid, dim3(NW * 32), smem, st, false, p);
 }
 
-template <typename T, int D, bool SPLIT>
+template <typename T, int D, bool SPLIT, bool APPEND>
 cudaError_t launch_simt_d(const DecodeParams& p, dim3 grid, cudaStream_t st) {
   const int G = p.group;
-  if (G <= 1) return launch_simt_t<T, D, 1, SPLIT>(p, grid, st);
-  if (G <= 2) return launch_simt_t<T, D, 2, SPLIT>(p, grid, st);
-  if (G <= 4) return launch_simt_t<T, D, 4, SPLIT>(p, grid, st);
-  return launch_simt_t<T, D, 8, SPLIT>(p, grid, st);
+  if (G <= 1) return launch_simt_t<T, D, 1, SPLIT, APPEND>(p, grid, st);
+  if (G <= 2) return launch_simt_t<T, D, 2, SPLIT, APPEND>(p, grid, st);
+  if (G <= 4) return launch_simt_t<T, D, 4, SPLIT, APPEND>(p, grid, st);
+  return launch_simt_t<T, D, 8, SPLIT, APPEND>(p, grid, st);
 }
 
-template <typename T, bool SPLIT>
+template <typename T, bool SPLIT, bool APPEND>
 cudaError_t launch_simt(const DecodeParams& p, dim3 grid, cudaStream_t st) {
   switch (p.head_dim) {
     case 64:
-      return launch_simt_d<T, 64, SPLIT>(p, grid, st);
+      return launch_simt_d<T, 64, SPLIT, APPEND>(p, grid, st);
     case 128:
-      return launch_simt_d<T, 128, SPLIT>(p, grid, st);
+      return launch_simt_d<T, 128, SPLIT, APPEND>(p, grid, st);
     default:
-      return launch_simt_d<T, 256, SPLIT>(p, grid, st);
+      return launch_simt_d<T, 256, SPLIT, APPEND>(p, grid, st);
   }
 }
 
-template <bool SPLIT>
+template <bool SPLIT, bool APPEND>
 cudaError_t launch_decode(const DecodeParams& p, pa_dtype_t dt, pa_kernel_t kernel, dim3 grid, cudaStream_t st) {
   const bool use_mma = (kernel == PA_KERNEL_MMA) || (kernel == PA_KERNEL_AUTO && dt == PA_BF16);
-  if (use_mma) return launch_mma<SPLIT>(p, grid, st);
-  if (dt == PA_BF16) return launch_simt<__nv_bfloat16, SPLIT>(p, grid, st);
-  return launch_simt<float, SPLIT>(p, grid, st);
+  if (use_mma) return launch_mma<SPLIT, APPEND>(p, grid, st);
+  if (dt == PA_BF16) return launch_simt<__nv_bfloat16, SPLIT, APPEND>(p, grid, st);
+  return launch_simt<float, SPLIT, APPEND>(p, grid, st);
 }
 
-template <typename OutT>
-cudaError_t launch_combine(const DecodeParams& p, cudaStream_t st) {
-  const int smem = (((p.max_parts + 3) & ~3) + pa::kCombineWarps * p.head_dim) * 4;
-  dim3 grid(p.hq, p.batch);
+template <typename OutT, int NWR>
+cudaError_t launch_combine_n(const DecodeParams& p, cudaStream_t st) {
+  constexpr int rows_per_cta = pa::kCombineWarps / NWR;
+  const int rows = p.batch * p.hq;
+  dim3 grid((rows + rows_per_cta - 1) / rows_per_cta);
+  dim3 block(pa::kCombineWarps * 32);
   switch (p.head_dim) {
     case 64:
-      pa::combine_kernel<OutT, 64><<<grid, pa::kCombineWarps * 32, smem, st>>>(p);
-      break;
+      return launch_ex(pa::combine_kernel<OutT, 64, NWR>, grid, block, 0, st, true, p);
     case 128:
-      pa::combine_kernel<OutT, 128><<<grid, pa::kCombineWarps * 32, smem, st>>>(p);
-      break;
+      return launch_ex(pa::combine_kernel<OutT, 128, NWR>, grid, block, 0, st, true, p);
     default:
-      pa::combine_kernel<OutT, 256><<<grid, pa::kCombineWarps * 32, smem, st>>>(p);
-      break;
+      return launch_ex(pa::combine_kernel<OutT, 256, NWR>, grid, block, 0, st, true, p);
   }
-  return cudaGetLastError();
+}
+
+// One warp per row when rows have few partitions; eight when they have many.
+template <typename OutT>
+cudaError_t launch_combine(const DecodeParams& p, cudaStream_t st) {
+  return p.max_parts > 16 ? launch_combine_n<OutT, 8>(p, st) : launch_combine_n<OutT, 1>(p, st);
+}
+
+int sm_count() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev < 64) {
+    const int v = cache[dev].load(std::memory_order_relaxed);
+    if (v > 0) return v;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  if (dev < 64) cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+// Opt in to `bytes` of dynamic shared memory (growing only), once per device
+// and size, for kernels whose size depends on the launch.
+template <typename Kernel>
+cudaError_t set_smem_at_least(Kernel k, int bytes, std::atomic<int>* done /* [64] */) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 64 && done[dev].load(std::memory_order_acquire) >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev < 64) {
+    int cur = done[dev].load(std::memory_order_acquire);
+    while (cur < bytes && !done[dev].compare_exchange_weak(cur, bytes)) {
+    }
+  }
+  return e;
+}
+
+template <int D, int NW, int ST, bool APPEND>
+cudaError_t launch_dynamic_t(const DecodeParams& p, cudaStream_t st) {
+  using Cfg = pa::DynCfg<D, NW, ST>;
+  CUtensorMap kmap, vmap;
+  const long long rows = (long long)p.num_blocks * p.hkv * p.block_size;
+  if (!tensor_map_encoder()) return cudaErrorNotSupported;
+  if (!encode_cache_map(&kmap, p.k_cache, D, rows) || !encode_cache_map(&vmap, p.v_cache, D, rows))
+    return cudaErrorInvalidValue;
+  auto kern = pa::decode_dynamic_kernel<D, NW, ST, APPEND>;
+  const int smem = Cfg::smem_bytes(p.group, p.batch);
+  static std::atomic<int> smem_done[64];
+  cudaError_t e = set_smem_at_least(kern, smem, smem_done);
+  if (e != cudaSuccess) return e;
+  int occ = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, Cfg::kThreads, smem);
+  if (e != cudaSuccess) return e;
+  if (occ < 1) return cudaErrorInvalidConfiguration;
+  return launch_ex(kern, dim3(occ * sm_count()), dim3(Cfg::kThreads), smem, st, false, kmap, vmap, p);
+}
+
+template <bool APPEND>
+cudaError_t launch_dynamic(const DecodeParams& p, cudaStream_t st) {
+  switch (p.head_dim) {
+    // Warps x stages per CTA, from a sweep on B200: several small CTAs per SM
+    // beat one deep ring (their merges and item switches overlap).
+    case 64:
+      return launch_dynamic_t<64, 4, 3, APPEND>(p, st);
+    case 128:
+      return launch_dynamic_t<128, 4, 2, APPEND>(p, st);
+    default:
+      return launch_dynamic_t<256, 3, 2, APPEND>(p, st);
+  }
+}
+
+int32_t auto_partition(int32_t batch, int32_t num_kv_heads, int32_t max_context_len, int32_t partition_tokens) {
+  if (partition_tokens > 0) return partition_tokens;
+  const long long work = (long long)(batch > 0 ? batch : 1) * (num_kv_heads > 0 ? num_kv_heads : 1) *
+                         (max_context_len > 0 ? max_context_len : 1);
+  int P = 512;
+  while (P > 64 && work / P < kTargetWorkUnits) P >>= 1;
+  return P;
+}
+
+long long splitk_parts(int32_t max_context_len, int32_t P) {
+  return ((long long)(max_context_len > 0 ? max_context_len : 1) + P - 1) / P;
+}
+
+size_t workspace_size(int32_t batch, int32_t num_q_heads, int32_t head_dim, int32_t max_context_len, int32_t P) {
+  const size_t rows = (size_t)batch * num_q_heads * (size_t)splitk_parts(max_context_len, P);
+  return align256(rows * head_dim * 4) + align256(rows * 2 * 4);
+}
+
+// Everything the decode entry points share.  split: partitioned launch plus
+// the combine; append: the fused decode step (k_new / v_new appended at L-1).
+struct DecodeCall {
+  const void* q;
+  const void* k_new;
+  const void* v_new;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  Shape shape;
+  float scale, softcap;
+  int32_t window;
+  void* out;
+  pa_dtype_t dtype;
+  bool split, append;
+  int32_t partition_tokens, max_context_len;
+  void* workspace;
+  size_t workspace_bytes;
+  pa_kernel_t kernel;
+  cudaStream_t stream;
+};
+
+pa_status_t run_decode(const DecodeCall& c) {
+  const Shape& s = c.shape;
+  pa_status_t st = check_decode_args(c.q, c.k_cache, c.v_cache, c.block_tables, c.context_lens, s, c.softcap,
+                                     c.out, c.dtype, c.kernel);
+  if (st != PA_OK) return st;
+  if (c.append && s.batch > 0) {
+    if (!c.k_new || !c.v_new || !aligned(c.k_new, 16) || !aligned(c.v_new, 16)) return PA_ERR_INVALID;
+  }
+  int P = kNoSplitPartition;
+  long long parts = 1;
+  bool dynamic = false;
+  if (c.split) {
+    if (c.partition_tokens < 0 || (c.partition_tokens > 0 && c.partition_tokens % 64 != 0)) return PA_ERR_INVALID;
+    if (c.max_context_len <= 0) return PA_ERR_INVALID;
+    const bool mma = (c.kernel == PA_KERNEL_MMA) || (c.kernel == PA_KERNEL_AUTO && c.dtype == PA_BF16);
+    dynamic = c.partition_tokens == 0 && mma && s.batch <= pa::kMaxDynamicBatch;
+    P = auto_partition(s.batch, s.hkv, c.max_context_len, c.partition_tokens);
+    parts = splitk_parts(c.max_context_len, P);
+    if (parts > kMaxPartsPerSeq) return PA_ERR_UNSUPPORTED;
+    const size_t need = workspace_size(s.batch, s.hq, s.d, c.max_context_len, P) + (dynamic ? kQueueBytes : 0);
+    if (s.batch > 0 && (!c.workspace || !aligned(c.workspace, 16) || c.workspace_bytes < need))
+      return PA_ERR_WORKSPACE;
+  }
+  if (s.batch == 0) return PA_OK;
+
+  DecodeParams p = make_params(c.q, c.k_cache, c.v_cache, c.block_tables, c.context_lens, s, c.scale, c.softcap,
+                               c.window, c.out);
+  p.k_new = c.k_new;
+  p.v_new = c.v_new;
+  cudaError_t e;
+  if (c.split) {
+    p.partition = P;
+    p.max_parts = (int)parts;
+    p.max_context = c.max_context_len < p.max_context ? c.max_context_len : p.max_context;
+    const size_t rows = (size_t)s.batch * s.hq * parts;
+    p.ws_o = static_cast<float*>(c.workspace);
+    p.ws_ml = reinterpret_cast<float*>(static_cast<char*>(c.workspace) + align256(rows * s.d * 4));
+    if (dynamic) {
+      p.dynamic = 1;
+      p.queue = reinterpret_cast<int*>(static_cast<char*>(c.workspace) +
+                                       workspace_size(s.batch, s.hq, s.d, c.max_context_len, P));
+      e = c.append ? launch_dynamic<true>(p, c.stream) : launch_dynamic<false>(p, c.stream);
+    } else {
+      dim3 grid((unsigned)parts, s.hkv, s.batch);
+      e = c.append ? launch_decode<true, true>(p, c.dtype, c.kernel, grid, c.stream)
+                   : launch_decode<true, false>(p, c.dtype, c.kernel, grid, c.stream);
+    }
+    if (e != cudaSuccess) return PA_ERR_CUDA;
+    // The dynamic schedule always runs the combine: it resets the work counter.
+    if (parts > 1 || dynamic) {
+      e = c.dtype == PA_BF16 ? launch_combine<__nv_bfloat16>(p, c.stream) : launch_combine<float>(p, c.stream);
+      if (e != cudaSuccess) return PA_ERR_CUDA;
+      t_last_launches = 2;
+    } else {
+      t_last_launches = 1;
+    }
+  } else {
+    dim3 grid(1, s.hkv, s.batch);
+    e = c.append ? launch_decode<false, true>(p, c.dtype, c.kernel, grid, c.stream)
+                 : launch_decode<false, false>(p, c.dtype, c.kernel, grid, c.stream);
+    if (e != cudaSuccess) return PA_ERR_CUDA;
+    t_last_launches = 1;
+  }
+  return PA_OK;
 }
 
 }  // namespace
@@ -267,41 +469,36 @@ pa_status_t pa_decode(const void* q, const void* k_cache, const void* v_cache, c
                       float scale, float softcap, int32_t window, void* out, pa_dtype_t dtype,
                       pa_kernel_t kernel, pa_stream_t stream) {
   t_last_launches = 0;
-  const Shape s{batch, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks};
-  pa_status_t st = check_decode_args(q, k_cache, v_cache, block_tables, context_lens, s, softcap, out, dtype, kernel);
-  if (st != PA_OK) return st;
-  if (batch == 0) return PA_OK;
-  DecodeParams p = make_params(q, k_cache, v_cache, block_tables, context_lens, s, scale, softcap, window, out);
-  dim3 grid(1, num_kv_heads, batch);
-  if (launch_decode<false>(p, dtype, kernel, grid, stream) != cudaSuccess) return PA_ERR_CUDA;
-  t_last_launches = 1;
-  return PA_OK;
+  DecodeCall c{};
+  c.q = q;
+  c.k_cache = k_cache;
+  c.v_cache = v_cache;
+  c.block_tables = block_tables;
+  c.context_lens = context_lens;
+  c.shape = Shape{batch, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks};
+  c.scale = scale;
+  c.softcap = softcap;
+  c.window = window;
+  c.out = out;
+  c.dtype = dtype;
+  c.kernel = kernel;
+  c.stream = stream;
+  return run_decode(c);
 }
 
 int32_t pa_decode_splitk_partition(int32_t batch, int32_t num_kv_heads, int32_t max_context_len,
                                    int32_t partition_tokens) {
-  if (partition_tokens > 0) return partition_tokens;
-  const long long work = (long long)(batch > 0 ? batch : 1) * (num_kv_heads > 0 ? num_kv_heads : 1) *
-                         (max_context_len > 0 ? max_context_len : 1);
-  int P = 512;
-  while (P > 64 && work / P < kTargetWorkUnits) P >>= 1;
-  return P;
+  return auto_partition(batch, num_kv_heads, max_context_len, partition_tokens);
 }
-
-static long long splitk_parts(int32_t max_context_len, int32_t P) {
-  return ((long long)(max_context_len > 0 ? max_context_len : 1) + P - 1) / P;
-}
-
-static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 size_t pa_decode_splitk_workspace_size(int32_t batch, int32_t num_q_heads, int32_t head_dim,
                                        int32_t max_context_len, int32_t partition_tokens,
                                        int32_t num_kv_heads) {
   if (batch <= 0 || num_q_heads <= 0 || head_dim <= 0) return 0;
-  const int P = pa_decode_splitk_partition(batch, num_kv_heads, max_context_len, partition_tokens);
+  const int P = auto_partition(batch, num_kv_heads, max_context_len, partition_tokens);
   if (P <= 0) return 0;
-  const size_t rows = (size_t)batch * num_q_heads * (size_t)splitk_parts(max_context_len, P);
-  return align256(rows * head_dim * 4) + align256(rows * 2 * 4);
+  // partition_tokens == 0 may select the dynamic schedule, which adds its work counter.
+  return workspace_size(batch, num_q_heads, head_dim, max_context_len, P) + (partition_tokens == 0 ? kQueueBytes : 0);
 }
 
 pa_status_t pa_decode_splitk(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
@@ -312,36 +509,59 @@ pa_status_t pa_decode_splitk(const void* q, const void* k_cache, const void* v_c
                              int32_t max_context_len, void* workspace, size_t workspace_bytes,
                              pa_kernel_t kernel, pa_stream_t stream) {
   t_last_launches = 0;
-  const Shape s{batch, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks};
-  pa_status_t st = check_decode_args(q, k_cache, v_cache, block_tables, context_lens, s, softcap, out, dtype, kernel);
-  if (st != PA_OK) return st;
-  if (partition_tokens < 0 || (partition_tokens > 0 && partition_tokens % 64 != 0)) return PA_ERR_INVALID;
-  if (max_context_len <= 0) return PA_ERR_INVALID;
-  if (batch == 0) return PA_OK;
-  const int P = pa_decode_splitk_partition(batch, num_kv_heads, max_context_len, partition_tokens);
-  const long long parts = splitk_parts(max_context_len, P);
-  if (parts > kMaxPartsPerSeq) return PA_ERR_UNSUPPORTED;
-  const size_t need = pa_decode_splitk_workspace_size(batch, num_q_heads, head_dim, max_context_len, P, num_kv_heads);
-  if (!workspace || !aligned(workspace, 16) || workspace_bytes < need) return PA_ERR_WORKSPACE;
+  DecodeCall c{};
+  c.q = q;
+  c.k_cache = k_cache;
+  c.v_cache = v_cache;
+  c.block_tables = block_tables;
+  c.context_lens = context_lens;
+  c.shape = Shape{batch, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks};
+  c.scale = scale;
+  c.softcap = softcap;
+  c.window = window;
+  c.out = out;
+  c.dtype = dtype;
+  c.split = true;
+  c.partition_tokens = partition_tokens;
+  c.max_context_len = max_context_len;
+  c.workspace = workspace;
+  c.workspace_bytes = workspace_bytes;
+  c.kernel = kernel;
+  c.stream = stream;
+  return run_decode(c);
+}
 
-  DecodeParams p = make_params(q, k_cache, v_cache, block_tables, context_lens, s, scale, softcap, window, out);
-  p.partition = P;
-  p.max_parts = (int)parts;
-  p.max_context = max_context_len < p.max_context ? max_context_len : p.max_context;
-  const size_t rows = (size_t)batch * num_q_heads * parts;
-  p.ws_o = static_cast<float*>(workspace);
-  p.ws_ml = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(rows * head_dim * 4));
-
-  dim3 grid((unsigned)parts, num_kv_heads, batch);
-  if (launch_decode<true>(p, dtype, kernel, grid, stream) != cudaSuccess) return PA_ERR_CUDA;
-  if (parts > 1) {
-    cudaError_t e = dtype == PA_BF16 ? launch_combine<__nv_bfloat16>(p, stream) : launch_combine<float>(p, stream);
-    if (e != cudaSuccess) return PA_ERR_CUDA;
-    t_last_launches = 2;
-  } else {
-    t_last_launches = 1;
-  }
-  return PA_OK;
+pa_status_t pa_decode_step(const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+                           const int32_t* block_tables, const int32_t* context_lens, int32_t batch,
+                           int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                           int32_t max_blocks_per_seq, int32_t num_blocks, float scale, float softcap,
+                           int32_t window, void* out, pa_dtype_t dtype, int32_t partition_tokens,
+                           int32_t max_context_len, void* workspace, size_t workspace_bytes, pa_kernel_t kernel,
+                           pa_stream_t stream) {
+  t_last_launches = 0;
+  DecodeCall c{};
+  c.q = q;
+  c.k_new = k_new;
+  c.v_new = v_new;
+  c.k_cache = k_cache;
+  c.v_cache = v_cache;
+  c.block_tables = block_tables;
+  c.context_lens = context_lens;
+  c.shape = Shape{batch, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks};
+  c.scale = scale;
+  c.softcap = softcap;
+  c.window = window;
+  c.out = out;
+  c.dtype = dtype;
+  c.append = true;
+  c.split = partition_tokens >= 0;
+  c.partition_tokens = partition_tokens;
+  c.max_context_len = max_context_len;
+  c.workspace = workspace;
+  c.workspace_bytes = workspace_bytes;
+  c.kernel = kernel;
+  c.stream = stream;
+  return run_decode(c);
 }
 
 pa_status_t pa_device_errors(uint32_t* bits, int32_t clear) {

@@ -152,7 +152,7 @@ def test_context_of_length_one_returns_v_exactly(dtype, d):
 
 
 def test_zero_length_context_gives_zero_rows():
-    w, b_cpu, b = _reduced("tinyllama_1b")
+    w, b_cpu, b = _reduced("tinyllama_1b", prefilled=True)
     cl = b.context_lens.clone()
     cl[3] = 0
     for split in (False, True):
@@ -284,3 +284,155 @@ def test_full_size_sampled_rows(name):
                         rows=rows)
     got = torch.stack([out[i, h] for i, h in rows])
     assert_close(got, ref, w.torch_dtype, f"{name} full size, sampled rows")
+
+
+# ---- fused decode step ------------------------------------------------------------
+
+
+@pytest.mark.parametrize("name", list(wl.WORKLOADS))
+@pytest.mark.parametrize("split", [False, True])
+@pytest.mark.parametrize("kernel", ["auto", "cuda_core"])
+def test_fused_step_equals_append_then_decode_bit_for_bit(name, split, kernel):
+    w, b_cpu, b = _reduced(name)
+    ref_out, ref_kc, ref_vc = gpu_step(b, kernel=kernel, split=split, partition=w.partition_tokens)
+    kc, vc = b.k_cache.clone(), b.v_cache.clone()
+    out = pa.decode_step(b.q, b.k_new, b.v_new, kc, vc, b.block_tables, b.context_lens, w.scale, w.softcap,
+                         w.window, split=split, max_context_len=max(1, b.max_context_len),
+                         partition_tokens=w.partition_tokens, kernel=kernel)
+    torch.cuda.synchronize()
+    assert torch.equal(bits(out), bits(ref_out))
+    assert torch.equal(bits(kc), bits(ref_kc)) and torch.equal(bits(vc), bits(ref_vc))
+    ref, _, _ = oracle_step(b_cpu)
+    assert_close(out, ref, w.torch_dtype, f"fused step {name} split={split} kernel={kernel}")
+    assert pa.device_errors() == 0
+
+
+@pytest.mark.parametrize("window", [0, 1, 100])
+def test_fused_step_with_window_and_softcap(window):
+    w, b_cpu, b = _reduced("gemma2_2b")
+    kc, vc = b.k_cache.clone(), b.v_cache.clone()
+    out = pa.decode_step(b.q, b.k_new, b.v_new, kc, vc, b.block_tables, b.context_lens, w.scale, w.softcap, window,
+                         split=True, max_context_len=b.max_context_len, partition_tokens=128)
+    torch.cuda.synchronize()
+    ref, kc_ref, vc_ref = oracle_step(b_cpu, window=window)
+    assert torch.equal(bits(kc), bits(kc_ref)) and torch.equal(bits(vc), bits(vc_ref))
+    assert_close(out, ref, torch.bfloat16, f"fused step window={window}")
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_fused_step_sampled_rows(name):
+    w = wl.WORKLOADS[name]
+    b = wl.make_batch(w, device="cuda")
+    cpu = dict(q=b.q.cpu(), k_new=b.k_new.cpu(), v_new=b.v_new.cpu(), slots=b.slot_mapping.cpu(),
+               kc=b.k_cache.cpu(), vc=b.v_cache.cpu(), tables=b.block_tables.cpu(), lens=b.context_lens.cpu())
+    part = pa.decode_splitk_partition(w.batch, w.num_kv_heads, b.max_context_len, w.partition_tokens)
+    out = pa.decode_step(b.q, b.k_new, b.v_new, b.k_cache, b.v_cache, b.block_tables, b.context_lens, w.scale,
+                         w.softcap, w.window, split=True, max_context_len=b.max_context_len, partition_tokens=part)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all()
+    assert pa.device_errors() == 0
+    oracle.write_kv(cpu["k_new"], cpu["v_new"], cpu["slots"], cpu["kc"], cpu["vc"])
+    # The appended rows landed bit-exactly.
+    L = cpu["lens"]
+    bs = w.block_size
+    for i in range(0, w.batch, max(1, w.batch // 16)):
+        t = int(L[i]) - 1
+        blk = int(cpu["tables"][i, t // bs])
+        assert torch.equal(bits(b.k_cache[blk, :, t % bs]), bits(cpu["k_new"][i]))
+        assert torch.equal(bits(b.v_cache[blk, :, t % bs]), bits(cpu["v_new"][i]))
+    g = torch.Generator().manual_seed(7)
+    rows = [(int(i), int(h)) for i, h in zip(torch.randint(0, w.batch, (48,), generator=g),
+                                             torch.randint(0, w.num_q_heads, (48,), generator=g))]
+    rows += [(int(L.argmax()), 1), (int(L.argmin()), 0)]
+    ref = oracle.decode(cpu["q"], cpu["kc"], cpu["vc"], cpu["tables"], cpu["lens"], w.scale, w.softcap, w.window,
+                        rows=rows)
+    got = torch.stack([out[i, h] for i, h in rows])
+    assert_close(got, ref, w.torch_dtype, f"{name} full-size fused step")
+
+
+# ---- dynamic (work-queue) split-K schedule ------------------------------------------
+# partition_tokens == 0 on the tensor-core path: persistent CTAs claim
+# (sequence, kv head, partition) items from a counter in the workspace.
+
+
+@pytest.mark.parametrize("name", ["tinyllama_1b", "gemma2_2b", "llama3_8b", "long_splitk"])
+@pytest.mark.parametrize("append", [False, True])
+def test_dynamic_schedule_parity(name, append):
+    w, b_cpu, b = _reduced(name)
+    kc, vc = b.k_cache.clone(), b.v_cache.clone()
+    if append:
+        out = pa.decode_step(b.q, b.k_new, b.v_new, kc, vc, b.block_tables, b.context_lens, w.scale, w.softcap,
+                             w.window, split=True, max_context_len=b.max_context_len, partition_tokens=0)
+    else:
+        pa.write_kv(b.k_new, b.v_new, b.slot_mapping, kc, vc)
+        out = pa.decode_splitk(b.q, kc, vc, b.block_tables, b.context_lens, w.scale, w.softcap, w.window,
+                               max_context_len=b.max_context_len, partition_tokens=0)
+    torch.cuda.synchronize()
+    ref, kc_ref, vc_ref = oracle_step(b_cpu)
+    assert torch.equal(bits(kc), bits(kc_ref)) and torch.equal(bits(vc), bits(vc_ref))
+    assert_close(out, ref, w.torch_dtype, f"dynamic {name} append={append}")
+    assert pa.device_errors() == 0
+
+
+@pytest.mark.parametrize("lengths", [[1, 2, 3], [0, 5, 0, 17], [1] * 40, [16, 32, 48, 64, 15, 17, 31, 33]])
+def test_dynamic_schedule_short_and_empty_sequences(lengths):
+    """Fewer items than CTAs, L = 0 rows, single-slice items."""
+    w = wl.WORKLOADS["llama3_8b"].replace(prefix_share=0.0)
+    b_cpu = wl.make_batch(w, lengths=lengths, prefilled=True)
+    b = to_dev(b_cpu)
+    out = pa.decode_splitk(b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, w.scale,
+                           max_context_len=max(1, max(lengths)), partition_tokens=0)
+    torch.cuda.synchronize()
+    ref, _, _ = oracle_step(b_cpu, append=False)
+    assert_close(out, ref, torch.bfloat16, f"dynamic lengths={lengths}")
+    for i, L in enumerate(lengths):
+        if L == 0:
+            assert torch.count_nonzero(out[i]).item() == 0
+
+
+def test_dynamic_schedule_many_units_per_cta():
+    """Many short sequences: thousands of items, prefix arrays of a large batch."""
+    w = wl.WORKLOADS["llama3_8b"].replace(prefix_share=0.0, lengths=("uniform", 1, 40))
+    b_cpu = wl.make_batch(w, batch=2000, prefilled=True)
+    b = to_dev(b_cpu)
+    out = pa.decode_splitk(b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, w.scale,
+                           max_context_len=b.max_context_len, partition_tokens=0)
+    torch.cuda.synchronize()
+    rows = [(i, h) for i in range(0, 2000, 37) for h in (0, 13, 31)]
+    ref = oracle.decode(b_cpu.q, b_cpu.k_cache, b_cpu.v_cache, b_cpu.block_tables, b_cpu.context_lens, w.scale,
+                        rows=rows)
+    got = torch.stack([out[i, h] for i, h in rows])
+    assert_close(got, ref, torch.bfloat16, "dynamic, many items per CTA")
+    assert pa.device_errors() == 0
+
+
+def test_dynamic_schedule_block_permutation_invariance_and_workspace_reuse():
+    w, b_cpu, b = _reduced("llama3_8b", prefilled=True)
+    need = pa.decode_splitk_workspace_size(b.q.shape[0], w.num_q_heads, w.head_dim, b.max_context_len, 0,
+                                           w.num_kv_heads)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")  # one workspace for every call
+    kw = dict(max_context_len=b.max_context_len, partition_tokens=0, workspace=ws)
+    base = pa.decode_splitk(b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, w.scale, **kw)
+    again = pa.decode_splitk(b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, w.scale, **kw)
+    nb = b.k_cache.shape[0]
+    perm = torch.randperm(nb, generator=torch.Generator().manual_seed(9)).cuda()
+    kc2, vc2 = torch.empty_like(b.k_cache), torch.empty_like(b.v_cache)
+    kc2[perm] = b.k_cache
+    vc2[perm] = b.v_cache
+    t2 = b.block_tables.clone()
+    m = t2 >= 0
+    t2[m] = perm[t2[m].long()].to(torch.int32)
+    moved = pa.decode_splitk(b.q, kc2, vc2, t2, b.context_lens, w.scale, **kw)
+    torch.cuda.synchronize()
+    assert torch.equal(bits(base), bits(again))
+    assert torch.equal(bits(base), bits(moved))
+
+
+@pytest.mark.parametrize("window", [1, 100, 1000])
+def test_dynamic_schedule_window(window):
+    w, b_cpu, b = _reduced("tinyllama_1b", prefilled=True)
+    out = pa.decode_splitk(b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, w.scale, 0.0, window,
+                           max_context_len=b.max_context_len, partition_tokens=0)
+    torch.cuda.synchronize()
+    ref, _, _ = oracle_step(b_cpu, window=window, append=False)
+    assert_close(out, ref, torch.bfloat16, f"dynamic window={window}")
