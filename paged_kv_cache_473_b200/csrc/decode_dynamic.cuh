@@ -1,26 +1,27 @@
 // Paged decode attention, bf16, tensor cores: the dynamic (work-queue) split-K
-// schedule.
+// schedule, one work item per warp.
 //
 // Work items are the non-empty (sequence b, kv head g, partition) triples of
 // the split-K decomposition: partition p of sequence b covers tokens
 // [p*P, p*P + P) of its attended range [s0, L).  The grid is persistent (as
-// many CTAs as fit on the GPU at once); every CTA claims items one at a time
-// from a counter in the workspace (atomicAdd), so CTAs on SMs that stream
-// faster simply take more items and all finish together.  Items are numbered
-// sequence-major: every CTA first builds, with block-wide scans over
-// context_lens, the number of items before each sequence, and decodes an item
-// number with a binary search in shared memory.
+// many CTAs as fit on the GPU at once) and every WARP claims items on its own
+// from a counter in the workspace (atomicAdd; the first two items of each warp
+// are fixed by its index), so warps on SMs that stream faster take more items
+// and the whole GPU finishes together.  A warp runs an
+// item alone: it streams the item's 16-token slices through its own ST-deep
+// ring of TMA-filled shared-memory stages, keeps the online-softmax state in
+// registers (attend_slice), and at the end writes either the normalised output
+// (the item is the sequence's only partition) or its partial state (m, l, o)
+// to the [B][Hq][max_parts] workspace, straight from registers.  No barrier
+// joins the warps of a CTA after the prologue, so an SM holds many independent
+// streams of loads.  Each warp claims two items ahead and its load cursor runs
+// into the next item before the current one is finished, so its ring stays
+// full across item boundaries.
 //
-// Inside a CTA, warp w takes the item's 16-token slices k with k mod NW == w
-// and runs its own ST-deep ring of TMA-filled stages (as the grid-scheduled
-// kernel does).  The next item is claimed while the current one is processed,
-// so a warp whose share of the current item is issued already loads the next
-// item's slices while the CTA merges the current one: the ring stays full
-// across item boundaries.  At the end of each item the warps merge their
-// softmax states through shared memory; items that cover a whole sequence
-// range are normalised and written, the others leave their partial state in
-// the [B][Hq][max_parts] workspace for the combine kernel, which also resets
-// the counter for the next call.
+// Items are numbered sequence-major; each CTA first builds, with block-wide
+// scans over context_lens, the number of items before each sequence and
+// decodes an item number with a binary search in shared memory.  The combine
+// kernel merges the partials and resets the counter for the next call.
 //
 // APPEND (the fused decode step): the item that ends at the sequence's last
 // token writes the step's new key/value row to the cache slot of position L-1
@@ -56,10 +57,6 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int& to
   return before + incl - v;
 }
 
-__device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
 // Partitions of sequence b's attended range [s0, L) (0 when it is empty).
 __device__ __forceinline__ int seq_parts(int L, int s0, int P) { return L > s0 ? (L + P - 1) / P - s0 / P : 0; }
 
@@ -76,16 +73,11 @@ struct DynCfg {
   static constexpr int kSliceBytes = SliceBytes<D>::kSlice;
   static constexpr int kRingBytes = NW * ST * kStageBytes;
   static constexpr int kThreads = NW * 32;
-  // After the 1024-aligned ring: barriers, claim slots, scratch, merge buffer, prefix arrays.
+  // After the 1024-aligned ring: barriers, scan scratch, prefix arrays.
   static constexpr int kBarOffset = kRingBytes;
-  static constexpr int kSlotOffset = kBarOffset + NW * ST * 8;  // 2 x {seq, item}
-  static constexpr int kScratchOffset = kSlotOffset + 16;
-  static constexpr int kMergeOffset = kScratchOffset + 32 * 4;
-  static __host__ __device__ constexpr int merge_bytes(int G) { return merge_smem_bytes<NW>(D, G); }
-  static __host__ __device__ constexpr int prefix_offset(int G) { return kMergeOffset + merge_bytes(G); }
-  static __host__ __device__ constexpr int smem_bytes(int G, int B) {
-    return prefix_offset(G) + (2 * B + 1) * 4 + 1024;
-  }
+  static constexpr int kScratchOffset = kBarOffset + NW * ST * 8;
+  static constexpr int kPrefixOffset = kScratchOffset + 32 * 4;
+  static __host__ __device__ constexpr int smem_bytes(int B) { return kPrefixOffset + (2 * B + 1) * 4 + 1024; }
 };
 
 template <int D, int NW, int ST, bool APPEND>
@@ -97,18 +89,19 @@ __global__ void __launch_bounds__(NW * 32)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int G = p.group, Hkv = p.hkv, P = p.partition, B = p.batch;
-  volatile int* slots = reinterpret_cast<volatile int*>(smem + Cfg::kSlotOffset);  // [2][{seq, item}]
-  int* scratch = reinterpret_cast<int*>(smem + Cfg::kScratchOffset);  // [0, 31): scans; [31]: abort flag
-  volatile int* cta_abort = scratch + 31;
-  const MergeSmem ms = merge_smem<NW>(smem + Cfg::kMergeOffset, D, G);
-  int* pre = reinterpret_cast<int*>(smem + Cfg::prefix_offset(G));  // [B+1] items before sequence b
-  int* lens = pre + B + 1;                                           // [B] clamped context lengths
+  int* scratch = reinterpret_cast<int*>(smem + Cfg::kScratchOffset);
+  int* pre = reinterpret_cast<int*>(smem + Cfg::kPrefixOffset);  // [B+1] items before sequence b
+  int* lens = pre + B + 1;                                        // [B] clamped context lengths
 
   pdl_launch_dependents();  // the combine kernel may launch now; it waits for this grid to finish
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
   const uint32_t ring = smem_addr(smem) + warp * ST * Cfg::kStageBytes;
   const uint32_t bars = smem_addr(smem + Cfg::kBarOffset) + warp * ST * 8;
+  // A warp's first two items are fixed by its index (W warps in the grid: items
+  // w and W + w); later ones are claimed from the counter, offset by 2W, so the
+  // launch does not start with every warp contending for one address.
+  const int W = gridDim.x * NW, wg = blockIdx.x * NW + warp;
   if (lane == 0) {
 #pragma unroll
     for (int s = 0; s < ST; ++s) mbar_init(bars + 8 * s, 1);
@@ -116,8 +109,6 @@ __global__ void __launch_bounds__(NW * 32)
     if (warp == 0) {
       prefetch_tensormap(&kmap);
       prefetch_tensormap(&vmap);
-      slots[2] = -1;  // claim slot 1 holds no item yet
-      *cta_abort = 0;
     }
   }
 
@@ -136,12 +127,7 @@ __global__ void __launch_bounds__(NW * 32)
     if (b < B) pre[b] = base + ex;
     base += total;
   }
-  if (tid == 0) {
-    pre[B] = base;
-    slots[1] = atomicAdd(p.queue, 1);  // the first item
-    __threadfence_block();
-    slots[0] = 0;
-  }
+  if (tid == 0) pre[B] = base;
   __syncthreads();
   const int T = pre[B];
 
@@ -168,25 +154,25 @@ __global__ void __launch_bounds__(NW * 32)
     it.whole = parts == 1;
     return it;
   };
-  // This warp's share of an item's slices: k = warp, warp + NW, ...
-  auto share = [&](const Item& it) { return it.n > warp ? (it.n - warp + NW - 1) / NW : 0; };
 
-  int s = 0;  // item sequence number within this CTA
-  int t_cur = slots[1];
-  if (t_cur >= T) return;  // nothing issued yet: safe to leave
+  int t_cur = wg;       // item being computed
+  int t_next = W + wg;  // item after it
+  if (t_cur >= T) return;  // nothing issued: safe to leave
+  int t_claim = 0;         // lane 0: the claim after t_next, in flight
+  if (lane == 0 && t_next < T) t_claim = 2 * W + atomicAdd(p.queue, 1);
 
   Item ci = decode(t_cur);
-  int cn = share(ci);
-  // Issue cursor: item `ii` (sequence number i_seq), slice index ik of in_.
+  // Load cursor: slice ik of item ii (ii == ci, or the next item once ci is fully issued).
   Item ii = ci;
-  int in_ = cn, ik = 0, i_seq = 0;
-  int gi = 0, gc = 0;  // slices issued / consumed by this warp (ring position)
-  int yrow = -1;       // cache rows of the issue item's warp-slices [kbatch, kbatch + 32), one per lane
+  int ik = 0;
+  bool i_in_next = false;
+  int gi = 0, gc = 0;  // slices issued / consumed (ring position)
+  int yrow = -1;       // cache rows of the load item's slices [kbatch, kbatch + 32), one per lane
   auto load_rows = [&](const Item& it, int base_k) {
-    const int i = base_k + lane;
+    const int k = base_k + lane;
     yrow = -1;
-    if (i < share(it)) {
-      const int t = (it.j0 + warp + NW * i) * kSliceTokens;
+    if (k < it.n) {
+      const int t = (it.j0 + k) * kSliceTokens;
       const int phys = p.block_tables[(size_t)it.b * p.max_blocks + (t >> p.log2_bs)];
       if (phys >= 0 && phys < p.num_blocks) yrow = cache_row(p, phys, it.g, t);
     }
@@ -196,29 +182,14 @@ __global__ void __launch_bounds__(NW * 32)
   const __nv_bfloat16* q0 = static_cast<const __nv_bfloat16*>(p.q);
   load_q_frags<D>(qf, q0 + ((size_t)ci.b * p.hq + (size_t)ci.g * G) * D, G, lane);
 
-  bool abort = false;
-  // Fill this warp's ring from the issue cursor; moves into the claimed next
-  // item once its number is published.  Warp-uniform.
-  auto try_issue = [&]() {
-    while (!abort && gi - gc < ST) {
-      if (ik >= in_) {
-        if (i_seq != s) return;  // already in the next item, which is fully issued
-        int seq_n = 0, t_n = 0;
-        if (lane == 0) {
-          seq_n = slots[2 * ((s + 1) & 1)];
-          t_n = slots[2 * ((s + 1) & 1) + 1];
-        }
-        seq_n = __shfl_sync(FULL, seq_n, 0);
-        t_n = __shfl_sync(FULL, t_n, 0);
-        if (seq_n != s + 1) return;  // the next claim is not published yet
-        i_seq = s + 1;
+  // Keep ST slices in flight: finish the current item's loads, then run into the next item.
+  auto fill = [&]() {
+    while (gi - gc < ST) {
+      if (ik >= ii.n) {
+        if (i_in_next || t_next >= T) return;
+        ii = decode(t_next);
         ik = 0;
-        if (t_n >= T) {
-          in_ = 0;
-          return;
-        }
-        ii = decode(t_n);
-        in_ = share(ii);
+        i_in_next = true;
         load_rows(ii, 0);
         load_q_frags<D>(qf_next, q0 + ((size_t)ii.b * p.hq + (size_t)ii.g * G) * D, G, lane);
         continue;
@@ -234,17 +205,8 @@ __global__ void __launch_bounds__(NW * 32)
   WarpAttn<D> st;
   st.reset();
   const float qk_scale = p.use_softcap ? p.scale : p.scale * kLog2e;
-  int t_next = 0;
-  if (tid == 0) t_next = atomicAdd(p.queue, 1);  // claim the next item early
-  bool published = false;
-  auto publish = [&]() {  // thread 0: make the claimed number visible as item s+1
-    if (tid == 0 && !published) {
-      slots[2 * ((s + 1) & 1) + 1] = t_next;
-      __threadfence_block();
-      slots[2 * ((s + 1) & 1)] = s + 1;
-      published = true;
-    }
-  };
+  const int n0 = 2 * (lane & 3);
+  bool aborted = false;
 
   while (true) {
     uint4 knew = make_uint4(0, 0, 0, 0), vnew = make_uint4(0, 0, 0, 0);
@@ -254,23 +216,17 @@ __global__ void __launch_bounds__(NW * 32)
       knew = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.k_new) + off);
       vnew = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.v_new) + off);
     }
-    for (int ck = 0; ck < cn; ++ck) {
-      try_issue();
-      bool ok = !abort && mbar_wait_bounded(bars + 8 * (gc % ST), (gc / ST) & 1, kWaitLimitNs);
+    for (int ck = 0; ck < ci.n; ++ck) {
+      fill();
+      bool ok = mbar_wait_bounded(bars + 8 * (gc % ST), (gc / ST) & 1, kWaitLimitNs);
       ok = __all_sync(FULL, ok);
       if (!ok) {
-        if (lane == 0) {
-          raise_error(PA_DEVERR_TIMEOUT);
-          *cta_abort = 1;
-        }
-        abort = true;
+        aborted = true;
         break;
       }
       const uint32_t kbase = ring + (gc % ST) * Cfg::kStageBytes;
       const uint32_t vbase = kbase + Cfg::kSliceBytes;
-      const int js = warp + NW * ck;  // slice within the item
-      const int t0 = (ci.j0 + js) * kSliceTokens;
-      if (append_item && js == ci.n - 1) {
+      if (append_item && ck == ci.n - 1) {
         // The item's last slice holds position L-1: append the new rows.
         overwrite_slice_row<D>(kbase, vbase, (ci.L - 1) & (kSliceTokens - 1), knew, vnew, lane);
         if (lane < D / 8) {
@@ -282,57 +238,88 @@ __global__ void __launch_bounds__(NW * 32)
           }
         }
       }
-      attend_slice<D>(st, qf, kbase, vbase, t0, ci.lo, ci.hi, qk_scale, p, lane);
+      attend_slice<D>(st, qf, kbase, vbase, (ci.j0 + ck) * kSliceTokens, ci.lo, ci.hi, qk_scale, p, lane);
       __syncwarp();
       ++gc;
-      publish();
     }
-    publish();
-    try_issue();  // start the next item's loads before merging this one
+    if (aborted) break;
+    fill();  // keep loading the next item while this one is stored
 
-    // ---- merge this item's warp states -------------------------------------------
+    // ---- store this item's result from registers ------------------------------------
     st.reduce_sums();
-    st.dump(ms.m, ms.l, ms.o, warp, G, G, lane);
-    st.reset();
-    named_barrier_sync(1, NW * 32);
-    abort = *cta_abort != 0;  // the same decision in every warp from here on
-    if (!abort) {
-      merge_warps<NW, __nv_bfloat16>(ms, G, D, grid_dest<__nv_bfloat16>(p, ci.b, ci.g, ci.part, ci.whole), tid,
-                                     NW * 32);
+    const size_t row0 = (size_t)ci.b * p.hq + (size_t)ci.g * G;
+    if (ci.whole) {
+      const float inv0 = 1.f / st.l0, inv1 = 1.f / st.l1;
+      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row0 * D;
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) {
+        const int d = mt * 16 + (lane >> 2);
+        if (n0 < G) {
+          out[(size_t)n0 * D + d] = __float2bfloat16_rn(st.o[mt][0] * inv0);
+          out[(size_t)n0 * D + d + 8] = __float2bfloat16_rn(st.o[mt][2] * inv0);
+        }
+        if (n0 + 1 < G) {
+          out[(size_t)(n0 + 1) * D + d] = __float2bfloat16_rn(st.o[mt][1] * inv1);
+          out[(size_t)(n0 + 1) * D + d + 8] = __float2bfloat16_rn(st.o[mt][3] * inv1);
+        }
+      }
+    } else {
+      const size_t slot0 = (row0 + n0) * p.max_parts + ci.part;  // head n0; head n0+1 is max_parts further
+      float* po = p.ws_o + slot0 * D;
+      const size_t hstride = (size_t)p.max_parts * D;
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) {
+        const int d = mt * 16 + (lane >> 2);
+        if (n0 < G) {
+          po[d] = st.o[mt][0];
+          po[d + 8] = st.o[mt][2];
+        }
+        if (n0 + 1 < G) {
+          po[hstride + d] = st.o[mt][1];
+          po[hstride + d + 8] = st.o[mt][3];
+        }
+      }
+      if (lane < 4) {
+        float* pml = p.ws_ml + slot0 * 2;
+        if (n0 < G) {
+          pml[0] = st.m0;
+          pml[1] = st.l0;
+        }
+        if (n0 + 1 < G) {
+          pml[(size_t)p.max_parts * 2 + 0] = st.m1;
+          pml[(size_t)p.max_parts * 2 + 1] = st.l1;
+        }
+      }
     }
-    named_barrier_sync(1, NW * 32);  // merge buffer free; item s+1 published
+    st.reset();
 
     // ---- next item ------------------------------------------------------------------
-    ++s;
-    t_cur = slots[2 * (s & 1) + 1];
-    if (t_cur >= T || abort) break;
-    ci = decode(t_cur);
-    cn = share(ci);
-    if (i_seq == s) {
+    t_cur = t_next;
+    if (t_cur >= T) break;
+    t_next = __shfl_sync(FULL, t_claim, 0);
+    if (lane == 0 && t_next < T) t_claim = 2 * W + atomicAdd(p.queue, 1);
+    if (i_in_next) {
+      ci = ii;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         qf[kk][0] = qf_next[kk][0];
         qf[kk][1] = qf_next[kk][1];
       }
-    } else {  // the issue cursor never entered this item
+      i_in_next = false;
+    } else {  // the load cursor had not reached this item yet
+      ci = decode(t_cur);
       ii = ci;
-      in_ = cn;
       ik = 0;
-      i_seq = s;
       load_rows(ii, 0);
       load_q_frags<D>(qf, q0 + ((size_t)ci.b * p.hq + (size_t)ci.g * G) * D, G, lane);
     }
-    if (tid == 0) t_next = atomicAdd(p.queue, 1);
-    published = false;
   }
 
-  // Every TMA load issued was waited for unless a wait timed out; then give
-  // loads still in flight a bounded time to land before the CTA's shared
-  // memory is released.
-  if (abort && lane == 0) {
-    const uint64_t t0 = global_timer_ns();
-    while (global_timer_ns() - t0 < kDrainLimitNs) {
-    }
+  if (aborted) {
+    if (lane == 0) raise_error(PA_DEVERR_TIMEOUT);
+    // Give this warp's loads still in flight a bounded time to land before the
+    // CTA's shared memory is released.
+    for (int i = gc; i < gi; ++i) (void)mbar_wait_bounded(bars + 8 * (i % ST), (i / ST) & 1, kDrainLimitNs);
   }
 }
 

@@ -300,7 +300,7 @@ cudaError_t launch_dynamic_t(const DecodeParams& p, cudaStream_t st) {
   if (!encode_cache_map(&kmap, p.k_cache, D, rows) || !encode_cache_map(&vmap, p.v_cache, D, rows))
     return cudaErrorInvalidValue;
   auto kern = pa::decode_dynamic_kernel<D, NW, ST, APPEND>;
-  const int smem = Cfg::smem_bytes(p.group, p.batch);
+  const int smem = Cfg::smem_bytes(p.batch);
   static std::atomic<int> smem_done[64];
   cudaError_t e = set_smem_at_least(kern, smem, smem_done);
   if (e != cudaSuccess) return e;
@@ -314,14 +314,14 @@ cudaError_t launch_dynamic_t(const DecodeParams& p, cudaStream_t st) {
 template <bool APPEND>
 cudaError_t launch_dynamic(const DecodeParams& p, cudaStream_t st) {
   switch (p.head_dim) {
-    // Warps x stages per CTA, from a sweep on B200: several small CTAs per SM
-    // beat one deep ring (their merges and item switches overlap).
+    // Warps are independent (one work item each); CTAs of a few warps with a
+    // 2-3 stage ring each put ~192 KB of loads in flight per SM.
     case 64:
-      return launch_dynamic_t<64, 4, 3, APPEND>(p, st);
+      return launch_dynamic_t<64, 4, 4, APPEND>(p, st);
     case 128:
       return launch_dynamic_t<128, 4, 2, APPEND>(p, st);
     default:
-      return launch_dynamic_t<256, 3, 2, APPEND>(p, st);
+      return launch_dynamic_t<256, 2, 2, APPEND>(p, st);
   }
 }
 
@@ -331,6 +331,20 @@ int32_t auto_partition(int32_t batch, int32_t num_kv_heads, int32_t max_context_
                          (max_context_len > 0 ? max_context_len : 1);
   int P = 512;
   while (P > 64 && work / P < kTargetWorkUnits) P >>= 1;
+  return P;
+}
+
+// Partition size of the dynamic schedule, where one warp runs one item: a
+// per-head_dim default (from a sweep on B200: long items cut the partials, the
+// combine's work and the per-item overhead; short ones cut the tail when the
+// last items finish), halved while there would be fewer items than resident
+// warps.
+int32_t dynamic_partition(int32_t batch, int32_t num_kv_heads, int32_t max_context_len, int32_t head_dim) {
+  const long long work = (long long)(batch > 0 ? batch : 1) * (num_kv_heads > 0 ? num_kv_heads : 1) *
+                         (max_context_len > 0 ? max_context_len : 1);
+  const int warps_per_sm = head_dim <= 64 ? 12 : head_dim <= 128 ? 12 : 6;
+  int P = head_dim <= 64 ? 256 : head_dim <= 128 ? 512 : 128;
+  while (P > 64 && work / P < (long long)warps_per_sm * 148) P >>= 1;
   return P;
 }
 
@@ -382,7 +396,8 @@ pa_status_t run_decode(const DecodeCall& c) {
     if (c.max_context_len <= 0) return PA_ERR_INVALID;
     const bool mma = (c.kernel == PA_KERNEL_MMA) || (c.kernel == PA_KERNEL_AUTO && c.dtype == PA_BF16);
     dynamic = c.partition_tokens == 0 && mma && s.batch <= pa::kMaxDynamicBatch;
-    P = auto_partition(s.batch, s.hkv, c.max_context_len, c.partition_tokens);
+    P = dynamic ? dynamic_partition(s.batch, s.hkv, c.max_context_len, s.d)
+                : auto_partition(s.batch, s.hkv, c.max_context_len, c.partition_tokens);
     parts = splitk_parts(c.max_context_len, P);
     if (parts > kMaxPartsPerSeq) return PA_ERR_UNSUPPORTED;
     const size_t need = workspace_size(s.batch, s.hq, s.d, c.max_context_len, P) + (dynamic ? kQueueBytes : 0);
@@ -497,8 +512,12 @@ size_t pa_decode_splitk_workspace_size(int32_t batch, int32_t num_q_heads, int32
   if (batch <= 0 || num_q_heads <= 0 || head_dim <= 0) return 0;
   const int P = auto_partition(batch, num_kv_heads, max_context_len, partition_tokens);
   if (P <= 0) return 0;
-  // partition_tokens == 0 may select the dynamic schedule, which adds its work counter.
-  return workspace_size(batch, num_q_heads, head_dim, max_context_len, P) + (partition_tokens == 0 ? kQueueBytes : 0);
+  size_t n = workspace_size(batch, num_q_heads, head_dim, max_context_len, P);
+  if (partition_tokens == 0) {  // may select the dynamic schedule: its partition and its work counter
+    const int Pd = dynamic_partition(batch, num_kv_heads, max_context_len, head_dim);
+    n = std::max(n, workspace_size(batch, num_q_heads, head_dim, max_context_len, Pd) + kQueueBytes);
+  }
+  return n;
 }
 
 pa_status_t pa_decode_splitk(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
