@@ -191,6 +191,39 @@ pa_status_t pa_decode_step(const void* q, const void* k_new, const void* v_new, 
                            pa_stream_t stream);
 
 /*
+ * pa_decode_splitk_noalloc -- pa_decode_splitk for callers that cannot allocate
+ * device memory.
+ *   The pages describe no such call; it exists for callers that must not call
+ *   cudaMalloc (or any allocating routine) on their path: code running inside
+ *   a CUDA stream capture that forbids allocation, real-time serving loops that
+ *   cannot afford an allocation's synchronisation, and hosts whose memory is
+ *   handed out by a foreign allocator the library cannot reach.  Such a caller
+ *   passes the same inputs and output as to pa_decode_splitk but no workspace:
+ *   the split-K scratch is a fixed array of PA_NOALLOC_SCRATCH_BYTES in the
+ *   library's own device memory (reserved on every GPU that loads the library,
+ *   for the life of the process).
+ *   Returns PA_ERR_WORKSPACE when the call would need more scratch than that
+ *   (pa_decode_splitk_workspace_size() > PA_NOALLOC_SCRATCH_BYTES); such calls
+ *   must use pa_decode_splitk with a workspace of their own.
+ *   The first call on a device looks up the array's device address (no
+ *   allocation); make that first call before any stream capture.  Every call
+ *   uses the same array, and it keeps what the last call left in it: the call
+ *   clears the part that must start at zero itself (the dynamic schedule's work
+ *   counter) with an asynchronous memset on `stream`.  Calls whose executions
+ *   overlap on the GPU (different streams, or different host threads without
+ *   ordering) race on the array and give wrong results; order them.
+ *   It allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ */
+#define PA_NOALLOC_SCRATCH_BYTES (16u << 20) /* 16 MiB */
+pa_status_t pa_decode_splitk_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                     const int32_t* block_tables, const int32_t* context_lens, int32_t batch,
+                                     int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                     int32_t block_size, int32_t max_blocks_per_seq, int32_t num_blocks,
+                                     float scale, float softcap, int32_t window, void* out, pa_dtype_t dtype,
+                                     int32_t partition_tokens, int32_t max_context_len, pa_kernel_t kernel,
+                                     pa_stream_t stream);
+
+/*
  * pa_device_errors -- read (and with clear != 0, reset) the device error word
  * of the current device.  Synchronises with the device.  *bits receives the
  * OR of every PA_DEVERR_* raised since the last clear.

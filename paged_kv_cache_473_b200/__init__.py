@@ -14,6 +14,7 @@ from ._binding import (  # noqa: F401
     PagedAttnError,
     decode,
     decode_splitk,
+    decode_splitk_noalloc,
     decode_step,
     decode_splitk_partition,
     decode_splitk_workspace_size,
@@ -28,6 +29,7 @@ __all__ = [
     "write_kv",
     "decode",
     "decode_splitk",
+    "decode_splitk_noalloc",
     "decode_step",
     "decode_splitk_partition",
     "decode_splitk_workspace_size",

@@ -53,6 +53,8 @@ def _load_library() -> ctypes.CDLL:
                                    _c_i32, _c_i32, _c_i32, _c_f32, _c_f32, _c_i32, _c_vp, _c_i32, _c_i32, _c_i32,
                                    _c_vp, _c_sz, _c_i32, _c_vp]
     lib.pa_decode_step.restype = _c_i32
+    lib.pa_decode_splitk_noalloc.argtypes = dec + [_c_i32, _c_i32, _c_i32, _c_vp]
+    lib.pa_decode_splitk_noalloc.restype = _c_i32
     lib.pa_decode_splitk_partition.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32]
     lib.pa_decode_splitk_partition.restype = _c_i32
     lib.pa_decode_splitk_workspace_size.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32]
@@ -191,6 +193,25 @@ def decode_step(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, k_cac
                             float(softcap), int(window), _ptr(out), _dtype_code(q), ptoks, int(max_context_len), wptr,
                             wbytes, KERNELS[kernel], _stream(stream))
     _check(st, "pa_decode_step")
+    return out
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def decode_splitk_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                          block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float, softcap: float = 0.0,
+                          window: int = 0, *, max_context_len: int, partition_tokens: int = 0,
+                          out: torch.Tensor, kernel: str = "auto", stream=None) -> torch.Tensor:
+    """``decode_splitk`` for callers that must not allocate device memory: the
+    split-K scratch is the library's own fixed array, and ``out`` must be given.
+    Calls must not overlap on the GPU (they share that array)."""
+    B, hq, d, nb, hkv, bs, out = _decode_common(q, k_cache, block_tables, out)
+    st = lib.pa_decode_splitk_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
+                                      B, hq, hkv, d, bs, block_tables.shape[1], nb, float(scale), float(softcap),
+                                      int(window), _ptr(out), _dtype_code(q), int(partition_tokens),
+                                      int(max_context_len), KERNELS[kernel], _stream(stream))
+    _check(st, "pa_decode_splitk_noalloc")
     return out
 
 

@@ -583,6 +583,65 @@ pa_status_t pa_decode_step(const void* q, const void* k_new, const void* v_new, 
   return run_decode(c);
 }
 
+}  // extern "C"
+
+namespace {
+
+// Split-K scratch of pa_decode_splitk_noalloc: reserved in device memory by the
+// module itself, so that call allocates nothing.  Host code must not use the
+// symbol as an address; it asks the runtime for the device address once per
+// device (noalloc_scratch).
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PA_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch on the current device (looked up on the
+// first call per device), or null when the lookup fails.
+void* noalloc_scratch() {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = a;
+  }
+  return addr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status_t pa_decode_splitk_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                     const int32_t* block_tables, const int32_t* context_lens, int32_t batch,
+                                     int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                     int32_t block_size, int32_t max_blocks_per_seq, int32_t num_blocks,
+                                     float scale, float softcap, int32_t window, void* out, pa_dtype_t dtype,
+                                     int32_t partition_tokens, int32_t max_context_len, pa_kernel_t kernel,
+                                     pa_stream_t stream) {
+  t_last_launches = 0;
+  if (batch > 0 && num_q_heads > 0 && head_dim > 0 && max_context_len > 0 && partition_tokens >= 0) {
+    const size_t need = pa_decode_splitk_workspace_size(batch, num_q_heads, head_dim, max_context_len,
+                                                        partition_tokens, num_kv_heads);
+    if (need > PA_NOALLOC_SCRATCH_BYTES) return PA_ERR_WORKSPACE;
+  }
+  void* ws = noalloc_scratch();
+  if (!ws) return PA_ERR_CUDA;
+  // The array keeps the previous call's contents; the dynamic schedule's work
+  // counter (after its partials) must start at zero.
+  if (partition_tokens == 0 && batch > 0 && num_kv_heads > 0 && head_dim > 0 && max_context_len > 0) {
+    const int Pd = dynamic_partition(batch, num_kv_heads, max_context_len, head_dim);
+    const size_t off = workspace_size(batch, num_q_heads, head_dim, max_context_len, Pd);
+    if (off + sizeof(int) <= PA_NOALLOC_SCRATCH_BYTES &&
+        cudaMemsetAsync(static_cast<char*>(ws) + off, 0, sizeof(int), stream) != cudaSuccess)
+      return PA_ERR_CUDA;
+  }
+  return pa_decode_splitk(q, k_cache, v_cache, block_tables, context_lens, batch, num_q_heads, num_kv_heads,
+                          head_dim, block_size, max_blocks_per_seq, num_blocks, scale, softcap, window, out, dtype,
+                          partition_tokens, max_context_len, ws, PA_NOALLOC_SCRATCH_BYTES, kernel, stream);
+}
+
 pa_status_t pa_device_errors(uint32_t* bits, int32_t clear) {
   if (!bits) return PA_ERR_INVALID;
   unsigned int v = 0;
