@@ -155,7 +155,7 @@ class ClockSampler:
                 self.reasons |= int(get_r(self._h))
             except Exception:  # noqa: BLE001
                 break
-            time.sleep(0.002)
+            time.sleep(0.0005)
 
     def __enter__(self):
         if self._nv is not None:
