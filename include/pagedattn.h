@@ -136,16 +136,21 @@ pa_status_t pa_decode(const void* q, const void* k_cache, const void* v_cache, c
  *   it sizes the grid and the workspace.
  *   Schedules: partition_tokens > 0 launches one CTA per (partition, kv head,
  *   sequence).  partition_tokens == 0 lets the library choose the partition
- *   size and, on the tensor-core path (bf16) with batch <= 2048, runs the
- *   dynamic schedule: a persistent grid whose CTAs claim (sequence, kv head,
- *   partition) items from a counter kept in the workspace, so that SMs that
- *   stream faster take more of the work.
+ *   size and, on the tensor-core path (bf16) with batch <= 2048 and
+ *   batch * num_kv_heads <= 65534, runs the
+ *   dynamic schedule: one persistent kernel whose warps claim (sequence, kv
+ *   head, partition) items from a counter kept in the workspace, so that SMs
+ *   that stream faster take more of the work; the last partial of each
+ *   (sequence, kv head) to arrive merges the others in the same kernel, so no
+ *   combine kernel runs.
  *   workspace: device memory of at least pa_decode_splitk_workspace_size()
- *   bytes, 16-byte aligned, zero-filled before its first use.  Each call
- *   leaves it ready for the next one (the dynamic schedule's counter returns
- *   to zero at the end of the call; the rest is scratch between the call's two
- *   kernels).  After a call that failed or raised PA_DEVERR_TIMEOUT, zero it
- *   again.  Calls that share a workspace must be ordered on one stream.
+ *   bytes, 16-byte aligned, zero-filled before its first use.  It starts with
+ *   a fixed 256 KiB counter region (the dynamic schedule's counters, which
+ *   return to zero at the end of every call), followed by the partials
+ *   (scratch within a call).  A workspace sized for the largest call serves
+ *   calls of any smaller shape and either schedule in any order without being
+ *   zeroed again.  After a call that failed or raised PA_DEVERR_TIMEOUT, zero
+ *   it again.  Calls that share a workspace must be ordered on one stream.
  *   Returns PA_ERR_WORKSPACE when the workspace is null, misaligned or small.
  */
 int32_t pa_decode_splitk_partition(int32_t batch, int32_t num_kv_heads, int32_t max_context_len,
@@ -208,8 +213,8 @@ pa_status_t pa_decode_step(const void* q, const void* k_new, const void* v_new, 
  *   The first call on a device looks up the array's device address (no
  *   allocation); make that first call before any stream capture.  Every call
  *   uses the same array, and it keeps what the last call left in it: the call
- *   clears the part that must start at zero itself (the dynamic schedule's work
- *   counter) with an asynchronous memset on `stream`.  Calls whose executions
+ *   clears the part that must start at zero itself (the dynamic schedule's
+ *   counters) with an asynchronous memset on `stream`.  Calls whose executions
  *   overlap on the GPU (different streams, or different host threads without
  *   ordering) race on the array and give wrong results; order them.
  *   It allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.

@@ -27,7 +27,6 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const Decod
   __shared__ float red_o[NWR > 1 ? kCombineWarps : 1][NWR > 1 ? D : 1];
   __shared__ float red_l[kCombineWarps];
   pdl_wait();  // the partials come from the preceding decode kernel
-  if (p.dynamic && blockIdx.x == 0 && threadIdx.x == 0) *p.queue = 0;  // ready for the next call
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int r = warp % NWR;
   const int row = blockIdx.x * ROWS + warp / NWR;
@@ -40,11 +39,6 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const Decod
     const int P = p.partition;
     pb = s0 / P;
     n = L > s0 ? (L + P - 1) / P - pb : 0;
-    if (p.dynamic && n == 0 && r == 0) {  // no work item covered this row
-      OutT* out = static_cast<OutT*>(p.out) + (size_t)row * D + lane * VEC;
-#pragma unroll
-      for (int v = 0; v < VEC; ++v) store_out<OutT>(out + v, 0.f);
-    }
     active = n > 1;
   }
   float acc[VEC];

@@ -33,7 +33,9 @@ struct DecodeParams {
   const void* v_new;
   float* ws_o;                  // split-K partial outputs [B][Hq][max_parts][D]
   float* ws_ml;                 // split-K partial (m, l)  [B][Hq][max_parts][2]
-  int* queue;                   // dynamic schedule: the work-item counter (zero between calls)
+  int* queue;                   // dynamic schedule: [0] work-item counter, [1] CTAs finished (zero between calls)
+  int* unit_count;              // dynamic schedule: partials stored per (sequence, kv head) (zero between calls)
+  int merge_in_kernel;          // dynamic schedule: the last partial of a unit merges it (else the combine kernel)
   int batch, hq, hkv, group, head_dim;
   int block_size, log2_bs, max_blocks, num_blocks;
   int window;
@@ -44,7 +46,6 @@ struct DecodeParams {
   float softcap;    // > 0 and finite: cap enabled
   float inv_softcap;
   int use_softcap;
-  int dynamic;      // the dynamic schedule ran: the combine also resets `queue` and writes L == 0 rows
 };
 
 // Token range one CTA attends.

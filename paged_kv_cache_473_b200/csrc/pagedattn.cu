@@ -28,7 +28,6 @@ thread_local int32_t t_last_launches = 0;
 constexpr int kNoSplitPartition = 1 << 30;
 constexpr int kMaxPartsPerSeq = 8192;
 constexpr int kMaxGridYZ = 65535;
-constexpr size_t kQueueBytes = 256;  // the dynamic schedule's work counter (after the partials)
 // Split-K auto partition: aim for at least this many (partition, kv head,
 // sequence) work units, i.e. several resident CTAs for each of B200's 148 SMs.
 constexpr long long kTargetWorkUnits = 8LL * 148;
@@ -291,8 +290,16 @@ cudaError_t set_smem_at_least(Kernel k, int bytes, std::atomic<int>* done /* [64
   return e;
 }
 
+// Launch the dynamic schedule with the persistent grid (as many CTAs as are
+// resident at once).  Sets p.merge_in_kernel: the partitions of each unit are
+// merged in-kernel when the step is small next to the resident warps (at most
+// 8 partitions per sequence and at most two work items per resident warp, a
+// bound from the host-known sizes), where the combine kernel's fixed cost
+// (launch, grid drain, L2 round trips) would be a large share of the step;
+// otherwise the combine kernel merges them with full-GPU parallelism after
+// the decode grid, and the merging warps do not stall their loads.
 template <int D, int NW, int ST, bool APPEND>
-cudaError_t launch_dynamic_t(const DecodeParams& p, cudaStream_t st) {
+cudaError_t launch_dynamic_t(DecodeParams& p, cudaStream_t st) {
   using Cfg = pa::DynCfg<D, NW, ST>;
   CUtensorMap kmap, vmap;
   const long long rows = (long long)p.num_blocks * p.hkv * p.block_size;
@@ -308,16 +315,19 @@ cudaError_t launch_dynamic_t(const DecodeParams& p, cudaStream_t st) {
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, Cfg::kThreads, smem);
   if (e != cudaSuccess) return e;
   if (occ < 1) return cudaErrorInvalidConfiguration;
-  return launch_ex(kern, dim3(occ * sm_count()), dim3(Cfg::kThreads), smem, st, false, kmap, vmap, p);
+  const int grid = occ * sm_count();
+  const long long unit_bound = (long long)p.batch * p.hkv * p.max_parts;
+  p.merge_in_kernel = (p.max_parts <= 8 && unit_bound <= 2LL * grid * NW) ? 1 : 0;
+  return launch_ex(kern, dim3(grid), dim3(Cfg::kThreads), smem, st, false, kmap, vmap, p);
 }
 
 template <bool APPEND>
-cudaError_t launch_dynamic(const DecodeParams& p, cudaStream_t st) {
+cudaError_t launch_dynamic(DecodeParams& p, cudaStream_t st) {
   switch (p.head_dim) {
     // Warps are independent (one work item each); CTAs of a few warps with a
-    // 2-3 stage ring each put ~192 KB of loads in flight per SM.
+    // 2-6 stage ring each put ~192 KB of loads in flight per SM.
     case 64:
-      return launch_dynamic_t<64, 4, 4, APPEND>(p, st);
+      return launch_dynamic_t<64, 4, 6, APPEND>(p, st);
     case 128:
       return launch_dynamic_t<128, 4, 2, APPEND>(p, st);
     default:
@@ -342,8 +352,10 @@ int32_t auto_partition(int32_t batch, int32_t num_kv_heads, int32_t max_context_
 int32_t dynamic_partition(int32_t batch, int32_t num_kv_heads, int32_t max_context_len, int32_t head_dim) {
   const long long work = (long long)(batch > 0 ? batch : 1) * (num_kv_heads > 0 ? num_kv_heads : 1) *
                          (max_context_len > 0 ? max_context_len : 1);
-  const int warps_per_sm = head_dim <= 64 ? 12 : head_dim <= 128 ? 12 : 6;
-  int P = head_dim <= 64 ? 256 : head_dim <= 128 ? 512 : 128;
+  const int warps_per_sm = head_dim <= 64 ? 8 : head_dim <= 128 ? 12 : 6;
+  // head_dim 128: 512-token partitions past 16K tokens keep the combine's
+  // per-row chain short; 256 below that balances the tail better.
+  int P = head_dim <= 64 ? 256 : head_dim <= 128 ? (max_context_len > 16384 ? 512 : 256) : 128;
   while (P > 64 && work / P < (long long)warps_per_sm * 148) P >>= 1;
   return P;
 }
@@ -352,9 +364,20 @@ long long splitk_parts(int32_t max_context_len, int32_t P) {
   return ((long long)(max_context_len > 0 ? max_context_len : 1) + P - 1) / P;
 }
 
+// Split-K workspace layout, for every schedule: a fixed-size counter region
+// first (the dynamic schedule's work-item counter, its count of finished CTAs
+// and one arrival count per (sequence, kv head)), then the partial outputs
+// [B][Hq][parts][D] and the partial (m, l) [B][Hq][parts][2].  The counters sit
+// at the same place whatever the call's shape, and no call writes partials
+// there, so counters that one call leaves at zero are zero for the next call
+// of any shape or schedule.
 size_t workspace_size(int32_t batch, int32_t num_q_heads, int32_t head_dim, int32_t max_context_len, int32_t P) {
   const size_t rows = (size_t)batch * num_q_heads * (size_t)splitk_parts(max_context_len, P);
-  return align256(rows * head_dim * 4) + align256(rows * 2 * 4);
+  return pa::kCounterBytes + align256(rows * head_dim * 4) + align256(rows * 2 * 4);
+}
+
+size_t dynamic_counter_bytes(int32_t batch, int32_t num_kv_heads) {
+  return (2 + (size_t)batch * num_kv_heads) * sizeof(int);
 }
 
 // Everything the decode entry points share.  split: partitioned launch plus
@@ -395,12 +418,13 @@ pa_status_t run_decode(const DecodeCall& c) {
     if (c.partition_tokens < 0 || (c.partition_tokens > 0 && c.partition_tokens % 64 != 0)) return PA_ERR_INVALID;
     if (c.max_context_len <= 0) return PA_ERR_INVALID;
     const bool mma = (c.kernel == PA_KERNEL_MMA) || (c.kernel == PA_KERNEL_AUTO && c.dtype == PA_BF16);
-    dynamic = c.partition_tokens == 0 && mma && s.batch <= pa::kMaxDynamicBatch;
+    dynamic = c.partition_tokens == 0 && mma && s.batch <= pa::kMaxDynamicBatch &&
+              (long long)s.batch * s.hkv <= pa::kMaxDynamicUnits;
     P = dynamic ? dynamic_partition(s.batch, s.hkv, c.max_context_len, s.d)
                 : auto_partition(s.batch, s.hkv, c.max_context_len, c.partition_tokens);
     parts = splitk_parts(c.max_context_len, P);
     if (parts > kMaxPartsPerSeq) return PA_ERR_UNSUPPORTED;
-    const size_t need = workspace_size(s.batch, s.hq, s.d, c.max_context_len, P) + (dynamic ? kQueueBytes : 0);
+    const size_t need = workspace_size(s.batch, s.hq, s.d, c.max_context_len, P);
     if (s.batch > 0 && (!c.workspace || !aligned(c.workspace, 16) || c.workspace_bytes < need))
       return PA_ERR_WORKSPACE;
   }
@@ -416,21 +440,27 @@ pa_status_t run_decode(const DecodeCall& c) {
     p.max_parts = (int)parts;
     p.max_context = c.max_context_len < p.max_context ? c.max_context_len : p.max_context;
     const size_t rows = (size_t)s.batch * s.hq * parts;
-    p.ws_o = static_cast<float*>(c.workspace);
-    p.ws_ml = reinterpret_cast<float*>(static_cast<char*>(c.workspace) + align256(rows * s.d * 4));
-    if (dynamic) {
-      p.dynamic = 1;
-      p.queue = reinterpret_cast<int*>(static_cast<char*>(c.workspace) +
-                                       workspace_size(s.batch, s.hq, s.d, c.max_context_len, P));
+    char* ws = static_cast<char*>(c.workspace);
+    p.ws_o = reinterpret_cast<float*>(ws + pa::kCounterBytes);
+    p.ws_ml = reinterpret_cast<float*>(ws + pa::kCounterBytes + align256(rows * s.d * 4));
+    if (dynamic) {  // resets its counters itself; merges in-kernel or through the combine
+      p.queue = reinterpret_cast<int*>(ws);
+      p.unit_count = p.queue + 2;
       e = c.append ? launch_dynamic<true>(p, c.stream) : launch_dynamic<false>(p, c.stream);
-    } else {
-      dim3 grid((unsigned)parts, s.hkv, s.batch);
-      e = c.append ? launch_decode<true, true>(p, c.dtype, c.kernel, grid, c.stream)
-                   : launch_decode<true, false>(p, c.dtype, c.kernel, grid, c.stream);
+      if (e != cudaSuccess) return PA_ERR_CUDA;
+      t_last_launches = 1;
+      if (!p.merge_in_kernel && parts > 1) {
+        e = launch_combine<__nv_bfloat16>(p, c.stream);
+        if (e != cudaSuccess) return PA_ERR_CUDA;
+        t_last_launches = 2;
+      }
+      return PA_OK;
     }
+    dim3 grid((unsigned)parts, s.hkv, s.batch);
+    e = c.append ? launch_decode<true, true>(p, c.dtype, c.kernel, grid, c.stream)
+                 : launch_decode<true, false>(p, c.dtype, c.kernel, grid, c.stream);
     if (e != cudaSuccess) return PA_ERR_CUDA;
-    // The dynamic schedule always runs the combine: it resets the work counter.
-    if (parts > 1 || dynamic) {
+    if (parts > 1) {
       e = c.dtype == PA_BF16 ? launch_combine<__nv_bfloat16>(p, c.stream) : launch_combine<float>(p, c.stream);
       if (e != cudaSuccess) return PA_ERR_CUDA;
       t_last_launches = 2;
@@ -513,9 +543,9 @@ size_t pa_decode_splitk_workspace_size(int32_t batch, int32_t num_q_heads, int32
   const int P = auto_partition(batch, num_kv_heads, max_context_len, partition_tokens);
   if (P <= 0) return 0;
   size_t n = workspace_size(batch, num_q_heads, head_dim, max_context_len, P);
-  if (partition_tokens == 0) {  // may select the dynamic schedule: its partition and its work counter
+  if (partition_tokens == 0) {  // may select the dynamic schedule: its partition and its counters
     const int Pd = dynamic_partition(batch, num_kv_heads, max_context_len, head_dim);
-    n = std::max(n, workspace_size(batch, num_q_heads, head_dim, max_context_len, Pd) + kQueueBytes);
+    n = std::max(n, workspace_size(batch, num_q_heads, head_dim, max_context_len, Pd));
   }
   return n;
 }
@@ -628,14 +658,12 @@ pa_status_t pa_decode_splitk_noalloc(const void* q, const void* k_cache, const v
   }
   void* ws = noalloc_scratch();
   if (!ws) return PA_ERR_CUDA;
-  // The array keeps the previous call's contents; the dynamic schedule's work
-  // counter (after its partials) must start at zero.
-  if (partition_tokens == 0 && batch > 0 && num_kv_heads > 0 && head_dim > 0 && max_context_len > 0) {
-    const int Pd = dynamic_partition(batch, num_kv_heads, max_context_len, head_dim);
-    const size_t off = workspace_size(batch, num_q_heads, head_dim, max_context_len, Pd);
-    if (off + sizeof(int) <= PA_NOALLOC_SCRATCH_BYTES &&
-        cudaMemsetAsync(static_cast<char*>(ws) + off, 0, sizeof(int), stream) != cudaSuccess)
-      return PA_ERR_CUDA;
+  // The array keeps the previous call's contents; the dynamic schedule's
+  // counters (after its partials) must start at zero.  A call that completes
+  // leaves them at zero, one that timed out may not: clear them every call.
+  if (partition_tokens == 0 && batch > 0 && num_kv_heads > 0) {
+    const size_t len = std::min(dynamic_counter_bytes(batch, num_kv_heads), pa::kCounterBytes);
+    if (cudaMemsetAsync(ws, 0, len, stream) != cudaSuccess) return PA_ERR_CUDA;
   }
   return pa_decode_splitk(q, k_cache, v_cache, block_tables, context_lens, batch, num_q_heads, num_kv_heads,
                           head_dim, block_size, max_blocks_per_seq, num_blocks, scale, softcap, window, out, dtype,

@@ -116,10 +116,12 @@ def test_workspace_size_formula():
     parts = -(-maxL // P)
     rows = B * hq * parts
     al = lambda x: (x + 255) // 256 * 256  # noqa: E731
-    assert pa.decode_splitk_workspace_size(B, hq, d, maxL, P, 8) == al(rows * d * 4) + al(rows * 2 * 4)
+    counters = (2 + 65534) * 4  # fixed counter region at the start of every split-K workspace
+    assert counters == 256 * 1024
+    assert pa.decode_splitk_workspace_size(B, hq, d, maxL, P, 8) == counters + al(rows * d * 4) + al(rows * 2 * 4)
     assert pa.decode_splitk_workspace_size(0, hq, d, maxL, P, 8) == 0
-    # The library's choice (0) covers the dynamic schedule's partials and its counter.
-    assert pa.decode_splitk_workspace_size(B, hq, d, maxL, 0, 8) >= al(rows * d * 4) + al(rows * 2 * 4) + 256
+    # The library's choice (0) covers the dynamic schedule's partials too.
+    assert pa.decode_splitk_workspace_size(B, hq, d, maxL, 0, 8) >= counters + al(rows * d * 4) + al(rows * 2 * 4)
 
 
 def test_auto_partition_heuristic():

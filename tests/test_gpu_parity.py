@@ -428,6 +428,33 @@ def test_dynamic_schedule_block_permutation_invariance_and_workspace_reuse():
     assert torch.equal(bits(base), bits(moved))
 
 
+def test_dynamic_schedule_counters_return_to_zero():
+    """The merge and work counters live in the workspace and must read zero
+    after every call: calls of different batches share one workspace, and every
+    output row must be written (NaN-filled beforehand) and correct each time."""
+    w = wl.WORKLOADS["tinyllama_1b"]
+    # (batch, seed, partition_tokens): shapes shrink and grow, and a fixed-partition
+    # call (grid schedule plus combine) writes its partials in between.
+    calls = [(24, w.seed, 0), (9, w.seed + 5, 0), (24, w.seed + 6, 128), (24, w.seed, 0)]
+    batches = [wl.make_batch(w, prefilled=True, batch=B, seed=sd) for B, sd, _ in calls]
+    need = max(pa.decode_splitk_workspace_size(bc.q.shape[0], w.num_q_heads, w.head_dim, 2048, P, w.num_kv_heads)
+               for bc, (_, _, P) in zip(batches, calls))
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    outs = []
+    for bc, (_, _, P) in zip(batches, calls):
+        b = to_dev(bc)
+        out = torch.full_like(b.q, float("nan"))
+        pa.decode_splitk(b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, w.scale,
+                         max_context_len=2048, partition_tokens=P, out=out, workspace=ws)
+        torch.cuda.synchronize()
+        ref, _, _ = oracle_step(bc, append=False)
+        assert not torch.isnan(out).any()
+        assert_close(out, ref, torch.bfloat16, f"dynamic reuse batch={bc.q.shape[0]}")
+        outs.append(out)
+    assert torch.equal(bits(outs[0]), bits(outs[3]))
+    assert pa.device_errors() == 0
+
+
 @pytest.mark.parametrize("window", [1, 100, 1000])
 def test_dynamic_schedule_window(window):
     w, b_cpu, b = _reduced("tinyllama_1b", prefilled=True)
