@@ -14,13 +14,19 @@ CPU tensors into it.  The functions below follow these passages:
   ``Q K^T / sqrt(d)``) and "PagedAttention"; flex-nano-vllm README (paged
   attention through a page table, Gemma 2).  Softmax, softcap and window
   readings are stated in the C file's header.
+* ``decode_multi`` -- several query tokens per sequence with a causal mask
+  (the README's "Features": chunked prefill, speculative decoding); each query
+  token is the decode above over the positions up to its own.
 
 Pins (tests/test_oracle_pins.py): agreement with torch's fp64
 ``scaled_dot_product_attention`` on contiguous K/V, permutation invariance over
 physical blocks, L = 1 returning V, identical keys giving mean(V), an infinite
 softcap equal to no softcap, softcap saturation and two-token closed forms,
 window special cases, the page-table example drawn on the nano-vllm README and
-incremental decoding equal to causal attention.
+incremental decoding equal to causal attention; for ``decode_multi``,
+agreement with torch's fp64 attention under an explicit causal (and window)
+mask on contiguous K/V, the T = 1 case equal to ``decode`` bit for bit, and
+causality (changing later positions leaves a row unchanged).
 """
 
 from __future__ import annotations
@@ -65,6 +71,9 @@ def _load():
         lib.oracle_decode.argtypes = [vp, i32, vp, vp, i32, i32p, i32p, i32, i32, i32, i32, i32, i32, i32, dbl, dbl,
                                       i32, i32p, i32, vp]
         lib.oracle_decode.restype = i32
+        lib.oracle_decode_multi.argtypes = [vp, i32, vp, vp, i32, i32p, i32p, i32, i32, i32, i32, i32, i32, i32, i32,
+                                            dbl, dbl, i32, i32p, i32, vp]
+        lib.oracle_decode_multi.restype = i32
         lib.oracle_num_threads.restype = i32
         lib.oracle_set_num_threads.argtypes = [i32]
         _lib = lib
@@ -140,6 +149,35 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_
                                bt.data_ptr(), cl.data_ptr(), B, hq, hkv, d, bs, bt.shape[1], nb, scale64, cap64,
                                int(window), None if rows_arr is None else rows_arr.data_ptr(), n_rows,
                                out.ctypes.data)
+    _check(st)
+    return out
+
+
+def decode_multi(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_tables: torch.Tensor,
+                 context_lens: torch.Tensor, scale: float, softcap: float = 0.0, window: int = 0,
+                 rows: Optional[Sequence[tuple]] = None) -> np.ndarray:
+    """fp64 multi-query attention: ``q`` is ``[B, T, Hq, D]``; query token j
+    of sequence b sits at position ``L - T + j`` and attends causally.
+    Returns ``[B, T, Hq, D]`` (or ``[len(rows), D]`` for ``(b, j, h)`` rows)."""
+    q, k_cache, v_cache = _cpu(q), _cpu(k_cache), _cpu(v_cache)
+    bt = _cpu(block_tables).to(torch.int32)
+    cl = _cpu(context_lens).to(torch.int32)
+    B, T, hq, d = q.shape
+    nb, hkv, bs, d2 = k_cache.shape
+    assert d == d2 and v_cache.shape == k_cache.shape and k_cache.dtype == v_cache.dtype
+    scale64 = float(np.float32(scale))
+    cap64 = float(np.float32(softcap)) if np.isfinite(softcap) else float(softcap)
+    if rows is None:
+        out = np.zeros((B, T, hq, d), dtype=np.float64)
+        rows_arr, n_rows = None, 0
+    else:
+        rows_arr = torch.tensor([list(r) for r in rows], dtype=torch.int32).reshape(-1, 3).contiguous()
+        n_rows = rows_arr.shape[0]
+        out = np.zeros((n_rows, d), dtype=np.float64)
+    st = _load().oracle_decode_multi(q.data_ptr(), _code(q), k_cache.data_ptr(), v_cache.data_ptr(), _code(k_cache),
+                                     bt.data_ptr(), cl.data_ptr(), B, T, hq, hkv, d, bs, bt.shape[1], nb, scale64,
+                                     cap64, int(window), None if rows_arr is None else rows_arr.data_ptr(), n_rows,
+                                     out.ctypes.data)
     _check(st)
     return out
 

@@ -26,6 +26,22 @@
  *              m   = max_t x_t,  w_t = exp(x_t - m),  Z = sum_t w_t
  *              out[b,h,:] = sum_t w_t * V_t[:] / Z
  *            L == 0 gives a zero row.
+ *
+ *   multi    Several new tokens per sequence (speculative-decoding verify, a
+ *            chunk of a chunked prefill): T query tokens per sequence whose
+ *            keys and values are already in the cache at positions
+ *            L-T .. L-1.  Query token j sits at position p_j = L - T + j and
+ *            attends causally: it is the decode above with the context
+ *            [0, p_j + 1), i.e. positions t in [s0_j, p_j + 1) with
+ *            s0_j = (W > 0 && p_j + 1 > W) ? p_j + 1 - W : 0.  A query with
+ *            p_j < 0 (L < T) gets a zero row.
+ *            Sources: nano-vllm (ovshake) README, "Features" ("Chunked
+ *            Prefill", "Speculative Decoding") and the speculative-decoding
+ *            command line (--num-speculative-tokens); causal attention over
+ *            the cache as in "Key Concepts Explained: KV Cache".  The pages do
+ *            not write the mask out; this file takes the causal mask of a
+ *            decoder-only model.
+ *
  *            Sources: nano-vllm (ovshake) README, "X-Ray Mode" (Step 1: 32 query
  *            heads share 8 KV heads; Step 2: scores = Q K^T / sqrt(head_dim))
  *            and "Key Concepts Explained: PagedAttention" (the per-sequence
@@ -111,24 +127,28 @@ int oracle_write_kv(const void* k_new, const void* v_new, const int64_t* slot_ma
   return ORACLE_OK;
 }
 
-/* One output row: sequence b, query head h.  Returns an ORACLE_* code. */
-static int decode_row(const void* q, int q_dtype, const void* k_cache, const void* v_cache, int kv_dtype,
-                      const int32_t* block_tables, const int32_t* context_lens, int hq, int hkv, int d,
-                      int bs, int max_blocks, int num_blocks, double scale, double softcap, int window,
-                      int b, int h, double* out_row, double* x /* scratch, >= max_blocks*bs */) {
+/* One output row: head h of query row `qrow` of q (a sequence-b query)
+ * attending the positions [s0, end) of sequence b, where end = L - back:
+ * back = 0 for decode, T - 1 - j for query token j of T (see the header).
+ * Returns an ORACLE_* code. */
+static int attend_row(const void* q, int q_dtype, int64_t qrow, const void* k_cache, const void* v_cache,
+                      int kv_dtype, const int32_t* block_tables, const int32_t* context_lens, int hq, int hkv,
+                      int d, int bs, int max_blocks, int num_blocks, double scale, double softcap, int window,
+                      int b, int h, int back, double* out_row, double* x /* scratch, >= max_blocks*bs */) {
   const int G = hq / hkv;
   const int g = h / G;
   const int L = context_lens[b];
   for (int j = 0; j < d; ++j) out_row[j] = 0.0;
   if (L < 0 || (int64_t)L > (int64_t)max_blocks * bs) return ORACLE_BAD_LENGTH;
-  const int s0 = (window > 0 && L > window) ? L - window : 0;
-  if (L - s0 <= 0) return ORACLE_OK;
+  const int end = L - back;
+  if (end <= 0) return ORACLE_OK;
+  const int s0 = (window > 0 && end > window) ? end - window : 0;
   const int use_cap = softcap > 0.0 && isfinite(softcap);
-  const int64_t qbase = ((int64_t)b * hq + h) * d;
+  const int64_t qbase = (qrow * hq + h) * d;
 
   /* Pass 1: scores. */
   double m = -INFINITY;
-  for (int t = s0; t < L; ++t) {
+  for (int t = s0; t < end; ++t) {
     int32_t phys = block_tables[(int64_t)b * max_blocks + t / bs];
     if (phys < 0 || phys >= num_blocks) return ORACLE_BAD_BLOCK;
     int64_t kbase = (((int64_t)phys * hkv + g) * bs + t % bs) * d;
@@ -141,7 +161,7 @@ static int decode_row(const void* q, int q_dtype, const void* k_cache, const voi
   }
   /* Pass 2: weights and the weighted sum of values. */
   double Z = 0.0;
-  for (int t = s0; t < L; ++t) {
+  for (int t = s0; t < end; ++t) {
     double w = exp(x[t - s0] - m);
     Z += w;
     int32_t phys = block_tables[(int64_t)b * max_blocks + t / bs];
@@ -178,8 +198,52 @@ int oracle_decode(const void* q, int q_dtype, const void* k_cache, const void* v
         int h = rows ? rows[2 * r + 1] : r % hq;
         int st = ORACLE_BAD_ARGS;
         if (b >= 0 && b < batch && h >= 0 && h < hq)
-          st = decode_row(q, q_dtype, k_cache, v_cache, kv_dtype, block_tables, context_lens, hq, hkv, d, bs,
-                          max_blocks, num_blocks, scale, softcap, window, b, h, out + (int64_t)r * d, x);
+          st = attend_row(q, q_dtype, b, k_cache, v_cache, kv_dtype, block_tables, context_lens, hq, hkv, d, bs,
+                          max_blocks, num_blocks, scale, softcap, window, b, h, 0, out + (int64_t)r * d, x);
+        if (st != ORACLE_OK) {
+#pragma omp critical
+          status = st;
+        }
+      }
+      free(x);
+    }
+  }
+  return status;
+}
+
+
+/*
+ * Multi-query rows: q is [batch, q_len, hq, d]; query token j of sequence b
+ * attends [s0_j, L - q_len + j + 1) (see the header).
+ * rows == NULL: every (b, j, h), out is [batch, q_len, hq, d].
+ * rows != NULL: n_rows triples (b, j, h) stored as rows[3*r .. 3*r+2]; out is [n_rows, d].
+ */
+int oracle_decode_multi(const void* q, int q_dtype, const void* k_cache, const void* v_cache, int kv_dtype,
+                        const int32_t* block_tables, const int32_t* context_lens, int batch, int q_len, int hq,
+                        int hkv, int d, int bs, int max_blocks, int num_blocks, double scale, double softcap,
+                        int window, const int32_t* rows, int n_rows, double* out) {
+  if (batch < 0 || q_len <= 0 || hq <= 0 || hkv <= 0 || hq % hkv != 0 || d <= 0 || bs <= 0 || max_blocks <= 0)
+    return ORACLE_BAD_ARGS;
+  const int n = rows ? n_rows : batch * q_len * hq;
+  const int64_t cap = (int64_t)max_blocks * bs;
+  int status = ORACLE_OK;
+#pragma omp parallel
+  {
+    double* x = (double*)malloc(sizeof(double) * (size_t)(cap > 0 ? cap : 1));
+    if (!x) {
+#pragma omp critical
+      status = ORACLE_NO_MEMORY;
+    } else {
+#pragma omp for schedule(dynamic, 1)
+      for (int r = 0; r < n; ++r) {
+        int b = rows ? rows[3 * r] : r / (q_len * hq);
+        int j = rows ? rows[3 * r + 1] : (r / hq) % q_len;
+        int h = rows ? rows[3 * r + 2] : r % hq;
+        int st = ORACLE_BAD_ARGS;
+        if (b >= 0 && b < batch && j >= 0 && j < q_len && h >= 0 && h < hq)
+          st = attend_row(q, q_dtype, (int64_t)b * q_len + j, k_cache, v_cache, kv_dtype, block_tables,
+                          context_lens, hq, hkv, d, bs, max_blocks, num_blocks, scale, softcap, window, b, h,
+                          q_len - 1 - j, out + (int64_t)r * d, x);
         if (st != ORACLE_OK) {
 #pragma omp critical
           status = st;

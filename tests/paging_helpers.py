@@ -55,3 +55,25 @@ def sdpa_decode(q, seqs_k, seqs_v, scale, window=0):
         o = F.scaled_dot_product_attention(qq, k, v, scale=scale, enable_gqa=True)
         out[b] = o[0, :, 0, :]
     return out
+
+
+def sdpa_multi(q, seqs_k, seqs_v, scale, window=0):
+    """torch fp64 attention of each sequence's last T queries (``q``: [B, T, Hq, D])
+    against its contiguous K/V, with an explicit boolean mask: query j at
+    position p = L - T + j sees positions t with t <= p and p - t < window
+    (window > 0)."""
+    B, T, Hq, D = q.shape
+    out = torch.zeros((B, T, Hq, D), dtype=torch.float64)
+    for b in range(B):
+        L = seqs_k[b].shape[0]
+        pos = torch.arange(L - T, L).unsqueeze(1)  # [T, 1]
+        t = torch.arange(L).unsqueeze(0)  # [1, L]
+        mask = t <= pos
+        if window > 0:
+            mask &= (pos - t) < window
+        k = seqs_k[b].to(torch.float64).permute(1, 0, 2).unsqueeze(0)  # [1, Hkv, L, D]
+        v = seqs_v[b].to(torch.float64).permute(1, 0, 2).unsqueeze(0)
+        qq = q[b].to(torch.float64).permute(1, 0, 2).unsqueeze(0)  # [1, Hq, T, D]
+        o = F.scaled_dot_product_attention(qq, k, v, attn_mask=mask, scale=scale, enable_gqa=True)
+        out[b] = o[0].permute(1, 0, 2)
+    return out

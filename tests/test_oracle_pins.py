@@ -15,7 +15,7 @@ import torch
 import torch.nn.functional as F
 
 import oracle
-from tests.paging_helpers import scatter_to_pool, sdpa_decode
+from tests.paging_helpers import scatter_to_pool, sdpa_decode, sdpa_multi
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -292,3 +292,89 @@ def test_sampled_rows_match_full_output():
     got = oracle.decode(q, kc, vc, tables, cl, 0.25, softcap=4.0, window=10, rows=rows)
     for i, (b, h) in enumerate(rows):
         assert np.array_equal(got[i], full[b, h])
+
+
+# ---- multi-query rows (several new tokens per sequence, causal) ---------------------
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("T", [1, 2, 5, 8])
+@pytest.mark.parametrize("window", [0, 3, 17])
+@pytest.mark.parametrize("hq,hkv,d,bs", [(8, 2, 64, 16), (6, 3, 16, 4)])
+def test_multi_agrees_with_torch_under_a_causal_mask(dtype, T, window, hq, hkv, d, bs):
+    gen = torch.Generator().manual_seed(100 + T + window + d)
+    lens = [T, 9 + T, 40, 23]
+    ks, vs = _rand_seqs(gen, lens, hkv, d, dtype)
+    q = torch.randn((len(lens), T, hq, d), generator=gen).to(dtype)
+    kc, vc, tables, cl = scatter_to_pool(ks, vs, bs, gen, dtype=dtype)
+    scale = 1.0 / math.sqrt(d)
+    got = oracle.decode_multi(q, kc, vc, tables, cl, scale, window=window)
+    ref = sdpa_multi(q, ks, vs, float(np.float32(scale)), window=window).numpy()
+    assert np.max(np.abs(got - ref)) <= 1e-12
+
+
+def test_multi_with_one_query_token_equals_decode_bit_exact():
+    gen = torch.Generator().manual_seed(61)
+    lens = [1, 17, 64, 33]
+    ks, vs = _rand_seqs(gen, lens, 2, 32, torch.bfloat16)
+    q = torch.randn((4, 8, 32), generator=gen).to(torch.bfloat16)
+    kc, vc, tables, cl = scatter_to_pool(ks, vs, 8, gen, dtype=torch.bfloat16)
+    for cap, win in [(0.0, 0), (50.0, 0), (0.0, 5)]:
+        a = oracle.decode(q, kc, vc, tables, cl, 0.2, cap, win)
+        b = oracle.decode_multi(q.unsqueeze(1), kc, vc, tables, cl, 0.2, cap, win)[:, 0]
+        assert np.array_equal(a, b)
+
+
+def test_multi_row_j_is_decode_over_its_own_prefix_with_softcap():
+    """Query token j of T is a decode step whose context ends at its own
+    position (the incremental reading of the KV cache) -- checked with the
+    softcap on, against the pinned decode."""
+    gen = torch.Generator().manual_seed(62)
+    T, lens = 5, [5, 12, 30]
+    ks, vs = _rand_seqs(gen, lens, 4, 16)
+    q = torch.randn((3, T, 8, 16), generator=gen)
+    kc, vc, tables, cl = scatter_to_pool(ks, vs, 4, gen)
+    got = oracle.decode_multi(q, kc, vc, tables, cl, 0.5, softcap=3.0, window=7)
+    for j in range(T):
+        cl_j = (cl - (T - 1 - j)).to(torch.int32)
+        ref = oracle.decode(q[:, j], kc, vc, tables, cl_j, 0.5, softcap=3.0, window=7)
+        assert np.max(np.abs(got[:, j] - ref)) <= 1e-12
+
+
+def test_multi_rows_do_not_see_later_positions():
+    gen = torch.Generator().manual_seed(63)
+    T, lens = 4, [11, 20]
+    ks, vs = _rand_seqs(gen, lens, 2, 16)
+    q = torch.randn((2, T, 4, 16), generator=gen)
+    kc, vc, tables, cl = scatter_to_pool(ks, vs, 4, gen)
+    base = oracle.decode_multi(q, kc, vc, tables, cl, 0.25)
+    for j in range(T):
+        ks2 = [k.clone() for k in ks]
+        vs2 = [v.clone() for v in vs]
+        for b, L in enumerate(lens):  # overwrite every position after query j's
+            ks2[b][L - T + j + 1:] = 7.0
+            vs2[b][L - T + j + 1:] = -3.0
+        kc2, vc2 = kc.clone(), vc.clone()
+        for b, L in enumerate(lens):
+            for t in range(L - T + j + 1, L):
+                blk = int(tables[b, t // 4])
+                kc2[blk, :, t % 4] = ks2[b][t]
+                vc2[blk, :, t % 4] = vs2[b][t]
+        got = oracle.decode_multi(q, kc2, vc2, tables, cl, 0.25)
+        assert np.array_equal(got[:, : j + 1], base[:, : j + 1])
+        if j + 1 < T:
+            assert not np.array_equal(got[:, j + 1:], base[:, j + 1:])
+
+
+def test_multi_queries_before_the_start_give_zero_rows_and_rows_match():
+    gen = torch.Generator().manual_seed(64)
+    T, lens = 6, [3, 10]  # sequence 0 holds fewer positions than query tokens
+    ks, vs = _rand_seqs(gen, lens, 2, 16)
+    q = torch.randn((2, T, 4, 16), generator=gen)
+    kc, vc, tables, cl = scatter_to_pool(ks, vs, 4, gen)
+    full = oracle.decode_multi(q, kc, vc, tables, cl, 0.25)
+    assert np.all(full[0, : T - 3] == 0.0) and np.all(np.isfinite(full))
+    rows = [(0, 5, 1), (1, 0, 3), (1, 5, 0), (0, 0, 2)]
+    part = oracle.decode_multi(q, kc, vc, tables, cl, 0.25, rows=rows)
+    for r, (b, j, h) in enumerate(rows):
+        assert np.array_equal(part[r], full[b, j, h])
