@@ -196,6 +196,39 @@ pa_status_t pa_decode_step(const void* q, const void* k_new, const void* v_new, 
                            pa_stream_t stream);
 
 /*
+ * pa_decode_multi -- attention for several new query tokens per sequence
+ * (speculative-decoding verify, one chunk of a chunked prefill).
+ *   q: [batch][q_len][num_q_heads][head_dim] bf16; out: the same shape.  The
+ *   q_len new tokens' keys and values must already be in the cache (append
+ *   them with pa_write_kv first) at positions L-q_len .. L-1, L =
+ *   context_lens[b].  Query token j sits at position p_j = L - q_len + j and
+ *   attends causally: positions t with s0_j <= t <= p_j, where s0_j = p_j + 1
+ *   - window when window > 0 and p_j + 1 > window, else 0; scores, softcap
+ *   and softmax as pa_decode.  A token with p_j < 0 (L < q_len) gets a zero
+ *   row; L = 0 gives zero rows.
+ *   bf16 only (PA_ERR_UNSUPPORTED for fp32); q_len * (num_q_heads /
+ *   num_kv_heads) <= 64 (PA_ERR_UNSUPPORTED above).
+ *   partition_tokens < 0: one CTA per (sequence, kv head), no workspace
+ *   (workspace may be NULL; max_context_len is ignored).  partition_tokens >= 0:
+ *   split-K as pa_decode_splitk's grid schedule (0 = library's choice), with a
+ *   workspace of pa_decode_multi_workspace_size() bytes under the same
+ *   contract as pa_decode_splitk's, and a combine kernel for sequences whose
+ *   range spans several partitions.
+ *   Passages: nano-vllm (ovshake) README, "Features" (chunked prefill,
+ *   speculative decoding) and the speculative-decoding command line
+ *   (--num-speculative-tokens); causal attention over the cache as in "Key
+ *   Concepts Explained: KV Cache".
+ */
+pa_status_t pa_decode_multi(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                            const int32_t* context_lens, int32_t batch, int32_t q_len, int32_t num_q_heads,
+                            int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq,
+                            int32_t num_blocks, float scale, float softcap, int32_t window, void* out,
+                            pa_dtype_t dtype, int32_t partition_tokens, int32_t max_context_len, void* workspace,
+                            size_t workspace_bytes, pa_stream_t stream);
+size_t pa_decode_multi_workspace_size(int32_t batch, int32_t q_len, int32_t num_q_heads, int32_t head_dim,
+                                      int32_t max_context_len, int32_t partition_tokens, int32_t num_kv_heads);
+
+/*
  * pa_decode_splitk_noalloc -- pa_decode_splitk for callers that cannot allocate
  * device memory.
  *   The pages describe no such call; it exists for callers that must not call

@@ -13,6 +13,8 @@ from ._binding import (  # noqa: F401
     KERNELS,
     PagedAttnError,
     decode,
+    decode_multi,
+    decode_multi_workspace_size,
     decode_splitk,
     decode_splitk_noalloc,
     decode_step,
@@ -28,6 +30,8 @@ from ._binding import (  # noqa: F401
 __all__ = [
     "write_kv",
     "decode",
+    "decode_multi",
+    "decode_multi_workspace_size",
     "decode_splitk",
     "decode_splitk_noalloc",
     "decode_step",

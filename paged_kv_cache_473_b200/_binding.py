@@ -59,6 +59,12 @@ def _load_library() -> ctypes.CDLL:
     lib.pa_decode_splitk_partition.restype = _c_i32
     lib.pa_decode_splitk_workspace_size.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32]
     lib.pa_decode_splitk_workspace_size.restype = _c_sz
+    lib.pa_decode_multi.argtypes = [_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32,
+                                    _c_i32, _c_i32, _c_f32, _c_f32, _c_i32, _c_vp, _c_i32, _c_i32, _c_i32, _c_vp, _c_sz,
+                                    _c_vp]
+    lib.pa_decode_multi.restype = _c_i32
+    lib.pa_decode_multi_workspace_size.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32]
+    lib.pa_decode_multi_workspace_size.restype = _c_sz
     lib.pa_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint32), _c_i32]
     lib.pa_device_errors.restype = _c_i32
     lib.pa_error_string.argtypes = [_c_i32]
@@ -193,6 +199,44 @@ def decode_step(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, k_cac
                             float(softcap), int(window), _ptr(out), _dtype_code(q), ptoks, int(max_context_len), wptr,
                             wbytes, KERNELS[kernel], _stream(stream))
     _check(st, "pa_decode_step")
+    return out
+
+
+def decode_multi_workspace_size(batch: int, q_len: int, num_q_heads: int, head_dim: int, max_context_len: int,
+                                partition_tokens: int = 0, num_kv_heads: int = 1) -> int:
+    return lib.pa_decode_multi_workspace_size(batch, q_len, num_q_heads, head_dim, max_context_len, partition_tokens,
+                                              num_kv_heads)
+
+
+def decode_multi(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_tables: torch.Tensor,
+                 context_lens: torch.Tensor, scale: float, softcap: float = 0.0, window: int = 0, *,
+                 split: bool = True, max_context_len: int = 0, partition_tokens: int = 0,
+                 out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+    """Attention of ``q`` ``[B, T, Hq, D]`` (T new tokens per sequence, already
+    appended to the cache at positions ``L-T .. L-1``) with a causal mask.
+
+    ``split=False``: one CTA per (sequence, kv head).  ``split=True``: split-K
+    with the combine (``max_context_len`` required; the workspace is allocated
+    zeroed with torch if not given).
+    """
+    B, T, hq, d = q.shape
+    nb, hkv, bs, _ = k_cache.shape
+    if out is None:
+        out = torch.empty_like(q)
+    ptoks = int(partition_tokens) if split else -1
+    wptr, wbytes = None, 0
+    if split:
+        if max_context_len <= 0:
+            raise ValueError("decode_multi(split=True) needs max_context_len")
+        need = decode_multi_workspace_size(B, T, hq, d, max_context_len, partition_tokens, hkv)
+        if workspace is None:
+            workspace = torch.zeros(max(need, 16), dtype=torch.uint8, device=q.device)
+        wptr, wbytes = _ptr(workspace), workspace.numel() * workspace.element_size()
+    st = lib.pa_decode_multi(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens), B, T, hq,
+                             hkv, d, bs, block_tables.shape[1], nb, float(scale), float(softcap), int(window),
+                             _ptr(out), _dtype_code(q), ptoks, int(max_context_len), wptr, wbytes, _stream(stream))
+    _check(st, "pa_decode_multi")
     return out
 
 

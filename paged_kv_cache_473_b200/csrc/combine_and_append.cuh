@@ -8,10 +8,13 @@ namespace pa {
 
 // ---- split-K combine ----------------------------------------------------------
 //
-// NWR warps per output row (sequence b, query head h).  The partitions of the
-// sequence's attended range each left (m_p, l_p, o_p) in the workspace (log2
-// domain, o_p unnormalised relative to m_p).  With M = max_p m_p:
+// NWR warps per output row (sequence b, query token j, query head h; j = 0
+// for decode).  The partitions of the sequence's attended range each left
+// (m_p, l_p, o_p) in the workspace (log2 domain, o_p unnormalised relative to
+// m_p).  With M = max_p m_p:
 //   out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p.
+// A partition that held none of a multi-query row's positions left m = -inf,
+// l = 0, o = 0 and weighs nothing; a row with no position at all is zero.
 // Warp r of a row takes partitions r, r + NWR, ...; lane k computes the
 // weights of every 32nd of those and broadcasts them, and each lane
 // accumulates D/32 consecutive dims.  With NWR > 1 the row's warps add their
@@ -30,12 +33,12 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const Decod
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int r = warp % NWR;
   const int row = blockIdx.x * ROWS + warp / NWR;
-  bool active = row < p.batch * p.hq;
+  bool active = row < p.batch * p.q_len * p.hq;
   int pb = 0, n = 0;
   if (active) {
-    const int b = row / p.hq;
+    const int b = row / (p.q_len * p.hq);
     const int L = clamp_context(p, b, false);
-    const int s0 = window_start(L, p.window);
+    const int s0 = window_start(max(L - p.q_len + 1, 0), p.window);  // the first query token's window
     const int P = p.partition;
     pb = s0 / P;
     n = L > s0 ? (L + P - 1) / P - pb : 0;
@@ -57,7 +60,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const Decod
     for (int c = 0; c < nj; c += 32) {
       const int j = c + lane;
       float w = 0.f;
-      if (j < nj) {
+      if (j < nj && M != -CUDART_INF_F) {
         const int i = r + NWR * j;
         w = exp2f(ml[2 * i] - M);
         den = fmaf(w, ml[2 * i + 1], den);
@@ -92,7 +95,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const Decod
   } else if (!active) {
     return;
   }
-  const float inv = 1.f / den;
+  const float inv = den > 0.f ? 1.f / den : 0.f;
   OutT* out = static_cast<OutT*>(p.out) + (size_t)row * D + lane * VEC;
 #pragma unroll
   for (int v = 0; v < VEC; ++v) store_out<OutT>(out + v, acc[v] * inv);

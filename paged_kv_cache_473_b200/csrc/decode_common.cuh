@@ -37,6 +37,7 @@ struct DecodeParams {
   int* unit_count;              // dynamic schedule: partials stored per (sequence, kv head) (zero between calls)
   int merge_in_kernel;          // dynamic schedule: the last partial of a unit merges it (else the combine kernel)
   int batch, hq, hkv, group, head_dim;
+  int q_len;        // query tokens per sequence (1 for decode; T for the multi-query rows [B][T][Hq][D])
   int block_size, log2_bs, max_blocks, num_blocks;
   int window;
   int partition;    // tokens per partition (a multiple of 64); 1 << 30 without split

@@ -1,0 +1,216 @@
+// Multi-query paged attention, bf16, tensor cores: T query tokens per sequence
+// (speculative-decoding verify, a chunk of a chunked prefill) whose keys and
+// values are already in the cache at positions L-T .. L-1.  Query token j sits
+// at position p_j = L - T + j and attends the positions [s0_j, p_j + 1) of its
+// sequence (causal; s0_j is the sliding-window start).
+//
+// One CTA per (partition, kv head, sequence).  The T*G query rows of the kv
+// head are the N columns of the attention tile, token-major (column
+// c = j*G + h); warp w owns columns [8w, 8w + 8) and runs the decode slice
+// attention (attend_slice) on them with per-column causal / window bounds.
+// Every warp needs every key and value of the range, so the K/V slices are
+// loaded once per CTA into a shared ring of ST stages: warp 0 issues the 2-D
+// TMA tile loads (full barrier per stage, with the byte count), every warp
+// consumes a stage and arrives on the stage's empty barrier, and warp 0 waits
+// for that before it refills the stage.  Each warp writes its own columns:
+// the normalised rows when the sequence's range is one partition, else the
+// partial state for the combine kernel.
+#pragma once
+
+#include "decode_common.cuh"
+#include "mma_slice.cuh"
+#include "ptx.cuh"
+
+namespace pa {
+
+constexpr int kMaxMultiColumns = 64;  // T * G query rows per kv head: 8 warps of 8 columns
+
+template <int D, int ST>
+struct MultiCfg {
+  static constexpr int kSliceBytes = SliceBytes<D>::kSlice;
+  static constexpr int kStageBytes = SliceBytes<D>::kStage;
+  static constexpr int kRingBytes = ST * kStageBytes;
+  static constexpr int kFullOffset = kRingBytes;           // ST full barriers
+  static constexpr int kEmptyOffset = kRingBytes + ST * 8;  // ST empty barriers
+  static constexpr int kSmemBytes = kRingBytes + 2 * ST * 8 + 1024;
+};
+
+// Token range of query column c (token j = c / G) inside the CTA's partition
+// [pl, ph): [max(s0_j, pl), min(p_j + 1, ph)).  Padding columns (c >= T*G)
+// take the CTA's union range so that their (discarded) softmax stays finite.
+__device__ __forceinline__ void column_range(int c, int G, int T, int L, int window, int pl, int ph, int ulo,
+                                             int uhi, int& lo, int& hi) {
+  if (c >= T * G) {
+    lo = ulo;
+    hi = uhi;
+    return;
+  }
+  const int end = L - T + c / G + 1;  // p_j + 1
+  lo = max(window_start(end, window), pl);
+  hi = min(end, ph);
+}
+
+template <int D, int ST, bool SPLIT>
+__global__ void __launch_bounds__(kMaxMultiColumns / 8 * 32)
+    decode_multi_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                        const DecodeParams p) {
+  using Cfg = MultiCfg<D, ST>;
+  constexpr uint32_t FULL = 0xffffffffu;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+  if (SPLIT) pdl_launch_dependents();  // the combine may launch; it waits for this grid to finish
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int NW = blockDim.x >> 5;
+  const int part = SPLIT ? (int)blockIdx.x : 0;
+  const int g = blockIdx.y, b = blockIdx.z;
+  const int G = p.group, T = p.q_len, P = p.partition;
+
+  const int L = clamp_context(p, b, threadIdx.x == 0 && part == 0);
+  // The union of the query tokens' ranges is [s0 of token 0, L).
+  const int ulo_seq = window_start(max(L - T + 1, 0), p.window);
+  const int n_parts = (L > ulo_seq) ? (L + P - 1) / P - ulo_seq / P : 0;
+  const bool final_write = !SPLIT || n_parts == 1;
+  const int pl = part * P, ph = pl + P;
+  const int ulo = max(ulo_seq, pl), uhi = min(L, ph);
+
+  // This lane's two accumulator columns and their ranges.
+  const int n0 = 2 * (lane & 3);
+  const int c0 = warp * 8 + n0;
+  ColRange cr;
+  column_range(c0, G, T, L, p.window, pl, ph, ulo, uhi, cr.lo0, cr.hi0);
+  column_range(c0 + 1, G, T, L, p.window, pl, ph, ulo, uhi, cr.lo1, cr.hi1);
+
+  // Output row (or workspace row) of column c: ((b*T + j)*Hq + g*G + h).
+  auto row_of = [&](int c) { return ((size_t)b * T + c / G) * p.hq + (size_t)g * G + c % G; };
+
+  if (ulo >= uhi) {  // nothing of this sequence falls in this partition
+    if (n_parts == 0 && part == 0) {  // L == 0: zero rows for every query column
+      for (int idx = threadIdx.x; idx < T * G * D; idx += blockDim.x)
+        static_cast<__nv_bfloat16*>(p.out)[row_of(idx / D) * D + idx % D] = __float2bfloat16_rn(0.f);
+    }
+    return;
+  }
+
+  const uint32_t ring = smem_addr(smem);
+  const uint32_t full = smem_addr(smem + Cfg::kFullOffset);
+  const uint32_t empty = smem_addr(smem + Cfg::kEmptyOffset);
+  if (threadIdx.x == 0) {
+    prefetch_tensormap(&kmap);
+    prefetch_tensormap(&vmap);
+#pragma unroll
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(full + 8 * s, 1);
+      mbar_init(empty + 8 * s, NW);
+    }
+    mbar_init_fence();
+  }
+  __syncthreads();
+
+  const int j0 = ulo / kSliceTokens;
+  const int n = (uhi + kSliceTokens - 1) / kSliceTokens - j0;
+  const int32_t* table = p.block_tables + (size_t)b * p.max_blocks;
+
+  // Warp 0 issues slice i into stage i % ST.
+  auto issue = [&](int i) {
+    const int t = (j0 + i) * kSliceTokens;
+    const int phys = table[t >> p.log2_bs];
+    const int y = (phys >= 0 && phys < p.num_blocks) ? cache_row(p, phys, g, t) : -1;
+    issue_slice<D>(ring + (i % ST) * Cfg::kStageBytes, full + 8 * (i % ST), &kmap, &vmap, y, lane);
+  };
+  int issued = 0;
+  if (warp == 0)
+    for (; issued < ST && issued < n; ++issued) issue(issued);
+
+  // Q^T as the B operand: column n = lane / 4 of the warp's 8 is query column
+  // 8*warp + n; padding columns are zero.
+  uint32_t qf[D / 16][2];
+  {
+    const int c = warp * 8 + (lane >> 2);
+    const bool real = c < T * G;
+    const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q) + row_of(real ? c : 0) * D;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const int d = kk * 16 + 2 * (lane & 3);
+      qf[kk][0] = real ? *reinterpret_cast<const uint32_t*>(qrow + d) : 0u;
+      qf[kk][1] = real ? *reinterpret_cast<const uint32_t*>(qrow + d + 8) : 0u;
+    }
+  }
+
+  WarpAttn<D> st;
+  st.reset();
+  const float qk_scale = p.use_softcap ? p.scale : p.scale * kLog2e;
+  bool failed = false;
+  int i = 0;
+  for (; i < n; ++i) {
+    const int s = i % ST;
+    const uint32_t par = (i / ST) & 1;
+    bool ok = mbar_wait_bounded(full + 8 * s, par, kWaitLimitNs);
+    ok = __all_sync(FULL, ok);
+    if (!ok) {
+      failed = true;
+      break;
+    }
+    const uint32_t kbase = ring + s * Cfg::kStageBytes;
+    attend_slice<D, true>(st, qf, kbase, kbase + Cfg::kSliceBytes, (j0 + i) * kSliceTokens, ulo, uhi, qk_scale, p,
+                          lane, cr);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty + 8 * s);
+    if (warp == 0 && issued < n) {  // refill this stage once every warp has released it
+      ok = mbar_wait_bounded(empty + 8 * s, par, kWaitLimitNs);
+      ok = __all_sync(FULL, ok);
+      if (!ok) {
+        failed = true;
+        ++i;
+        break;
+      }
+      issue(issued++);
+    }
+  }
+
+  if (failed) {
+    if (lane == 0) raise_error(PA_DEVERR_TIMEOUT);
+    // Warp 0 owns the loads: let those still in flight land before the CTA exits.
+    if (warp == 0)
+      for (int k = i; k < issued; ++k) (void)mbar_wait_bounded(full + 8 * (k % ST), (k / ST) & 1, kDrainLimitNs);
+    return;
+  }
+  st.reduce_sums();
+
+  // ---- this warp's columns: final rows or partials, from registers -----------------
+  const int cols = T * G;
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const int c = c0 + e;
+    if (c >= cols) continue;
+    const float m = e ? st.m1 : st.m0;
+    const float l = e ? st.l1 : st.l0;
+    const size_t row = row_of(c);
+    if (final_write) {
+      const float inv = l > 0.f ? 1.f / l : 0.f;  // a column with no position gives a zero row
+      __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + row * D;
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) {
+        const int d = mt * 16 + (lane >> 2);
+        o[d] = __float2bfloat16_rn(st.o[mt][e] * inv);
+        o[d + 8] = __float2bfloat16_rn(st.o[mt][2 + e] * inv);
+      }
+    } else {
+      float* po = p.ws_o + (row * p.max_parts + part) * D;
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) {
+        const int d = mt * 16 + (lane >> 2);
+        po[d] = st.o[mt][e];
+        po[d + 8] = st.o[mt][2 + e];
+      }
+      if (lane < 4) {
+        float* pml = p.ws_ml + (row * p.max_parts + part) * 2;
+        pml[0] = m;
+        pml[1] = l;
+      }
+    }
+  }
+}
+
+}  // namespace pa

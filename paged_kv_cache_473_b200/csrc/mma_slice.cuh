@@ -139,12 +139,21 @@ __device__ __forceinline__ void overwrite_slice_row(uint32_t kbase, uint32_t vba
   __syncwarp();
 }
 
+// Per-column token ranges of the lane's two columns n0, n0 + 1 (multi-query
+// rows: each query token has its own causal end and window start).
+struct ColRange {
+  int lo0, hi0, lo1, hi1;
+};
+
 // Attend the slice of tokens [t0, t0+16) whose K/V rows sit at kbase/vbase;
-// only tokens in [lo, hi) count.
-template <int D>
+// only tokens in [lo, hi) count.  COLS: column n0 (n0 + 1) of this lane only
+// counts tokens in [cr.lo0, cr.hi0) ([cr.lo1, cr.hi1)), inside [lo, hi); a
+// column may then see no token of the slice at all, which the safe maximum
+// below turns into a zero weight.
+template <int D, bool COLS = false>
 __device__ __forceinline__ void attend_slice(WarpAttn<D>& st, const uint32_t (&qf)[D / 16][2], uint32_t kbase,
                                              uint32_t vbase, int t0, int lo, int hi, float qk_scale,
-                                             const DecodeParams& p, int lane) {
+                                             const DecodeParams& p, int lane, const ColRange& cr = ColRange{}) {
   constexpr uint32_t FULL = 0xffffffffu;
   const uint32_t k_lane = ((lane & 7) | (lane & 8)) * 128;          // row = lane%8 + 8*((lane/8)%2)
   const uint32_t v_lane = ((lane & 7) | ((lane >> 4) << 3)) * 128;  // row = lane%8 + 8*(lane/16)
@@ -170,10 +179,19 @@ __device__ __forceinline__ void attend_slice(WarpAttn<D>& st, const uint32_t (&q
   }
   const bool partial = (t0 < lo) || (t0 + kSliceTokens > hi);
   uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;
+  if (COLS) {
+    const int ta = t0 + (lane >> 2), tb = ta + 8;
+    if (!(ta >= cr.lo0 && ta < cr.hi0)) x[0] = -CUDART_INF_F;
+    if (!(ta >= cr.lo1 && ta < cr.hi1)) x[1] = -CUDART_INF_F;
+    if (!(tb >= cr.lo0 && tb < cr.hi0)) x[2] = -CUDART_INF_F;
+    if (!(tb >= cr.lo1 && tb < cr.hi1)) x[3] = -CUDART_INF_F;
+  }
   if (partial) {
     const int ta = t0 + (lane >> 2), tb = ta + 8;
-    if (!(ta >= lo && ta < hi)) x[0] = x[1] = -CUDART_INF_F;
-    if (!(tb >= lo && tb < hi)) x[2] = x[3] = -CUDART_INF_F;
+    if (!COLS) {
+      if (!(ta >= lo && ta < hi)) x[0] = x[1] = -CUDART_INF_F;
+      if (!(tb >= lo && tb < hi)) x[2] = x[3] = -CUDART_INF_F;
+    }
     // Tokens held by this lane in the V^T fragments: 2*(lane%4) (+1) and +8.
     const int tc = t0 + 2 * (lane & 3);
     auto ok = [&](int t) { return t >= lo && t < hi; };
@@ -189,11 +207,15 @@ __device__ __forceinline__ void attend_slice(WarpAttn<D>& st, const uint32_t (&q
     mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, off));
   }
   const float mn0 = fmaxf(st.m0, mx0), mn1 = fmaxf(st.m1, mx1);
-  const float al0 = exp2f(st.m0 - mn0), al1 = exp2f(st.m1 - mn1);
+  // Reference for the exponentials: the new maximum, or 0 for a column that
+  // has seen no token yet (then every weight and the rescale factor are 0).
+  const float r0 = (COLS && mn0 == -CUDART_INF_F) ? 0.f : mn0;
+  const float r1 = (COLS && mn1 == -CUDART_INF_F) ? 0.f : mn1;
+  const float al0 = exp2f(st.m0 - r0), al1 = exp2f(st.m1 - r1);
   st.m0 = mn0;
   st.m1 = mn1;
-  const uint32_t plo = pack_bf16x2(exp2f(x[0] - mn0), exp2f(x[1] - mn1));
-  const uint32_t phi = pack_bf16x2(exp2f(x[2] - mn0), exp2f(x[3] - mn1));
+  const uint32_t plo = pack_bf16x2(exp2f(x[0] - r0), exp2f(x[1] - r1));
+  const uint32_t phi = pack_bf16x2(exp2f(x[2] - r0), exp2f(x[3] - r1));
   st.l0 = st.l0 * al0 + bf16_lo(plo) + bf16_lo(phi);
   st.l1 = st.l1 * al1 + bf16_hi(plo) + bf16_hi(phi);
 #pragma unroll

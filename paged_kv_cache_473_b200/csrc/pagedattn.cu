@@ -18,6 +18,7 @@
 #include "decode_mma.cuh"
 #include "decode_simt.cuh"
 #include "decode_dynamic.cuh"
+#include "decode_multi.cuh"
 
 namespace {
 
@@ -128,6 +129,7 @@ DecodeParams make_params(const void* q, const void* kc, const void* vc, const in
   p.use_softcap = (softcap > 0.f && std::isfinite(softcap)) ? 1 : 0;
   p.softcap = p.use_softcap ? softcap : 0.f;
   p.inv_softcap = p.use_softcap ? 1.f / softcap : 0.f;
+  p.q_len = 1;
   return p;
 }
 
@@ -196,6 +198,36 @@ cudaError_t launch_mma(const DecodeParams& p, dim3 grid, cudaStream_t st) {
   }
 }
 
+template <int D, int ST, bool SPLIT>
+cudaError_t launch_multi_t(const DecodeParams& p, dim3 grid, int warps, cudaStream_t st) {
+  using Cfg = pa::MultiCfg<D, ST>;
+  CUtensorMap kmap, vmap;
+  const long long rows = (long long)p.num_blocks * p.hkv * p.block_size;
+  if (!tensor_map_encoder()) return cudaErrorNotSupported;
+  if (!encode_cache_map(&kmap, p.k_cache, D, rows) || !encode_cache_map(&vmap, p.v_cache, D, rows))
+    return cudaErrorInvalidValue;
+  auto kern = pa::decode_multi_kernel<D, ST, SPLIT>;
+  static std::atomic<uint64_t> smem_done{0};
+  cudaError_t e = set_smem(kern, Cfg::kSmemBytes, smem_done);
+  if (e != cudaSuccess) return e;
+  return launch_ex(kern, grid, dim3(warps * 32), Cfg::kSmemBytes, st, false, kmap, vmap, p);
+}
+
+// Multi-query rows: one warp per 8 of the T*G query columns of a kv head; the
+// CTA's shared ring holds 32-64 KB of K/V slices.
+template <bool SPLIT>
+cudaError_t launch_multi(const DecodeParams& p, dim3 grid, cudaStream_t st) {
+  const int warps = (p.q_len * p.group + 7) / 8;
+  switch (p.head_dim) {
+    case 64:
+      return launch_multi_t<64, 8, SPLIT>(p, grid, warps, st);
+    case 128:
+      return launch_multi_t<128, 6, SPLIT>(p, grid, warps, st);
+    default:
+      return launch_multi_t<256, 4, SPLIT>(p, grid, warps, st);
+  }
+}
+
 template <typename T, int D, int GP, bool SPLIT, bool APPEND>
 cudaError_t launch_simt_t(const DecodeParams& p, dim3 grid, cudaStream_t st) {
   constexpr int NW = 4;
@@ -239,7 +271,7 @@ cudaError_t launch_decode(const DecodeParams& p, pa_dtype_t dt, pa_kernel_t kern
 template <typename OutT, int NWR>
 cudaError_t launch_combine_n(const DecodeParams& p, cudaStream_t st) {
   constexpr int rows_per_cta = pa::kCombineWarps / NWR;
-  const int rows = p.batch * p.hq;
+  const int rows = p.batch * p.q_len * p.hq;
   dim3 grid((rows + rows_per_cta - 1) / rows_per_cta);
   dim3 block(pa::kCombineWarps * 32);
   switch (p.head_dim) {
@@ -371,8 +403,9 @@ long long splitk_parts(int32_t max_context_len, int32_t P) {
 // at the same place whatever the call's shape, and no call writes partials
 // there, so counters that one call leaves at zero are zero for the next call
 // of any shape or schedule.
-size_t workspace_size(int32_t batch, int32_t num_q_heads, int32_t head_dim, int32_t max_context_len, int32_t P) {
-  const size_t rows = (size_t)batch * num_q_heads * (size_t)splitk_parts(max_context_len, P);
+size_t workspace_size(int32_t batch, int32_t num_q_heads, int32_t head_dim, int32_t max_context_len, int32_t P,
+                      int32_t q_len = 1) {
+  const size_t rows = (size_t)batch * q_len * num_q_heads * (size_t)splitk_parts(max_context_len, P);
   return pa::kCounterBytes + align256(rows * head_dim * 4) + align256(rows * 2 * 4);
 }
 
@@ -611,6 +644,67 @@ pa_status_t pa_decode_step(const void* q, const void* k_new, const void* v_new, 
   c.kernel = kernel;
   c.stream = stream;
   return run_decode(c);
+}
+
+pa_status_t pa_decode_multi(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                            const int32_t* context_lens, int32_t batch, int32_t q_len, int32_t num_q_heads,
+                            int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq,
+                            int32_t num_blocks, float scale, float softcap, int32_t window, void* out,
+                            pa_dtype_t dtype, int32_t partition_tokens, int32_t max_context_len, void* workspace,
+                            size_t workspace_bytes, pa_stream_t stream) {
+  t_last_launches = 0;
+  const Shape s{batch, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks};
+  pa_status_t st = check_decode_args(q, k_cache, v_cache, block_tables, context_lens, s, softcap, out, dtype,
+                                     PA_KERNEL_MMA);
+  if (st != PA_OK) return st;
+  if (q_len <= 0) return PA_ERR_INVALID;
+  if ((long long)q_len * (num_q_heads / num_kv_heads) > pa::kMaxMultiColumns) return PA_ERR_UNSUPPORTED;
+  const bool split = partition_tokens >= 0;
+  int P = kNoSplitPartition;
+  long long parts = 1;
+  if (split) {
+    if (partition_tokens > 0 && partition_tokens % 64 != 0) return PA_ERR_INVALID;
+    if (max_context_len <= 0) return PA_ERR_INVALID;
+    P = auto_partition(batch, num_kv_heads, max_context_len, partition_tokens);
+    parts = splitk_parts(max_context_len, P);
+    if (parts > kMaxPartsPerSeq) return PA_ERR_UNSUPPORTED;
+    const size_t need = workspace_size(batch, num_q_heads, head_dim, max_context_len, P, q_len);
+    if (batch > 0 && (!workspace || !aligned(workspace, 16) || workspace_bytes < need)) return PA_ERR_WORKSPACE;
+  }
+  if (batch == 0) return PA_OK;
+  DecodeParams p = make_params(q, k_cache, v_cache, block_tables, context_lens, s, scale, softcap, window, out);
+  p.q_len = q_len;
+  cudaError_t e;
+  if (split) {
+    p.partition = P;
+    p.max_parts = (int)parts;
+    p.max_context = max_context_len < p.max_context ? max_context_len : p.max_context;
+    const size_t rows = (size_t)batch * q_len * num_q_heads * parts;
+    char* ws = static_cast<char*>(workspace);
+    p.ws_o = reinterpret_cast<float*>(ws + pa::kCounterBytes);
+    p.ws_ml = reinterpret_cast<float*>(ws + pa::kCounterBytes + align256(rows * head_dim * 4));
+    e = launch_multi<true>(p, dim3((unsigned)parts, num_kv_heads, batch), stream);
+    if (e != cudaSuccess) return PA_ERR_CUDA;
+    t_last_launches = 1;
+    if (parts > 1) {
+      e = launch_combine<__nv_bfloat16>(p, stream);
+      if (e != cudaSuccess) return PA_ERR_CUDA;
+      t_last_launches = 2;
+    }
+  } else {
+    e = launch_multi<false>(p, dim3(1, num_kv_heads, batch), stream);
+    if (e != cudaSuccess) return PA_ERR_CUDA;
+    t_last_launches = 1;
+  }
+  return PA_OK;
+}
+
+size_t pa_decode_multi_workspace_size(int32_t batch, int32_t q_len, int32_t num_q_heads, int32_t head_dim,
+                                      int32_t max_context_len, int32_t partition_tokens, int32_t num_kv_heads) {
+  if (batch <= 0 || q_len <= 0 || num_q_heads <= 0 || head_dim <= 0 || partition_tokens < 0) return 0;
+  const int P = auto_partition(batch, num_kv_heads, max_context_len, partition_tokens);
+  if (P <= 0) return 0;
+  return workspace_size(batch, num_q_heads, head_dim, max_context_len, P, q_len);
 }
 
 }  // extern "C"

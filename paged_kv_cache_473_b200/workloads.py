@@ -271,6 +271,33 @@ def make_batch(
     )
 
 
+def make_multi_queries(batch: Batch, q_len: int, seed: Optional[int] = None, device=None) -> dict:
+    """Multi-query inputs for ``batch``: ``q`` ``[B, T, Hq, D]`` for the last
+    ``T = q_len`` positions of every sequence, the new rows ``k_new``/``v_new``
+    ``[B*T, Hkv, D]`` and their slots ``[B*T]`` (int64; position L-T+j of
+    sequence b at row b*T + j, -1 where that position is < 0), all N(0,1)
+    drawn in fp32 and rounded to the workload's dtype."""
+    w = batch.workload
+    B, T = batch.context_lens.numel(), int(q_len)
+    dev = torch.device(device) if device is not None else batch.q.device
+    gd = torch.Generator(device=dev)
+    gd.manual_seed((w.seed if seed is None else seed) * 104729 + 31 * T + 5)
+    dt = w.torch_dtype
+    q = _randn((B, T, w.num_q_heads, w.head_dim), gd, dev, dt)
+    k_new = _randn((B * T, w.num_kv_heads, w.head_dim), gd, dev, dt)
+    v_new = _randn((B * T, w.num_kv_heads, w.head_dim), gd, dev, dt)
+    L = batch.context_lens.to("cpu").to(torch.int64)
+    tables = batch.block_tables.to("cpu")
+    bs = w.block_size
+    slots = torch.full((B * T,), -1, dtype=torch.int64)
+    for b in range(B):
+        for j in range(T):
+            t = int(L[b]) - T + j
+            if t >= 0:
+                slots[b * T + j] = int(tables[b, t // bs]) * bs + t % bs
+    return {"q": q, "k_new": k_new, "v_new": v_new, "slot_mapping": slots.to(dev)}
+
+
 def kv_bytes(batch: Batch, unique: bool = False, window: Optional[int] = None) -> int:
     """KV bytes one decode pass must read: sum over sequences of
     ``L_eff * Hkv * 2 * D * elem_bytes`` (``L_eff`` = attended positions).

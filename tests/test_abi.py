@@ -28,7 +28,8 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ["pa_write_kv", "pa_decode", "pa_decode_splitk", "pa_decode_splitk_workspace_size",
-              "pa_decode_splitk_partition", "pa_device_errors", "pa_error_string", "pa_last_launch_count"]:
+              "pa_decode_splitk_partition", "pa_device_errors", "pa_error_string", "pa_last_launch_count",
+              "pa_decode_step", "pa_decode_splitk_noalloc", "pa_decode_multi", "pa_decode_multi_workspace_size"]:
         assert n in names
 
 
@@ -141,3 +142,41 @@ def test_write_kv_host_checks():
     assert f(A, A, A, -1, A, A, 8, 16, 2, 64, bnd.PA_BF16, None) == bnd.PA_ERR_INVALID
     assert f(A, A, A, 4, A, A, 8, 16, 2, 4, bnd.PA_BF16, None) == bnd.PA_ERR_UNSUPPORTED
     assert f(A, A, A, 0, A, A, 8, 16, 2, 64, bnd.PA_BF16, None) == bnd.PA_OK
+
+
+def _multi(**kw):
+    a = dict(q=A, k=A, v=A, bt=A, cl=A, B=2, T=4, hq=8, hkv=2, d=128, bs=16, mb=4, nb=8, scale=0.1, cap=0.0, win=0,
+             out=A, dt=bnd.PA_BF16, P=-1, maxL=64, ws=None, wsb=0)
+    a.update(kw)
+    return bnd.lib.pa_decode_multi(a["q"], a["k"], a["v"], a["bt"], a["cl"], a["B"], a["T"], a["hq"], a["hkv"],
+                                   a["d"], a["bs"], a["mb"], a["nb"], a["scale"], a["cap"], a["win"], a["out"],
+                                   a["dt"], a["P"], a["maxL"], a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize(
+    "kw,status",
+    [
+        (dict(T=0), bnd.PA_ERR_INVALID),
+        (dict(q=None), bnd.PA_ERR_INVALID),
+        (dict(q=MIS), bnd.PA_ERR_INVALID),
+        (dict(dt=bnd.PA_F32), bnd.PA_ERR_UNSUPPORTED),  # tensor-core path only
+        (dict(T=17), bnd.PA_ERR_UNSUPPORTED),  # 17 * 4 query columns > 64
+        (dict(d=96), bnd.PA_ERR_UNSUPPORTED),
+        (dict(P=0), bnd.PA_ERR_WORKSPACE),  # split without a workspace
+        (dict(P=100, ws=A, wsb=1 << 30), bnd.PA_ERR_INVALID),  # not a multiple of 64
+        (dict(P=0, maxL=0, ws=A, wsb=1 << 30), bnd.PA_ERR_INVALID),
+        (dict(B=0), bnd.PA_OK),
+        (dict(B=0, P=0), bnd.PA_OK),
+    ],
+)
+def test_multi_host_checks(kw, status):
+    assert _multi(**kw) == status
+    assert pa.last_launch_count() == 0
+
+
+def test_multi_workspace_size_formula():
+    B, T, hq, d, maxL, P = 8, 4, 32, 128, 8192, 512
+    rows = B * T * hq * (-(-maxL // P))
+    al = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    assert pa.decode_multi_workspace_size(B, T, hq, d, maxL, P, 8) == 256 * 1024 + al(rows * d * 4) + al(rows * 8)
+    assert pa.decode_multi_workspace_size(B, T, hq, d, maxL, -1, 8) == 0
