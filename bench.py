@@ -313,6 +313,41 @@ class Runner:
         return g, ev
 
 
+class MultiRunner(Runner):
+    """Multi-query rows on one workload: T query tokens per sequence whose K/V
+    rows are already in the cache (positions L-T .. L-1), attending causally
+    (pa_decode_multi, library-chosen split).  A step is only that call."""
+
+    def __init__(self, w: wl.Workload, rank: int, q_len: int):
+        super().__init__(w, rank, "auto", True, 0, fused=True)
+        b = self.batch
+        for kc, vc in self.pools:  # make position L-1 live too: every query position is in the cache
+            self.pa.write_kv(b.k_new, b.v_new, b.slot_mapping, kc, vc)
+        self.T = q_len
+        self.q = wl.make_multi_queries(b, q_len)["q"]
+        self.out = torch.empty_like(self.q)
+        nbytes = self.pa.decode_multi_workspace_size(self.B, q_len, w.num_q_heads, w.head_dim, self.max_ctx, 0,
+                                                     w.num_kv_heads)
+        self.ws = torch.zeros(max(16, nbytes), dtype=torch.uint8, device="cuda")
+        torch.cuda.synchronize()
+
+    def decode(self, r, x):
+        w, b = self.w, self.batch
+        kc, vc = self.pools[r]
+        self.pa.decode_multi(self.q, kc, vc, b.block_tables, b.context_lens, w.scale, w.softcap, w.window,
+                             split=True, max_context_len=self.max_ctx, partition_tokens=0, out=self.out,
+                             workspace=self.ws)
+        return self.pa.last_launch_count()
+
+    def step(self, r, x=None, ev=None):
+        if ev is not None:
+            ev[0].record()
+        n = self.decode(r, None)
+        if ev is not None:
+            ev[1].record()
+        self.launches_per_step = n
+
+
 def run_timed(runner: Runner, K: int, W: int, world: int, device_index: int):
     """Warm up W steps, then time exactly K graph-replayed steps."""
     for i in range(W):
@@ -488,6 +523,31 @@ def shape_summary(w: wl.Workload, rank: int, kernel: str, K: int, W: int, world:
     return res
 
 
+def multi_summary(w: wl.Workload, q_len: int, rank: int, K: int, W: int, world: int, dev_idx: int, peak: float):
+    """Multi-query rows (pa_decode_multi) on a decode workload: tokens/s counts
+    the B*T query tokens of a step."""
+    runner = MultiRunner(w, rank, q_len)
+    total_ms, _, _ = run_timed(runner, K, W, world, dev_idx)
+    ms = total_ms / K
+    gbs = runner.kv_bytes / (ms * 1e-3) / 1e9
+    res = {
+        "q_len": q_len,
+        "tokens_per_s": round(runner.B * q_len / (ms * 1e-3), 1),
+        "ms_per_step": round(ms, 5),
+        "decode_gbs": round(gbs, 1),
+        "decode_frac": round(gbs / peak, 4),
+        "launches_per_step": runner.launches_per_step,
+        "flop_per_kv_byte": q_len * w.num_q_heads // w.num_kv_heads * (1 if w.elem_bytes == 2 else 2),
+        "kv_bytes": runner.kv_bytes,
+    }
+    del runner
+    torch.cuda.empty_cache()
+    return res
+
+
+MULTI_SHAPES = (("tinyllama_1b", 4), ("llama3_8b", 4), ("gemma2_2b", 8))
+
+
 def main_ours(args, world, rank, local):
     w = wl.WORKLOADS[args.workload]
     split = not args.no_split
@@ -558,6 +618,9 @@ def main_ours(args, world, rank, local):
             extra[n] = shape_summary(wl.WORKLOADS[n], rank, args.kernel, 50, 5, world, local, peak)
             if wl.WORKLOADS[n].partition_tokens:  # also the dynamic schedule
                 extra[n + "@dynamic"] = shape_summary(wl.WORKLOADS[n], rank, args.kernel, 50, 5, world, local, peak, 0)
+        for n, T in MULTI_SHAPES:
+            if args.shapes == "auto" or n in names or n == w.name:
+                extra[f"{n}@multi{T}"] = multi_summary(wl.WORKLOADS[n], T, rank, 50, 5, world, local, peak)
         line["per_shape"] = extra
         runner = None
     if world == 1 and rank == 0 and not args.no_cpu:
