@@ -17,6 +17,9 @@ CPU tensors into it.  The functions below follow these passages:
 * ``decode_multi`` -- several query tokens per sequence with a causal mask
   (the README's "Features": chunked prefill, speculative decoding); each query
   token is the decode above over the positions up to its own.
+* ``prefill`` -- ``write_kv`` of a prompt's (or chunk's) rows followed by
+  ``decode_multi`` per sequence ("Key Concepts Explained: KV Cache": prefill
+  computes and stores the prompt's keys and values).
 
 Pins (tests/test_oracle_pins.py): agreement with torch's fp64
 ``scaled_dot_product_attention`` on contiguous K/V, permutation invariance over
@@ -179,6 +182,28 @@ def decode_multi(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, 
                                      cap64, int(window), None if rows_arr is None else rows_arr.data_ptr(), n_rows,
                                      out.ctypes.data)
     _check(st)
+    return out
+
+
+def prefill(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, slot_mapping: torch.Tensor,
+            cu_q_lens: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_tables: torch.Tensor,
+            context_lens: torch.Tensor, scale: float, softcap: float = 0.0, window: int = 0) -> np.ndarray:
+    """Paged prefill: append the new rows (``write_kv``, in place on the CPU
+    caches), then sequence b's query rows ``[cu[b], cu[b+1])`` -- its last
+    ``T_b`` positions -- attend causally (``decode_multi`` with ``T = T_b``).
+    Returns ``[total, Hq, D]`` fp64."""
+    if k_new is not None:
+        write_kv(k_new, v_new, slot_mapping, k_cache, v_cache)
+    cu = [int(x) for x in _cpu(cu_q_lens)]
+    q = _cpu(q)
+    tables, lens = _cpu(block_tables), _cpu(context_lens)
+    out = np.zeros((q.shape[0], q.shape[1], q.shape[2]), dtype=np.float64)
+    for b in range(len(cu) - 1):
+        T = cu[b + 1] - cu[b]
+        if T == 0:
+            continue
+        out[cu[b]:cu[b + 1]] = decode_multi(q[cu[b]:cu[b + 1]].unsqueeze(0), k_cache, v_cache, tables[b:b + 1],
+                                            lens[b:b + 1], scale, softcap, window)[0]
     return out
 
 

@@ -378,3 +378,51 @@ def test_multi_queries_before_the_start_give_zero_rows_and_rows_match():
     part = oracle.decode_multi(q, kc, vc, tables, cl, 0.25, rows=rows)
     for r, (b, j, h) in enumerate(rows):
         assert np.array_equal(part[r], full[b, j, h])
+
+
+# ---- prefill (append a prompt, attend it causally) --------------------------------
+
+
+@pytest.mark.parametrize("hq,hkv,bs", [(8, 2, 4), (4, 4, 16), (6, 1, 8)])
+def test_prefill_from_scratch_equals_causal_attention(hq, hkv, bs):
+    """Prompts written into an empty paged cache and attended in one call are
+    causal self-attention over each prompt (torch fp64, is_causal)."""
+    gen = torch.Generator().manual_seed(71 + hq + bs)
+    d, lens = 16, [1, 7, 20, 13]
+    B = len(lens)
+    ks, vs = _rand_seqs(gen, lens, hkv, d)
+    qs = [torch.randn((L, hq, d), generator=gen) for L in lens]
+    kc, vc, tables, cl = scatter_to_pool(ks, vs, bs, gen)
+    kc.fill_(float("nan"))  # the cache starts empty: prefill must write every row itself
+    vc.fill_(float("nan"))
+    cu = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int32)
+    slots = []
+    for b, L in enumerate(lens):
+        slots += [int(tables[b, t // bs]) * bs + t % bs for t in range(L)]
+    got = oracle.prefill(torch.cat(qs), torch.cat(ks), torch.cat(vs), torch.tensor(slots, dtype=torch.int64), cu, kc,
+                         vc, tables, cl, 0.25)
+    for b, L in enumerate(lens):
+        ref = F.scaled_dot_product_attention(qs[b].double().permute(1, 0, 2).unsqueeze(0),
+                                             ks[b].double().permute(1, 0, 2).unsqueeze(0),
+                                             vs[b].double().permute(1, 0, 2).unsqueeze(0), is_causal=True,
+                                             scale=0.25, enable_gqa=True)[0].permute(1, 0, 2)
+        assert np.max(np.abs(got[int(cu[b]):int(cu[b + 1])] - ref.numpy())) <= 1e-12
+
+
+def test_chunked_prefill_equals_one_shot_prefill():
+    """Two chunks (the second attending the first from the cache) give the
+    rows of a single prefill of the whole prompt."""
+    gen = torch.Generator().manual_seed(73)
+    hq, hkv, d, bs, L, c1 = 4, 2, 16, 4, 19, 8
+    ks, vs = _rand_seqs(gen, [L], hkv, d)
+    q = torch.randn((L, hq, d), generator=gen)
+    kc, vc, tables, cl = scatter_to_pool(ks, vs, bs, gen)
+    slots = torch.tensor([int(tables[0, t // bs]) * bs + t % bs for t in range(L)], dtype=torch.int64)
+    one = oracle.prefill(q, ks[0], vs[0], slots, torch.tensor([0, L], dtype=torch.int32), kc.clone(), vc.clone(),
+                         tables, cl, 0.3)
+    kc2, vc2 = kc.clone(), vc.clone()
+    first = oracle.prefill(q[:c1], ks[0][:c1], vs[0][:c1], slots[:c1], torch.tensor([0, c1], dtype=torch.int32),
+                           kc2, vc2, tables, torch.tensor([c1], dtype=torch.int32), 0.3)
+    second = oracle.prefill(q[c1:], ks[0][c1:], vs[0][c1:], slots[c1:], torch.tensor([0, L - c1], dtype=torch.int32),
+                            kc2, vc2, tables, cl, 0.3)
+    assert np.array_equal(np.concatenate([first, second]), one)
