@@ -229,6 +229,37 @@ size_t pa_decode_multi_workspace_size(int32_t batch, int32_t q_len, int32_t num_
                                       int32_t max_context_len, int32_t partition_tokens, int32_t num_kv_heads);
 
 /*
+ * pa_prefill -- paged prefill: append a batch of prompts' (or prompt chunks')
+ * key/value rows and attend them causally over the paged cache.
+ *   Sequence b's new tokens are rows [cu_q_lens[b], cu_q_lens[b+1]) of q
+ *   ([total_q][num_q_heads][head_dim]), k_new, v_new ([total_q][num_kv_heads]
+ *   [head_dim]), slot_mapping ([total_q] int64) and out (like q): T_b tokens,
+ *   the last T_b positions of the context, L = context_lens[b] (which counts
+ *   them).  cu_q_lens: [batch + 1] int32 device array, non-decreasing, with
+ *   cu_q_lens[batch] <= total_q and every T_b <= max_q_len (else
+ *   PA_DEVERR_CONTEXT and the sequence's rows are not written).
+ *   First the rows are appended exactly as pa_write_kv(k_new, v_new,
+ *   slot_mapping, total_q) does; pass k_new = v_new = NULL to skip the append
+ *   when the rows are already in the cache.  Then token j of sequence b, at
+ *   position p = L - T_b + j, attends positions [s0, p] as in pa_decode_multi
+ *   (causal, window, softcap).  A chunk of a chunked prefill is the same call
+ *   with the earlier chunks already in the cache.
+ *   bf16 only.  One launch for the append and one for the attention, whose
+ *   CTAs each take 64 / G query tokens of one sequence and one kv head; no
+ *   workspace.
+ *   Passages: nano-vllm (ovshake) README, "Key Concepts Explained: KV Cache"
+ *   (prefill processes the prompt and stores its keys and values) and
+ *   "Features" (chunked prefill); MinivLLM (the pages' second project) times
+ *   prefilling and decoding separately.
+ */
+pa_status_t pa_prefill(const void* q, const void* k_new, const void* v_new, const int64_t* slot_mapping,
+                       const int32_t* cu_q_lens, int32_t total_q, int32_t max_q_len, void* k_cache, void* v_cache,
+                       const int32_t* block_tables, const int32_t* context_lens, int32_t batch, int32_t num_q_heads,
+                       int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq,
+                       int32_t num_blocks, float scale, float softcap, int32_t window, void* out, pa_dtype_t dtype,
+                       pa_stream_t stream);
+
+/*
  * pa_decode_splitk_noalloc -- pa_decode_splitk for callers that cannot allocate
  * device memory.
  *   The pages describe no such call; it exists for callers that must not call

@@ -24,6 +24,7 @@ from ._binding import (  # noqa: F401
     error_string,
     last_launch_count,
     lib,
+    prefill,
     write_kv,
 )
 
@@ -40,5 +41,6 @@ __all__ = [
     "device_errors",
     "error_string",
     "last_launch_count",
+    "prefill",
     "PagedAttnError",
 ]

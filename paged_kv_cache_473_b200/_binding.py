@@ -65,6 +65,10 @@ def _load_library() -> ctypes.CDLL:
     lib.pa_decode_multi.restype = _c_i32
     lib.pa_decode_multi_workspace_size.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32]
     lib.pa_decode_multi_workspace_size.restype = _c_sz
+    lib.pa_prefill.argtypes = [_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_i32, _c_i32, _c_vp, _c_vp, _c_vp, _c_vp, _c_i32,
+                               _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_f32, _c_f32, _c_i32, _c_vp, _c_i32,
+                               _c_vp]
+    lib.pa_prefill.restype = _c_i32
     lib.pa_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint32), _c_i32]
     lib.pa_device_errors.restype = _c_i32
     lib.pa_error_string.argtypes = [_c_i32]
@@ -237,6 +241,27 @@ def decode_multi(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, 
                              hkv, d, bs, block_tables.shape[1], nb, float(scale), float(softcap), int(window),
                              _ptr(out), _dtype_code(q), ptoks, int(max_context_len), wptr, wbytes, _stream(stream))
     _check(st, "pa_decode_multi")
+    return out
+
+
+def prefill(q: torch.Tensor, k_new: Optional[torch.Tensor], v_new: Optional[torch.Tensor],
+            slot_mapping: Optional[torch.Tensor], cu_q_lens: torch.Tensor, k_cache: torch.Tensor,
+            v_cache: torch.Tensor, block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
+            softcap: float = 0.0, window: int = 0, *, max_q_len: int, out: Optional[torch.Tensor] = None,
+            stream=None) -> torch.Tensor:
+    """Paged prefill: append ``k_new``/``v_new`` ``[total, Hkv, D]`` at
+    ``slot_mapping`` (skipped when both are None), then sequence b's query
+    rows ``q[cu_q_lens[b]:cu_q_lens[b+1]]`` -- its last positions -- attend
+    causally.  ``max_q_len`` bounds every sequence's row count."""
+    total, hq, d = q.shape
+    nb, hkv, bs, _ = k_cache.shape
+    if out is None:
+        out = torch.empty_like(q)
+    st = lib.pa_prefill(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(slot_mapping), _ptr(cu_q_lens), total,
+                        int(max_q_len), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
+                        cu_q_lens.numel() - 1, hq, hkv, d, bs, block_tables.shape[1], nb, float(scale),
+                        float(softcap), int(window), _ptr(out), _dtype_code(q), _stream(stream))
+    _check(st, "pa_prefill")
     return out
 
 

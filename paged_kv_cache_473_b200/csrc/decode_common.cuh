@@ -38,6 +38,10 @@ struct DecodeParams {
   int merge_in_kernel;          // dynamic schedule: the last partial of a unit merges it (else the combine kernel)
   int batch, hq, hkv, group, head_dim;
   int q_len;        // query tokens per sequence (1 for decode; T for the multi-query rows [B][T][Hq][D])
+  const int32_t* cu_q;  // prefill: sequence b's query rows are [cu_q[b], cu_q[b+1]) of [total][Hq][D] (else null)
+  int q_tile;           // prefill: query tokens per CTA
+  int max_q_len;        // prefill: bound on cu_q[b+1] - cu_q[b] (the grid covers it)
+  int total_q;          // prefill: rows of q and out (bound on cu_q[B])
   int block_size, log2_bs, max_blocks, num_blocks;
   int window;
   int partition;    // tokens per partition (a multiple of 64); 1 << 30 without split

@@ -15,6 +15,12 @@
 // for that before it refills the stage.  Each warp writes its own columns:
 // the normalised rows when the sequence's range is one partition, else the
 // partial state for the combine kernel.
+//
+// Prefill (p.cu_q set): the same kernel over variable-length query blocks.
+// Sequence b's new tokens are rows [cu_q[b], cu_q[b+1]) of q and out, T_b of
+// them, the last T_b positions of its context; CTA x takes the query tile of
+// tokens [x*q_tile, x*q_tile + q_tile) (q_tile*G <= 64 columns) and attends,
+// without split, the union of its tokens' causal ranges.
 #pragma once
 
 #include "decode_common.cuh"
@@ -35,18 +41,19 @@ struct MultiCfg {
   static constexpr int kSmemBytes = kRingBytes + 2 * ST * 8 + 1024;
 };
 
-// Token range of query column c (token j = c / G) inside the CTA's partition
-// [pl, ph): [max(s0_j, pl), min(p_j + 1, ph)).  Padding columns (c >= T*G)
-// take the CTA's union range so that their (discarded) softmax stays finite.
-__device__ __forceinline__ void column_range(int c, int G, int T, int L, int window, int pl, int ph, int ulo,
-                                             int uhi, int& lo, int& hi) {
-  if (c >= T * G) {
+// Token range of query column c (token j = j0 + c / G of the T) inside the
+// CTA's partition [pl, ph): [max(s0_j, pl), min(p_j + 1, ph)).  Padding
+// columns (c >= ntok*G) take the CTA's union range so that their (discarded)
+// softmax stays finite.
+__device__ __forceinline__ void column_range(int c, int G, int T, int j0, int ntok, int L, int window, int pl, int ph,
+                                             int ulo, int uhi, int& lo, int& hi) {
+  if (c >= ntok * G) {
     lo = ulo;
     hi = uhi;
     return;
   }
-  const int end = L - T + c / G + 1;  // p_j + 1
-  lo = max(window_start(end, window), pl);
+  const int end = L - T + j0 + c / G + 1;  // p_j + 1
+  lo = max(window_start(max(end, 0), window), pl);
   hi = min(end, ph);
 }
 
@@ -63,31 +70,56 @@ __global__ void __launch_bounds__(kMaxMultiColumns / 8 * 32)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int NW = blockDim.x >> 5;
-  const int part = SPLIT ? (int)blockIdx.x : 0;
   const int g = blockIdx.y, b = blockIdx.z;
-  const int G = p.group, T = p.q_len, P = p.partition;
+  const int G = p.group, P = p.partition;
+  const bool varlen = p.cu_q != nullptr;
 
-  const int L = clamp_context(p, b, threadIdx.x == 0 && part == 0);
-  // The union of the query tokens' ranges is [s0 of token 0, L).
-  const int ulo_seq = window_start(max(L - T + 1, 0), p.window);
-  const int n_parts = (L > ulo_seq) ? (L + P - 1) / P - ulo_seq / P : 0;
+  // This CTA's query tokens: j0 .. j0 + ntok - 1 of the sequence's T, at q/out
+  // rows row0 .. row0 + ntok - 1 (times Hq).
+  int part, T, j0, ntok;
+  size_t row0;
+  if (varlen) {
+    const int a = p.cu_q[b], e = p.cu_q[b + 1];
+    if (a < 0 || e < a || e > p.total_q || e - a > p.max_q_len) {  // malformed offsets: report, write nothing
+      if (blockIdx.x == 0 && g == 0 && threadIdx.x == 0) raise_error(PA_DEVERR_CONTEXT);
+      return;
+    }
+    T = e - a;
+    part = 0;
+    j0 = blockIdx.x * p.q_tile;
+    ntok = min(p.q_tile, T - j0);
+    row0 = (size_t)a + j0;
+    if (ntok <= 0) return;
+  } else {
+    part = SPLIT ? (int)blockIdx.x : 0;
+    T = p.q_len;
+    j0 = 0;
+    ntok = T;
+    row0 = (size_t)b * T;
+  }
+
+  const int L = clamp_context(p, b, threadIdx.x == 0 && part == 0 && j0 == 0);
+  // The union of the tile's ranges is [s0 of its first token, p of its last + 1).
+  const int uend = min(L, L - T + j0 + ntok);
+  const int ulo_seq = window_start(max(L - T + j0 + 1, 0), p.window);
+  const int n_parts = (uend > ulo_seq) ? (uend + P - 1) / P - ulo_seq / P : 0;
   const bool final_write = !SPLIT || n_parts == 1;
   const int pl = part * P, ph = pl + P;
-  const int ulo = max(ulo_seq, pl), uhi = min(L, ph);
+  const int ulo = max(ulo_seq, pl), uhi = min(uend, ph);
 
   // This lane's two accumulator columns and their ranges.
   const int n0 = 2 * (lane & 3);
   const int c0 = warp * 8 + n0;
   ColRange cr;
-  column_range(c0, G, T, L, p.window, pl, ph, ulo, uhi, cr.lo0, cr.hi0);
-  column_range(c0 + 1, G, T, L, p.window, pl, ph, ulo, uhi, cr.lo1, cr.hi1);
+  column_range(c0, G, T, j0, ntok, L, p.window, pl, ph, ulo, uhi, cr.lo0, cr.hi0);
+  column_range(c0 + 1, G, T, j0, ntok, L, p.window, pl, ph, ulo, uhi, cr.lo1, cr.hi1);
 
-  // Output row (or workspace row) of column c: ((b*T + j)*Hq + g*G + h).
-  auto row_of = [&](int c) { return ((size_t)b * T + c / G) * p.hq + (size_t)g * G + c % G; };
+  // Output row (or workspace row) of column c: ((row0 + c / G)*Hq + g*G + h).
+  auto row_of = [&](int c) { return (row0 + c / G) * p.hq + (size_t)g * G + c % G; };
 
   if (ulo >= uhi) {  // nothing of this sequence falls in this partition
-    if (n_parts == 0 && part == 0) {  // L == 0: zero rows for every query column
-      for (int idx = threadIdx.x; idx < T * G * D; idx += blockDim.x)
+    if (n_parts == 0 && part == 0) {  // no position for any token: zero rows for every query column
+      for (int idx = threadIdx.x; idx < ntok * G * D; idx += blockDim.x)
         static_cast<__nv_bfloat16*>(p.out)[row_of(idx / D) * D + idx % D] = __float2bfloat16_rn(0.f);
     }
     return;
@@ -108,13 +140,13 @@ __global__ void __launch_bounds__(kMaxMultiColumns / 8 * 32)
   }
   __syncthreads();
 
-  const int j0 = ulo / kSliceTokens;
-  const int n = (uhi + kSliceTokens - 1) / kSliceTokens - j0;
+  const int js = ulo / kSliceTokens;  // first 16-token slice
+  const int n = (uhi + kSliceTokens - 1) / kSliceTokens - js;
   const int32_t* table = p.block_tables + (size_t)b * p.max_blocks;
 
   // Warp 0 issues slice i into stage i % ST.
   auto issue = [&](int i) {
-    const int t = (j0 + i) * kSliceTokens;
+    const int t = (js + i) * kSliceTokens;
     const int phys = table[t >> p.log2_bs];
     const int y = (phys >= 0 && phys < p.num_blocks) ? cache_row(p, phys, g, t) : -1;
     issue_slice<D>(ring + (i % ST) * Cfg::kStageBytes, full + 8 * (i % ST), &kmap, &vmap, y, lane);
@@ -128,7 +160,7 @@ __global__ void __launch_bounds__(kMaxMultiColumns / 8 * 32)
   uint32_t qf[D / 16][2];
   {
     const int c = warp * 8 + (lane >> 2);
-    const bool real = c < T * G;
+    const bool real = c < ntok * G;
     const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q) + row_of(real ? c : 0) * D;
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
@@ -153,7 +185,7 @@ __global__ void __launch_bounds__(kMaxMultiColumns / 8 * 32)
       break;
     }
     const uint32_t kbase = ring + s * Cfg::kStageBytes;
-    attend_slice<D, true>(st, qf, kbase, kbase + Cfg::kSliceBytes, (j0 + i) * kSliceTokens, ulo, uhi, qk_scale, p,
+    attend_slice<D, true>(st, qf, kbase, kbase + Cfg::kSliceBytes, (js + i) * kSliceTokens, ulo, uhi, qk_scale, p,
                           lane, cr);
     __syncwarp();
     if (lane == 0) mbar_arrive(empty + 8 * s);
@@ -179,7 +211,7 @@ __global__ void __launch_bounds__(kMaxMultiColumns / 8 * 32)
   st.reduce_sums();
 
   // ---- this warp's columns: final rows or partials, from registers -----------------
-  const int cols = T * G;
+  const int cols = ntok * G;
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
     const int c = c0 + e;

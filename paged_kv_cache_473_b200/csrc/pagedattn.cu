@@ -213,11 +213,12 @@ cudaError_t launch_multi_t(const DecodeParams& p, dim3 grid, int warps, cudaStre
   return launch_ex(kern, grid, dim3(warps * 32), Cfg::kSmemBytes, st, false, kmap, vmap, p);
 }
 
-// Multi-query rows: one warp per 8 of the T*G query columns of a kv head; the
-// CTA's shared ring holds 32-64 KB of K/V slices.
+// Multi-query rows: one warp per 8 of the T*G query columns of a kv head (or
+// of the q_tile*G columns of a prefill tile); the CTA's shared ring holds
+// 32-64 KB of K/V slices.
 template <bool SPLIT>
 cudaError_t launch_multi(const DecodeParams& p, dim3 grid, cudaStream_t st) {
-  const int warps = (p.q_len * p.group + 7) / 8;
+  const int warps = ((p.cu_q ? p.q_tile : p.q_len) * p.group + 7) / 8;
   switch (p.head_dim) {
     case 64:
       return launch_multi_t<64, 8, SPLIT>(p, grid, warps, st);
@@ -696,6 +697,42 @@ pa_status_t pa_decode_multi(const void* q, const void* k_cache, const void* v_ca
     if (e != cudaSuccess) return PA_ERR_CUDA;
     t_last_launches = 1;
   }
+  return PA_OK;
+}
+
+pa_status_t pa_prefill(const void* q, const void* k_new, const void* v_new, const int64_t* slot_mapping,
+                       const int32_t* cu_q_lens, int32_t total_q, int32_t max_q_len, void* k_cache, void* v_cache,
+                       const int32_t* block_tables, const int32_t* context_lens, int32_t batch, int32_t num_q_heads,
+                       int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq,
+                       int32_t num_blocks, float scale, float softcap, int32_t window, void* out, pa_dtype_t dtype,
+                       pa_stream_t stream) {
+  t_last_launches = 0;
+  const Shape s{batch, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks};
+  pa_status_t st = check_decode_args(q, k_cache, v_cache, block_tables, context_lens, s, softcap, out, dtype,
+                                     PA_KERNEL_MMA);
+  if (st != PA_OK) return st;
+  if (total_q < 0 || max_q_len < 0) return PA_ERR_INVALID;
+  if (batch == 0 || total_q == 0 || max_q_len == 0) return PA_OK;
+  if (!cu_q_lens || !aligned(cu_q_lens, 4)) return PA_ERR_INVALID;
+  const bool append = k_new != nullptr || v_new != nullptr;
+  if (append) {
+    if (!k_new || !v_new || !slot_mapping) return PA_ERR_INVALID;
+    st = pa_write_kv(k_new, v_new, slot_mapping, total_q, k_cache, v_cache, num_blocks, block_size, num_kv_heads,
+                     head_dim, dtype, stream);
+    if (st != PA_OK) return st;
+  }
+  const int G = num_q_heads / num_kv_heads;
+  const int q_tile = pa::kMaxMultiColumns / G;  // G <= 8: 8 .. 64 tokens per CTA
+  const long long tiles = ((long long)max_q_len + q_tile - 1) / q_tile;
+  if (tiles > INT_MAX) return PA_ERR_UNSUPPORTED;
+  DecodeParams p = make_params(q, k_cache, v_cache, block_tables, context_lens, s, scale, softcap, window, out);
+  p.cu_q = cu_q_lens;
+  p.q_tile = q_tile;
+  p.max_q_len = max_q_len;
+  p.total_q = total_q;
+  cudaError_t e = launch_multi<false>(p, dim3((unsigned)tiles, num_kv_heads, batch), stream);
+  if (e != cudaSuccess) return PA_ERR_CUDA;
+  t_last_launches = append ? 2 : 1;
   return PA_OK;
 }
 

@@ -298,6 +298,39 @@ def make_multi_queries(batch: Batch, q_len: int, seed: Optional[int] = None, dev
     return {"q": q, "k_new": k_new, "v_new": v_new, "slot_mapping": slots.to(dev)}
 
 
+def make_prefill_inputs(batch: Batch, q_lens, seed: Optional[int] = None, device=None) -> dict:
+    """Prefill inputs for ``batch``: sequence b's last ``q_lens[b]`` positions
+    are new.  Returns ``q`` ``[total, Hq, D]``, ``k_new``/``v_new`` ``[total,
+    Hkv, D]``, their slots ``[total]`` (int64), ``cu_q_lens`` ``[B+1]`` (int32)
+    and ``max_q_len``, N(0,1) drawn in fp32 and rounded to the workload's dtype."""
+    w = batch.workload
+    ql = [int(x) for x in q_lens]
+    B = batch.context_lens.numel()
+    assert len(ql) == B
+    total = sum(ql)
+    dev = torch.device(device) if device is not None else batch.q.device
+    gd = torch.Generator(device=dev)
+    gd.manual_seed((w.seed if seed is None else seed) * 15485863 + total)
+    dt = w.torch_dtype
+    q = _randn((max(total, 1), w.num_q_heads, w.head_dim), gd, dev, dt)[:total]
+    k_new = _randn((max(total, 1), w.num_kv_heads, w.head_dim), gd, dev, dt)[:total]
+    v_new = _randn((max(total, 1), w.num_kv_heads, w.head_dim), gd, dev, dt)[:total]
+    L = batch.context_lens.to("cpu").to(torch.int64)
+    tables = batch.block_tables.to("cpu")
+    bs = w.block_size
+    slots = torch.full((total,), -1, dtype=torch.int64)
+    cu = [0]
+    for b in range(B):
+        for j in range(ql[b]):
+            t = int(L[b]) - ql[b] + j
+            if t >= 0:
+                slots[cu[-1] + j] = int(tables[b, t // bs]) * bs + t % bs
+        cu.append(cu[-1] + ql[b])
+    return {"q": q.contiguous(), "k_new": k_new.contiguous(), "v_new": v_new.contiguous(),
+            "slot_mapping": slots.to(dev), "cu_q_lens": torch.tensor(cu, dtype=torch.int32, device=dev),
+            "max_q_len": max(ql) if ql else 0}
+
+
 def kv_bytes(batch: Batch, unique: bool = False, window: Optional[int] = None) -> int:
     """KV bytes one decode pass must read: sum over sequences of
     ``L_eff * Hkv * 2 * D * elem_bytes`` (``L_eff`` = attended positions).

@@ -29,7 +29,8 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ["pa_write_kv", "pa_decode", "pa_decode_splitk", "pa_decode_splitk_workspace_size",
               "pa_decode_splitk_partition", "pa_device_errors", "pa_error_string", "pa_last_launch_count",
-              "pa_decode_step", "pa_decode_splitk_noalloc", "pa_decode_multi", "pa_decode_multi_workspace_size"]:
+              "pa_decode_step", "pa_decode_splitk_noalloc", "pa_decode_multi", "pa_decode_multi_workspace_size",
+              "pa_prefill"]:
         assert n in names
 
 
@@ -180,3 +181,32 @@ def test_multi_workspace_size_formula():
     al = lambda x: (x + 255) // 256 * 256  # noqa: E731
     assert pa.decode_multi_workspace_size(B, T, hq, d, maxL, P, 8) == 256 * 1024 + al(rows * d * 4) + al(rows * 8)
     assert pa.decode_multi_workspace_size(B, T, hq, d, maxL, -1, 8) == 0
+
+
+def _prefill(**kw):
+    a = dict(q=A, kn=A, vn=A, sl=A, cu=A, total=64, maxq=32, k=A, v=A, bt=A, cl=A, B=2, hq=8, hkv=2, d=128, bs=16,
+             mb=4, nb=8, scale=0.1, cap=0.0, win=0, out=A, dt=bnd.PA_BF16)
+    a.update(kw)
+    return bnd.lib.pa_prefill(a["q"], a["kn"], a["vn"], a["sl"], a["cu"], a["total"], a["maxq"], a["k"], a["v"],
+                              a["bt"], a["cl"], a["B"], a["hq"], a["hkv"], a["d"], a["bs"], a["mb"], a["nb"],
+                              a["scale"], a["cap"], a["win"], a["out"], a["dt"], None)
+
+
+@pytest.mark.parametrize(
+    "kw,status",
+    [
+        (dict(cu=None), bnd.PA_ERR_INVALID),
+        (dict(cu=A + 2), bnd.PA_ERR_INVALID),
+        (dict(total=-1), bnd.PA_ERR_INVALID),
+        (dict(kn=None), bnd.PA_ERR_INVALID),  # k_new without v_new
+        (dict(sl=None), bnd.PA_ERR_INVALID),
+        (dict(dt=bnd.PA_F32), bnd.PA_ERR_UNSUPPORTED),
+        (dict(hq=24, hkv=2), bnd.PA_ERR_UNSUPPORTED),  # group 12 > 8
+        (dict(B=0), bnd.PA_OK),
+        (dict(total=0), bnd.PA_OK),
+        (dict(maxq=0), bnd.PA_OK),
+    ],
+)
+def test_prefill_host_checks(kw, status):
+    assert _prefill(**kw) == status
+    assert pa.last_launch_count() == 0

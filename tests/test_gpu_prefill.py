@@ -1,0 +1,89 @@
+"""GPU parity of paged prefill (pa_prefill) against the CPU oracle: prompts (or
+prompt chunks) of different lengths appended into the paged cache and attended
+causally.  The append must be bit-exact; the attention within the decode
+tolerances (bf16: max-abs 2e-2, mean-abs 2e-3)."""
+
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_473_b200 as pa
+from paged_kv_cache_473_b200 import workloads as wl
+from tests.gpu_helpers import assert_close, bits, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _clear_device_errors():
+    if torch.cuda.is_available():
+        pa.device_errors()
+    yield
+
+
+def _run(name, lengths, q_lens, window=None, softcap=None, append=True):
+    w = wl.WORKLOADS[name].replace(prefix_share=0.0)
+    b_cpu = wl.make_batch(w, lengths=lengths, prefilled=True)
+    x = wl.make_prefill_inputs(b_cpu, q_lens)
+    b = to_dev(b_cpu)
+    win = w.window if window is None else window
+    cap = w.softcap if softcap is None else softcap
+    kc, vc = b.k_cache.clone(), b.v_cache.clone()
+    dev = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+    out = pa.prefill(dev["q"], dev["k_new"] if append else None, dev["v_new"] if append else None,
+                     dev["slot_mapping"] if append else None, dev["cu_q_lens"], kc, vc, b.block_tables,
+                     b.context_lens, w.scale, cap, win, max_q_len=x["max_q_len"])
+    torch.cuda.synchronize()
+    kc_ref, vc_ref = b_cpu.k_cache.clone(), b_cpu.v_cache.clone()
+    ref = oracle.prefill(x["q"], x["k_new"] if append else None, x["v_new"], x["slot_mapping"], x["cu_q_lens"],
+                         kc_ref, vc_ref, b_cpu.block_tables, b_cpu.context_lens, w.scale, cap, win)
+    return w, out, ref, (kc, vc), (kc_ref, vc_ref)
+
+
+@pytest.mark.parametrize("name", ["tinyllama_1b", "gemma2_2b", "llama3_8b"])
+def test_prefill_prompts_from_scratch(name):
+    """Whole prompts: every context position is new (T_b = L_b), ragged lengths
+    spanning several query tiles and a partial last tile."""
+    lengths = [1, 9, 64, 130, 257]
+    w, out, ref, (kc, vc), (kc_ref, vc_ref) = _run(name, lengths, lengths)
+    assert torch.equal(bits(kc), bits(kc_ref)) and torch.equal(bits(vc), bits(vc_ref))
+    assert_close(out, ref, torch.bfloat16, f"prefill {name}")
+    assert pa.device_errors() == 0
+
+
+@pytest.mark.parametrize("name", ["tinyllama_1b", "llama3_8b"])
+def test_chunked_prefill_over_an_existing_context(name):
+    """A chunk of new tokens on top of cached positions, and sequences with no
+    new token in this call."""
+    lengths = [300, 45, 1000, 17, 64]
+    q_lens = [100, 45, 7, 0, 33]
+    w, out, ref, (kc, vc), (kc_ref, vc_ref) = _run(name, lengths, q_lens)
+    assert torch.equal(bits(kc), bits(kc_ref)) and torch.equal(bits(vc), bits(vc_ref))
+    assert_close(out, ref, torch.bfloat16, f"chunked prefill {name}")
+
+
+@pytest.mark.parametrize("window", [1, 16, 100])
+def test_prefill_window_and_softcap(window):
+    lengths = [200, 77]
+    w, out, ref, _, _ = _run("gemma2_2b", lengths, [150, 77], window=window)
+    assert_close(out, ref, torch.bfloat16, f"prefill window={window} softcap 50")
+
+
+def test_prefill_attend_only():
+    """k_new = v_new = NULL: the rows are already in the cache."""
+    lengths = [120, 33]
+    w, out, ref, _, _ = _run("llama3_8b", lengths, [40, 33], append=False)
+    assert_close(out, ref, torch.bfloat16, "prefill without append")
+
+
+def test_prefill_bad_offsets_are_reported_not_written():
+    w = wl.WORKLOADS["tinyllama_1b"]
+    b = wl.make_batch(w, lengths=[40, 40], prefilled=True, device="cuda")
+    x = wl.make_prefill_inputs(b, [10, 10])
+    cu = torch.tensor([0, 10, 30], dtype=torch.int32, device="cuda")  # past total_q = 20
+    out = torch.full_like(x["q"], 7.0)
+    pa.prefill(x["q"], None, None, None, cu, b.k_cache, b.v_cache, b.block_tables, b.context_lens, w.scale,
+               max_q_len=20, out=out)
+    torch.cuda.synchronize()
+    assert pa.device_errors() & pa.DEVERR_CONTEXT
+    assert torch.all(out[10:] == 7.0)  # the malformed sequence's rows are untouched
