@@ -39,6 +39,7 @@ from paged_kv_cache_473_b200 import workloads as wl  # noqa: E402
 METRIC = "paged decode tokens/s and achieved HBM GB/s (% of B200 peak) per batch shape"
 HEADLINE = "tinyllama_1b"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 # Decode launches are bracketed by timing events on every EVENT_EVERY-th step
 # only: an event node between graph kernels stops the graph from overlapping the
 # next launch, which on the 65 MB TinyLlama step alone costs ~8 us per step.
@@ -193,6 +194,16 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def tensor_peak() -> float:
+    """Dense bf16 tensor peak (TFLOP/s) for a kernel timed on its own: the
+    measured burst figure, else the pool's earlier measurement."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except Exception:  # noqa: BLE001
+        return FALLBACK_BF16_TFLOPS
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_473_b200", "csrc")
@@ -337,6 +348,38 @@ class MultiRunner(Runner):
         self.pa.decode_multi(self.q, kc, vc, b.block_tables, b.context_lens, w.scale, w.softcap, w.window,
                              split=True, max_context_len=self.max_ctx, partition_tokens=0, out=self.out,
                              workspace=self.ws)
+        return self.pa.last_launch_count()
+
+    def step(self, r, x=None, ev=None):
+        if ev is not None:
+            ev[0].record()
+        n = self.decode(r, None)
+        if ev is not None:
+            ev[1].record()
+        self.launches_per_step = n
+
+
+class PrefillRunner(Runner):
+    """Paged prefill of whole prompts (pa_prefill: append + causal attention)
+    with a workload's heads: ``n_prompts`` prompts of ``prompt_len`` tokens.
+    A step is only that call."""
+
+    def __init__(self, w: wl.Workload, rank: int, n_prompts: int, prompt_len: int):
+        w = w.replace(prefix_share=0.0, batch=n_prompts, lengths=("fixed", (prompt_len,) * n_prompts))
+        super().__init__(w, rank, "auto", False, -1, fused=True)
+        b = self.batch
+        self.x = wl.make_prefill_inputs(b, [prompt_len] * n_prompts)
+        self.T = prompt_len
+        self.out = torch.empty_like(self.x["q"])
+        # causal attention flops: QK^T and PV, 2 flops per multiply-add, T(T+1)/2 pairs per prompt and head
+        self.flops = n_prompts * 4 * w.num_q_heads * w.head_dim * prompt_len * (prompt_len + 1) // 2
+        torch.cuda.synchronize()
+
+    def decode(self, r, x):
+        w, b, x = self.w, self.batch, self.x
+        kc, vc = self.pools[r]
+        self.pa.prefill(x["q"], x["k_new"], x["v_new"], x["slot_mapping"], x["cu_q_lens"], kc, vc, b.block_tables,
+                        b.context_lens, w.scale, w.softcap, w.window, max_q_len=x["max_q_len"], out=self.out)
         return self.pa.last_launch_count()
 
     def step(self, r, x=None, ev=None):
@@ -546,6 +589,31 @@ def multi_summary(w: wl.Workload, q_len: int, rank: int, K: int, W: int, world: 
 
 
 MULTI_SHAPES = (("tinyllama_1b", 4), ("llama3_8b", 4), ("gemma2_2b", 8))
+PREFILL_SHAPES = (("llama3_8b", 16, 1024), ("tinyllama_1b", 16, 1024))
+
+
+def prefill_summary(w: wl.Workload, n_prompts: int, prompt_len: int, rank: int, K: int, W: int, world: int,
+                    dev_idx: int):
+    """Paged prefill of whole prompts: prompt tokens/s and causal-attention
+    TFLOP/s against the measured dense bf16 peak (tensor-bound)."""
+    runner = PrefillRunner(w, rank, n_prompts, prompt_len)
+    total_ms, _, _ = run_timed(runner, K, W, world, dev_idx)
+    ms = total_ms / K
+    tflops = runner.flops / (ms * 1e-3) / 1e12
+    peak = tensor_peak()
+    res = {
+        "prompts": n_prompts,
+        "prompt_len": prompt_len,
+        "tokens_per_s": round(n_prompts * prompt_len / (ms * 1e-3), 1),
+        "ms_per_step": round(ms, 5),
+        "tflops": round(tflops, 1),
+        "tensor_peak_tflops": peak,
+        "tensor_frac": round(tflops / peak, 4),
+        "launches_per_step": runner.launches_per_step,
+    }
+    del runner
+    torch.cuda.empty_cache()
+    return res
 
 
 def main_ours(args, world, rank, local):
@@ -621,6 +689,9 @@ def main_ours(args, world, rank, local):
         for n, T in MULTI_SHAPES:
             if args.shapes == "auto" or n in names or n == w.name:
                 extra[f"{n}@multi{T}"] = multi_summary(wl.WORKLOADS[n], T, rank, 50, 5, world, local, peak)
+        for n, P_, T in PREFILL_SHAPES:
+            if args.shapes == "auto" or n in names or n == w.name:
+                extra[f"{n}@prefill{P_}x{T}"] = prefill_summary(wl.WORKLOADS[n], P_, T, rank, 20, 3, world, local)
         line["per_shape"] = extra
         runner = None
     if world == 1 and rank == 0 and not args.no_cpu:
