@@ -6,6 +6,8 @@ package is its Python binding plus seeded synthetic batch generators
 """
 
 from ._binding import (  # noqa: F401
+    BlockManager,
+    copy_blocks,
     DEVERR_BLOCK,
     DEVERR_CONTEXT,
     DEVERR_SLOT,
@@ -29,6 +31,8 @@ from ._binding import (  # noqa: F401
 )
 
 __all__ = [
+    "BlockManager",
+    "copy_blocks",
     "write_kv",
     "decode",
     "decode_multi",

@@ -69,6 +69,33 @@ def _load_library() -> ctypes.CDLL:
                                _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_f32, _c_f32, _c_i32, _c_vp, _c_i32,
                                _c_vp]
     lib.pa_prefill.restype = _c_i32
+    lib.pa_copy_blocks.argtypes = [_c_vp, _c_vp, _c_vp, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_vp]
+    lib.pa_copy_blocks.restype = _c_i32
+    # host block manager (include/block_manager.h)
+    lib.pa_bm_create.argtypes = [_c_i32, _c_i32]
+    lib.pa_bm_create.restype = _c_vp
+    lib.pa_bm_destroy.argtypes = [_c_vp]
+    lib.pa_bm_destroy.restype = None
+    lib.pa_bm_num_free.argtypes = [_c_vp]
+    lib.pa_bm_num_free.restype = _c_i32
+    lib.pa_bm_blocks_needed.argtypes = [_c_vp, _c_vp, _c_i32]
+    lib.pa_bm_blocks_needed.restype = _c_i32
+    lib.pa_bm_add_sequence.argtypes = [_c_vp, _c_i64, _c_vp, _c_i32, _c_vp]
+    lib.pa_bm_add_sequence.restype = _c_i32
+    lib.pa_bm_append_slots.argtypes = [_c_vp, _c_vp, _c_vp, _c_i32, _c_vp, _c_vp, _c_vp]
+    lib.pa_bm_append_slots.restype = _c_i32
+    lib.pa_bm_fork.argtypes = [_c_vp, _c_i64, _c_i64]
+    lib.pa_bm_fork.restype = _c_i32
+    lib.pa_bm_free_sequence.argtypes = [_c_vp, _c_i64]
+    lib.pa_bm_free_sequence.restype = _c_i32
+    lib.pa_bm_length.argtypes = [_c_vp, _c_i64]
+    lib.pa_bm_length.restype = _c_i32
+    lib.pa_bm_block_tables.argtypes = [_c_vp, _c_vp, _c_i32, _c_i32, _c_vp, _c_vp]
+    lib.pa_bm_block_tables.restype = _c_i32
+    lib.pa_bm_slots.argtypes = [_c_vp, _c_i64, _c_i32, _c_i32, _c_vp]
+    lib.pa_bm_slots.restype = _c_i32
+    lib.pa_bm_ref_count.argtypes = [_c_vp, _c_i32]
+    lib.pa_bm_ref_count.restype = _c_i32
     lib.pa_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint32), _c_i32]
     lib.pa_device_errors.restype = _c_i32
     lib.pa_error_string.argtypes = [_c_i32]
@@ -263,6 +290,104 @@ def prefill(q: torch.Tensor, k_new: Optional[torch.Tensor], v_new: Optional[torc
                         float(softcap), int(window), _ptr(out), _dtype_code(q), _stream(stream))
     _check(st, "pa_prefill")
     return out
+
+
+def copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, pairs: torch.Tensor, stream=None) -> None:
+    """Copy whole blocks inside both caches: ``pairs`` is a device int32
+    ``[n, 2]`` tensor of (src, dst) block ids (copy-on-write)."""
+    nb, hkv, bs, d = k_cache.shape
+    pairs = pairs.to(torch.int32).contiguous()
+    st = lib.pa_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(pairs), pairs.shape[0], nb, bs, hkv, d,
+                            _dtype_code(k_cache), _stream(stream))
+    _check(st, "pa_copy_blocks")
+
+
+def _i64_array(xs):
+    xs = [int(x) for x in xs]
+    return (ctypes.c_int64 * max(1, len(xs)))(*xs), len(xs)
+
+
+class BlockManager:
+    """The library's host block manager (include/block_manager.h): on-demand
+    allocation, reference counts, fork, copy-on-write and a prefix cache of
+    full blocks.  Host memory only; the copy-on-write pairs it returns are
+    carried out on the GPU with :func:`copy_blocks`."""
+
+    def __init__(self, num_blocks: int, block_size: int):
+        self._h = lib.pa_bm_create(int(num_blocks), int(block_size))
+        if not self._h:
+            raise PagedAttnError(PA_ERR_INVALID, "pa_bm_create")
+        self.num_blocks, self.block_size = int(num_blocks), int(block_size)
+
+    def close(self) -> None:
+        if self._h:
+            lib.pa_bm_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:  # noqa: BLE001
+            pass
+
+    @property
+    def num_free(self) -> int:
+        return lib.pa_bm_num_free(self._h)
+
+    def blocks_needed(self, num_tokens: int, token_ids=None) -> int:
+        arr = _i64_array(token_ids)[0] if token_ids is not None else None
+        return lib.pa_bm_blocks_needed(self._h, arr, int(num_tokens))
+
+    def add_sequence(self, seq_id: int, num_tokens: int, token_ids=None) -> int:
+        """Register a prompt; returns how many leading positions came from the prefix cache."""
+        arr = None
+        if token_ids is not None:
+            arr, n = _i64_array(token_ids)
+            if n != num_tokens:
+                raise ValueError("token_ids must hold num_tokens ids")
+        cached = ctypes.c_int32(0)
+        _check(lib.pa_bm_add_sequence(self._h, int(seq_id), arr, int(num_tokens), ctypes.byref(cached)),
+               "pa_bm_add_sequence")
+        return cached.value
+
+    def append_slots(self, seq_ids, token_ids=None):
+        """One decode step: returns (slots int64 [n], copy-on-write pairs int32 [k, 2])."""
+        ids, n = _i64_array(seq_ids)
+        toks = _i64_array(token_ids)[0] if token_ids is not None else None
+        slots = (ctypes.c_int64 * max(1, n))()
+        cow = (ctypes.c_int32 * max(2, 2 * n))()
+        ncow = ctypes.c_int32(0)
+        _check(lib.pa_bm_append_slots(self._h, ids, toks, n, slots, cow, ctypes.byref(ncow)), "pa_bm_append_slots")
+        k = ncow.value
+        return (torch.tensor(list(slots)[:n], dtype=torch.int64),
+                torch.tensor(list(cow)[: 2 * k], dtype=torch.int32).reshape(k, 2))
+
+    def fork(self, parent_id: int, child_id: int) -> None:
+        _check(lib.pa_bm_fork(self._h, int(parent_id), int(child_id)), "pa_bm_fork")
+
+    def free(self, seq_id: int) -> None:
+        _check(lib.pa_bm_free_sequence(self._h, int(seq_id)), "pa_bm_free_sequence")
+
+    def length(self, seq_id: int) -> int:
+        return lib.pa_bm_length(self._h, int(seq_id))
+
+    def block_tables(self, seq_ids, max_blocks: int):
+        """(tables int32 [n, max_blocks], -1 padded; context_lens int32 [n]) on the host."""
+        ids, n = _i64_array(seq_ids)
+        tables = torch.empty((n, int(max_blocks)), dtype=torch.int32)
+        lens = torch.empty((n,), dtype=torch.int32)
+        _check(lib.pa_bm_block_tables(self._h, ids, n, int(max_blocks), tables.data_ptr(), lens.data_ptr()),
+               "pa_bm_block_tables")
+        return tables, lens
+
+    def slots(self, seq_id: int, start: int, count: int) -> torch.Tensor:
+        out = torch.empty((int(count),), dtype=torch.int64)
+        _check(lib.pa_bm_slots(self._h, int(seq_id), int(start), int(count), out.data_ptr() if count else None),
+               "pa_bm_slots")
+        return out
+
+    def ref_count(self, block: int) -> int:
+        return lib.pa_bm_ref_count(self._h, int(block))
 
 
 NOALLOC_SCRATCH_BYTES = 16 << 20

@@ -13,6 +13,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libpagedattn.so")
 MAIN = os.path.join(CSRC, "pagedattn.cu")
+# Translation units: the kernels and their C ABI, and the host block manager.
+UNITS = [MAIN, os.path.join(CSRC, "block_manager.cpp")]
 
 NVCC_FLAGS = [
     "-gencode",
@@ -34,9 +36,8 @@ def _nvcc() -> str:
 
 
 def sources() -> list:
-    return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))) + [
-        os.path.join(ROOT, "include", "pagedattn.h")
-    ]
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh")) +
+                  glob.glob(os.path.join(CSRC, "*.cpp")) + glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 
 def up_to_date() -> bool:
@@ -50,7 +51,7 @@ def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
     if not force and up_to_date():
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [_nvcc(), *NVCC_FLAGS, *(extra_flags or []), "-I", os.path.join(ROOT, "include"), "-o", tmp, MAIN]
+    cmd = [_nvcc(), *NVCC_FLAGS, *(extra_flags or []), "-I", os.path.join(ROOT, "include"), "-o", tmp, *UNITS]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.run(cmd, check=True)

@@ -131,4 +131,25 @@ __global__ void __launch_bounds__(256)
   v_cache[dst] = v[src];
 }
 
+// ---- block copies (copy-on-write) ----------------------------------------------------
+//
+// blockIdx.x: pair i = (src, dst) of pairs[]; threads stride over the block's
+// 16-byte chunks (chunks_per_block of them in each cache).  Ids outside the
+// pool raise PA_DEVERR_BLOCK and the pair is skipped.
+__global__ void __launch_bounds__(256)
+    copy_blocks_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache, const int32_t* __restrict__ pairs,
+                       int num_blocks, int64_t chunks_per_block) {
+  const int src = pairs[2 * blockIdx.x], dst = pairs[2 * blockIdx.x + 1];
+  if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+    if (threadIdx.x == 0 && blockIdx.y == 0) raise_error(PA_DEVERR_BLOCK);
+    return;
+  }
+  const int64_t s0 = (int64_t)src * chunks_per_block, d0 = (int64_t)dst * chunks_per_block;
+  for (int64_t c = (int64_t)blockIdx.y * blockDim.x + threadIdx.x; c < chunks_per_block;
+       c += (int64_t)gridDim.y * blockDim.x) {
+    k_cache[d0 + c] = k_cache[s0 + c];
+    v_cache[d0 + c] = v_cache[s0 + c];
+  }
+}
+
 }  // namespace pa

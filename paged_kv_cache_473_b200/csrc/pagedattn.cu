@@ -13,6 +13,7 @@
 #include <utility>
 
 #include "../../include/pagedattn.h"
+#include "../../include/block_manager.h"
 #include "combine_and_append.cuh"
 #include "decode_common.cuh"
 #include "decode_mma.cuh"
@@ -799,6 +800,26 @@ pa_status_t pa_decode_splitk_noalloc(const void* q, const void* k_cache, const v
   return pa_decode_splitk(q, k_cache, v_cache, block_tables, context_lens, batch, num_q_heads, num_kv_heads,
                           head_dim, block_size, max_blocks_per_seq, num_blocks, scale, softcap, window, out, dtype,
                           partition_tokens, max_context_len, ws, PA_NOALLOC_SCRATCH_BYTES, kernel, stream);
+}
+
+pa_status_t pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, int32_t n, int32_t num_blocks,
+                           int32_t block_size, int32_t num_kv_heads, int32_t head_dim, pa_dtype_t dtype,
+                           pa_stream_t stream) {
+  t_last_launches = 0;
+  if (n < 0 || num_blocks <= 0 || block_size <= 0 || num_kv_heads <= 0 || head_dim <= 0) return PA_ERR_INVALID;
+  if (dtype != PA_F32 && dtype != PA_BF16) return PA_ERR_INVALID;
+  if (n == 0) return PA_OK;
+  if (!k_cache || !v_cache || !pairs || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(pairs, 4))
+    return PA_ERR_INVALID;
+  const int64_t bytes = (int64_t)num_kv_heads * block_size * head_dim * (dtype == PA_F32 ? 4 : 2);
+  if (bytes % 16 != 0) return PA_ERR_UNSUPPORTED;
+  const int64_t chunks = bytes / 16;
+  const unsigned ys = (unsigned)std::min<int64_t>((chunks + 255) / 256, 64);
+  pa::copy_blocks_kernel<<<dim3((unsigned)n, ys), 256, 0, stream>>>(
+      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), pairs, num_blocks, chunks);
+  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  t_last_launches = 1;
+  return PA_OK;
 }
 
 pa_status_t pa_device_errors(uint32_t* bits, int32_t clear) {

@@ -20,7 +20,8 @@ MIS = 0x10004
 
 
 def declared_functions():
-    src = open(HEADER).read()
+    import glob
+    src = "".join(open(h).read() for h in sorted(glob.glob(os.path.join(os.path.dirname(HEADER), "*.h"))))
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", src)))
 
@@ -30,7 +31,7 @@ def test_header_declares_the_entry_points():
     for n in ["pa_write_kv", "pa_decode", "pa_decode_splitk", "pa_decode_splitk_workspace_size",
               "pa_decode_splitk_partition", "pa_device_errors", "pa_error_string", "pa_last_launch_count",
               "pa_decode_step", "pa_decode_splitk_noalloc", "pa_decode_multi", "pa_decode_multi_workspace_size",
-              "pa_prefill"]:
+              "pa_prefill", "pa_copy_blocks", "pa_bm_create", "pa_bm_append_slots", "pa_bm_block_tables"]:
         assert n in names
 
 
@@ -209,4 +210,23 @@ def _prefill(**kw):
 )
 def test_prefill_host_checks(kw, status):
     assert _prefill(**kw) == status
+    assert pa.last_launch_count() == 0
+
+
+@pytest.mark.parametrize(
+    "kw,status",
+    [
+        (dict(n=-1), bnd.PA_ERR_INVALID),
+        (dict(k=None), bnd.PA_ERR_INVALID),
+        (dict(pairs=A + 2), bnd.PA_ERR_INVALID),
+        (dict(dt=7), bnd.PA_ERR_INVALID),
+        (dict(d=3, dt=bnd.PA_BF16, hkv=1, bs=1), bnd.PA_ERR_UNSUPPORTED),  # 6-byte blocks
+        (dict(n=0), bnd.PA_OK),
+    ],
+)
+def test_copy_blocks_host_checks(kw, status):
+    a = dict(k=A, v=A, pairs=A, n=2, nb=8, bs=16, hkv=2, d=128, dt=bnd.PA_BF16)
+    a.update(kw)
+    assert bnd.lib.pa_copy_blocks(a["k"], a["v"], a["pairs"], a["n"], a["nb"], a["bs"], a["hkv"], a["d"], a["dt"],
+                                  None) == status
     assert pa.last_launch_count() == 0
