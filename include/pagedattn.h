@@ -260,6 +260,40 @@ pa_status_t pa_prefill(const void* q, const void* k_new, const void* v_new, cons
                        pa_stream_t stream);
 
 /*
+ * pa_decode_cascade -- split-K decode that reads a shared prefix once.
+ *   Sequences 0 .. n_sharers-1 of the batch share their first prefix_len
+ *   positions: the first prefix_len / block_size entries of their block
+ *   tables are the same physical blocks, holding valid rows (prefix caching
+ *   shares full blocks).  The result equals pa_decode_splitk's, within the
+ *   same tolerance; only the order of the additions differs.
+ *   Three launches: (1) the prefix pass loads each prefix block once per kv
+ *   head and attends it for every sharer (64 / G sharers x G query heads per
+ *   CTA, on the multi-query kernel), writing split-K partials; (2) the
+ *   split-K decode attends every sequence's own range (sharers from position
+ *   prefix_len on); (3) the log-sum-exp combine merges both.  A sharer whose
+ *   table differs from sequence 0's inside the prefix raises PA_DEVERR_BLOCK
+ *   (its prefix rows are then sequence 0's).
+ *   prefix_len: a multiple of 64 and of block_size, <= max_context_len and
+ *   <= max_blocks_per_seq * block_size (else PA_ERR_INVALID).
+ *   partition_tokens: 0 lets the library choose (halved until it divides
+ *   prefix_len), else a multiple of 64 that divides prefix_len.  The workspace
+ *   is pa_decode_cascade_workspace_size() bytes under pa_decode_splitk's
+ *   contract.  n_sharers = 0 or prefix_len = 0 runs pa_decode_splitk.  bf16.
+ *   Passages: nano-vllm (ovshake) README, "Features" ("Prefix Caching: share
+ *   KV cache blocks for common prefixes") and "PagedAttention" (sequences
+ *   reach shared blocks through their tables).
+ */
+pa_status_t pa_decode_cascade(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                              const int32_t* context_lens, int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                              int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq, int32_t num_blocks,
+                              float scale, float softcap, int32_t window, void* out, pa_dtype_t dtype,
+                              int32_t n_sharers, int32_t prefix_len, int32_t partition_tokens,
+                              int32_t max_context_len, void* workspace, size_t workspace_bytes, pa_stream_t stream);
+size_t pa_decode_cascade_workspace_size(int32_t batch, int32_t num_q_heads, int32_t head_dim,
+                                        int32_t max_context_len, int32_t prefix_len, int32_t partition_tokens,
+                                        int32_t num_kv_heads);
+
+/*
  * pa_decode_splitk_noalloc -- pa_decode_splitk for callers that cannot allocate
  * device memory.
  *   The pages describe no such call; it exists for callers that must not call

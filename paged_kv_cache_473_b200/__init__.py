@@ -15,6 +15,8 @@ from ._binding import (  # noqa: F401
     KERNELS,
     PagedAttnError,
     decode,
+    decode_cascade,
+    decode_cascade_workspace_size,
     decode_multi,
     decode_multi_workspace_size,
     decode_splitk,
@@ -35,6 +37,8 @@ __all__ = [
     "copy_blocks",
     "write_kv",
     "decode",
+    "decode_cascade",
+    "decode_cascade_workspace_size",
     "decode_multi",
     "decode_multi_workspace_size",
     "decode_splitk",

@@ -96,6 +96,10 @@ def _load_library() -> ctypes.CDLL:
     lib.pa_bm_slots.restype = _c_i32
     lib.pa_bm_ref_count.argtypes = [_c_vp, _c_i32]
     lib.pa_bm_ref_count.restype = _c_i32
+    lib.pa_decode_cascade.argtypes = dec + [_c_i32, _c_i32, _c_i32, _c_i32, _c_vp, _c_sz, _c_vp]
+    lib.pa_decode_cascade.restype = _c_i32
+    lib.pa_decode_cascade_workspace_size.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32]
+    lib.pa_decode_cascade_workspace_size.restype = _c_sz
     lib.pa_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint32), _c_i32]
     lib.pa_device_errors.restype = _c_i32
     lib.pa_error_string.argtypes = [_c_i32]
@@ -200,6 +204,33 @@ def decode_splitk(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                               _ptr(out), _dtype_code(q), int(partition_tokens), int(max_context_len),
                               _ptr(workspace), wbytes, KERNELS[kernel], _stream(stream))
     _check(st, "pa_decode_splitk")
+    return out
+
+
+def decode_cascade_workspace_size(batch: int, num_q_heads: int, head_dim: int, max_context_len: int,
+                                  prefix_len: int, partition_tokens: int = 0, num_kv_heads: int = 1) -> int:
+    return lib.pa_decode_cascade_workspace_size(batch, num_q_heads, head_dim, max_context_len, prefix_len,
+                                                partition_tokens, num_kv_heads)
+
+
+def decode_cascade(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_tables: torch.Tensor,
+                   context_lens: torch.Tensor, scale: float, softcap: float = 0.0, window: int = 0, *,
+                   n_sharers: int, prefix_len: int, max_context_len: int, partition_tokens: int = 0,
+                   out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    """Split-K decode where sequences ``0 .. n_sharers-1`` share their first
+    ``prefix_len`` positions (same blocks): the prefix is read once per kv head
+    for all of them, then merged with each sequence's own range."""
+    B, hq, d, nb, hkv, bs, out = _decode_common(q, k_cache, block_tables, out)
+    need = decode_cascade_workspace_size(B, hq, d, max_context_len, prefix_len, partition_tokens, hkv)
+    if workspace is None:
+        workspace = torch.zeros(max(need, 16), dtype=torch.uint8, device=q.device)
+    wbytes = workspace.numel() * workspace.element_size()
+    st = lib.pa_decode_cascade(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens), B, hq,
+                               hkv, d, bs, block_tables.shape[1], nb, float(scale), float(softcap), int(window),
+                               _ptr(out), _dtype_code(q), int(n_sharers), int(prefix_len), int(partition_tokens),
+                               int(max_context_len), _ptr(workspace), wbytes, _stream(stream))
+    _check(st, "pa_decode_cascade")
     return out
 
 

@@ -42,6 +42,13 @@ struct DecodeParams {
   int q_tile;           // prefill: query tokens per CTA
   int max_q_len;        // prefill: bound on cu_q[b+1] - cu_q[b] (the grid covers it)
   int total_q;          // prefill: rows of q and out (bound on cu_q[B])
+  // Cascade: sequences 0 .. n_sharers-1 share positions [0, prefix_len) (a
+  // multiple of the partition).  The prefix pass (cascade_prefix = 1) attends
+  // them once for all sharers; the other passes start those sequences at
+  // prefix_len.
+  int cascade_prefix;
+  int n_sharers;
+  int prefix_len;
   int block_size, log2_bs, max_blocks, num_blocks;
   int window;
   int partition;    // tokens per partition (a multiple of 64); 1 << 30 without split
@@ -79,6 +86,7 @@ __device__ __forceinline__ CtaRange cta_range(const DecodeParams& p, int b, int 
   r.s0 = window_start(r.L, p.window);
   const int P = p.partition;
   r.lo = max(r.s0, part * P);
+  if (b < p.n_sharers) r.lo = max(r.lo, p.prefix_len);  // the cascade's prefix pass attended the shared prefix
   r.hi = min(r.L, part * P + P);
   r.n_parts = (r.L > r.s0) ? (r.L + P - 1) / P - r.s0 / P : 0;
   r.final_write = (r.n_parts == 1);

@@ -41,21 +41,14 @@ struct MultiCfg {
   static constexpr int kSmemBytes = kRingBytes + 2 * ST * 8 + 1024;
 };
 
-// Token range of query column c (token j = j0 + c / G of the T) inside the
-// CTA's partition [pl, ph): [max(s0_j, pl), min(p_j + 1, ph)).  Padding
-// columns (c >= ntok*G) take the CTA's union range so that their (discarded)
-// softmax stays finite.
-__device__ __forceinline__ void column_range(int c, int G, int T, int j0, int ntok, int L, int window, int pl, int ph,
-                                             int ulo, int uhi, int& lo, int& hi) {
-  if (c >= ntok * G) {
-    lo = ulo;
-    hi = uhi;
-    return;
-  }
-  const int end = L - T + j0 + c / G + 1;  // p_j + 1
-  lo = max(window_start(max(end, 0), window), pl);
-  hi = min(end, ph);
-}
+// One query column of the CTA: its output (or workspace) row, its token range
+// inside the CTA's partition, and whether it writes the normalised row itself.
+struct QueryCol {
+  size_t row;
+  int lo, hi;
+  bool fin;
+  bool real;  // false: a padding column (no query, no output)
+};
 
 template <int D, int ST, bool SPLIT>
 __global__ void __launch_bounds__(kMaxMultiColumns / 8 * 32)
@@ -70,59 +63,128 @@ __global__ void __launch_bounds__(kMaxMultiColumns / 8 * 32)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int NW = blockDim.x >> 5;
-  const int g = blockIdx.y, b = blockIdx.z;
+  const int g = blockIdx.y;
   const int G = p.group, P = p.partition;
+  const bool cascade = p.cascade_prefix != 0;
   const bool varlen = p.cu_q != nullptr;
 
-  // This CTA's query tokens: j0 .. j0 + ntok - 1 of the sequence's T, at q/out
-  // rows row0 .. row0 + ntok - 1 (times Hq).
-  int part, T, j0, ntok;
-  size_t row0;
-  if (varlen) {
-    const int a = p.cu_q[b], e = p.cu_q[b + 1];
-    if (a < 0 || e < a || e > p.total_q || e - a > p.max_q_len) {  // malformed offsets: report, write nothing
-      if (blockIdx.x == 0 && g == 0 && threadIdx.x == 0) raise_error(PA_DEVERR_CONTEXT);
+  // ---- the CTA's K/V range and its query columns ---------------------------------------
+  // kv_seq: the sequence whose block table addresses the K/V; [pl, ph): the
+  // partition; [ulo, uhi): the positions any column may attend in it (all of
+  // them valid cache rows); ncols: real query columns.
+  int part = SPLIT ? (int)blockIdx.x : 0;
+  int kv_seq, ncols, ulo, uhi;
+  int T = 0, j0 = 0, L = 0, n_parts = 0, sbase = 0;
+  size_t row0 = 0;
+  if (cascade) {
+    // Columns: sharer sequences sbase .. x G heads; the K/V are the shared
+    // prefix, addressed through the first sharer's table.
+    sbase = blockIdx.z * p.q_tile;
+    ncols = min(p.q_tile, p.n_sharers - sbase) * G;
+    kv_seq = 0;
+    if (ncols <= 0) return;
+    ulo = part * P;
+    uhi = min(ulo + P, p.prefix_len);
+  } else {
+    kv_seq = blockIdx.z;
+    if (varlen) {
+      const int a = p.cu_q[kv_seq], e = p.cu_q[kv_seq + 1];
+      if (a < 0 || e < a || e > p.total_q || e - a > p.max_q_len) {  // malformed offsets: report, write nothing
+        if (blockIdx.x == 0 && g == 0 && threadIdx.x == 0) raise_error(PA_DEVERR_CONTEXT);
+        return;
+      }
+      T = e - a;
+      part = 0;
+      j0 = blockIdx.x * p.q_tile;
+      row0 = (size_t)a + j0;
+    } else {
+      T = p.q_len;
+      row0 = (size_t)kv_seq * T;
+    }
+    const int ntok = min(varlen ? p.q_tile : T, T - j0);
+    if (ntok <= 0) return;
+    ncols = ntok * G;
+    L = clamp_context(p, kv_seq, threadIdx.x == 0 && part == 0 && j0 == 0);
+    // The union of the tile's ranges is [s0 of its first token, p of its last + 1).
+    const int uend = min(L, L - T + j0 + ntok);
+    const int ulo_seq = window_start(max(L - T + j0 + 1, 0), p.window);
+    n_parts = (uend > ulo_seq) ? (uend + P - 1) / P - ulo_seq / P : 0;
+    ulo = max(ulo_seq, part * P);
+    uhi = min(uend, part * P + P);
+    if (ulo >= uhi) {  // nothing of this sequence falls in this partition
+      if (n_parts == 0 && part == 0) {  // no position for any token: zero rows for every query column
+        for (int idx = threadIdx.x; idx < ncols * D; idx += blockDim.x) {
+          const int c = idx / D;
+          static_cast<__nv_bfloat16*>(p.out)[((row0 + c / G) * p.hq + (size_t)g * G + c % G) * D + idx % D] =
+              __float2bfloat16_rn(0.f);
+        }
+      }
       return;
     }
-    T = e - a;
-    part = 0;
-    j0 = blockIdx.x * p.q_tile;
-    ntok = min(p.q_tile, T - j0);
-    row0 = (size_t)a + j0;
-    if (ntok <= 0) return;
-  } else {
-    part = SPLIT ? (int)blockIdx.x : 0;
-    T = p.q_len;
-    j0 = 0;
-    ntok = T;
-    row0 = (size_t)b * T;
   }
-
-  const int L = clamp_context(p, b, threadIdx.x == 0 && part == 0 && j0 == 0);
-  // The union of the tile's ranges is [s0 of its first token, p of its last + 1).
-  const int uend = min(L, L - T + j0 + ntok);
-  const int ulo_seq = window_start(max(L - T + j0 + 1, 0), p.window);
-  const int n_parts = (uend > ulo_seq) ? (uend + P - 1) / P - ulo_seq / P : 0;
-  const bool final_write = !SPLIT || n_parts == 1;
   const int pl = part * P, ph = pl + P;
-  const int ulo = max(ulo_seq, pl), uhi = min(uend, ph);
+  const bool cta_final = !SPLIT || n_parts == 1;
 
-  // This lane's two accumulator columns and their ranges.
+  // Column c < ncols.  Token columns (multi-query rows, prefill tiles): token
+  // j0 + c / G at position p = L - T + j0 + c / G attends [s0(p + 1), p + 1).
+  // Sharer columns (cascade): sequence b = sbase + c / G attends its
+  // positions below the prefix length; it writes its row itself only when
+  // its whole range is this one partition (or it has no position at all).
+  auto column = [&](int c) -> QueryCol {
+    QueryCol q;
+    const int h = c % G;
+    q.real = true;
+    if (cascade) {
+      const int b = sbase + c / G;
+      const int Lb = clamp_context(p, b, false);
+      const int s0 = window_start(Lb, p.window);
+      const int nb = Lb > s0 ? (Lb + P - 1) / P - s0 / P : 0;
+      q.row = (size_t)b * p.hq + (size_t)g * G + h;
+      q.lo = max(s0, pl);
+      q.hi = min(min(Lb, p.prefix_len), ph);
+      q.fin = (nb == 1 && part == s0 / P) || (nb == 0 && part == 0);
+    } else {
+      const int end = L - T + j0 + c / G + 1;  // p + 1
+      q.row = (row0 + c / G) * p.hq + (size_t)g * G + h;
+      q.lo = max(window_start(max(end, 0), p.window), pl);
+      q.hi = min(end, ph);
+      q.fin = cta_final;
+    }
+    return q;
+  };
+
+  // This lane's two accumulator columns and their ranges (padding columns take
+  // the union, so that their discarded softmax stays finite).
   const int n0 = 2 * (lane & 3);
   const int c0 = warp * 8 + n0;
+  QueryCol qc[2];
   ColRange cr;
-  column_range(c0, G, T, j0, ntok, L, p.window, pl, ph, ulo, uhi, cr.lo0, cr.hi0);
-  column_range(c0 + 1, G, T, j0, ntok, L, p.window, pl, ph, ulo, uhi, cr.lo1, cr.hi1);
-
-  // Output row (or workspace row) of column c: ((row0 + c / G)*Hq + g*G + h).
-  auto row_of = [&](int c) { return (row0 + c / G) * p.hq + (size_t)g * G + c % G; };
-
-  if (ulo >= uhi) {  // nothing of this sequence falls in this partition
-    if (n_parts == 0 && part == 0) {  // no position for any token: zero rows for every query column
-      for (int idx = threadIdx.x; idx < ntok * G * D; idx += blockDim.x)
-        static_cast<__nv_bfloat16*>(p.out)[row_of(idx / D) * D + idx % D] = __float2bfloat16_rn(0.f);
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    if (c0 + e < ncols) {
+      qc[e] = column(c0 + e);
+    } else {
+      qc[e].row = 0;
+      qc[e].lo = ulo;
+      qc[e].hi = uhi;
+      qc[e].fin = false;
+      qc[e].real = false;
     }
-    return;
+  }
+  cr.lo0 = qc[0].lo;
+  cr.hi0 = qc[0].hi;
+  cr.lo1 = qc[1].lo;
+  cr.hi1 = qc[1].hi;
+  if (cascade && lane < 4) {
+    // Every sharer must map the prefix to the same blocks as the first one.
+    const int32_t* ref = p.block_tables + (size_t)kv_seq * p.max_blocks;
+    for (int e = 0; e < 2; ++e) {
+      if (c0 + e >= ncols || (c0 + e) % G) continue;
+      const int b = sbase + (c0 + e) / G;
+      const int32_t* tb = p.block_tables + (size_t)b * p.max_blocks;
+      for (int t = ulo; t < uhi; t += p.block_size)
+        if (tb[t >> p.log2_bs] != ref[t >> p.log2_bs]) raise_error(PA_DEVERR_BLOCK);
+    }
   }
 
   const uint32_t ring = smem_addr(smem);
@@ -142,9 +204,9 @@ __global__ void __launch_bounds__(kMaxMultiColumns / 8 * 32)
 
   const int js = ulo / kSliceTokens;  // first 16-token slice
   const int n = (uhi + kSliceTokens - 1) / kSliceTokens - js;
-  const int32_t* table = p.block_tables + (size_t)b * p.max_blocks;
 
   // Warp 0 issues slice i into stage i % ST.
+  const int32_t* table = p.block_tables + (size_t)kv_seq * p.max_blocks;
   auto issue = [&](int i) {
     const int t = (js + i) * kSliceTokens;
     const int phys = table[t >> p.log2_bs];
@@ -156,12 +218,13 @@ __global__ void __launch_bounds__(kMaxMultiColumns / 8 * 32)
     for (; issued < ST && issued < n; ++issued) issue(issued);
 
   // Q^T as the B operand: column n = lane / 4 of the warp's 8 is query column
-  // 8*warp + n; padding columns are zero.
+  // 8*warp + n, whose query row is its output row; padding columns are zero.
   uint32_t qf[D / 16][2];
   {
     const int c = warp * 8 + (lane >> 2);
-    const bool real = c < ntok * G;
-    const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q) + row_of(real ? c : 0) * D;
+    const QueryCol qcol = c < ncols ? column(c) : QueryCol{0, 0, 0, false, false};
+    const bool real = qcol.real;
+    const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q) + (real ? qcol.row : 0) * D;
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
       const int d = kk * 16 + 2 * (lane & 3);
@@ -211,15 +274,13 @@ __global__ void __launch_bounds__(kMaxMultiColumns / 8 * 32)
   st.reduce_sums();
 
   // ---- this warp's columns: final rows or partials, from registers -----------------
-  const int cols = ntok * G;
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
-    const int c = c0 + e;
-    if (c >= cols) continue;
+    if (!qc[e].real) continue;
     const float m = e ? st.m1 : st.m0;
     const float l = e ? st.l1 : st.l0;
-    const size_t row = row_of(c);
-    if (final_write) {
+    const size_t row = qc[e].row;
+    if (qc[e].fin) {
       const float inv = l > 0.f ? 1.f / l : 0.f;  // a column with no position gives a zero row
       __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + row * D;
 #pragma unroll

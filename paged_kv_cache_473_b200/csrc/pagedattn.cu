@@ -219,7 +219,8 @@ cudaError_t launch_multi_t(const DecodeParams& p, dim3 grid, int warps, cudaStre
 // 32-64 KB of K/V slices.
 template <bool SPLIT>
 cudaError_t launch_multi(const DecodeParams& p, dim3 grid, cudaStream_t st) {
-  const int warps = ((p.cu_q ? p.q_tile : p.q_len) * p.group + 7) / 8;
+  // Columns per CTA: a prefill tile's or a cascade group's q_tile x G, else T x G.
+  const int warps = (((p.cu_q || p.cascade_prefix) ? p.q_tile : p.q_len) * p.group + 7) / 8;
   switch (p.head_dim) {
     case 64:
       return launch_multi_t<64, 8, SPLIT>(p, grid, warps, st);
@@ -735,6 +736,84 @@ pa_status_t pa_prefill(const void* q, const void* k_new, const void* v_new, cons
   if (e != cudaSuccess) return PA_ERR_CUDA;
   t_last_launches = append ? 2 : 1;
   return PA_OK;
+}
+
+// Cascade partition: the requested one (it must divide prefix_len), or the
+// library's choice halved until it divides prefix_len (a multiple of 64).
+int32_t cascade_partition(int32_t batch, int32_t num_kv_heads, int32_t max_context_len, int32_t prefix_len,
+                          int32_t partition_tokens) {
+  if (partition_tokens > 0) return prefix_len % partition_tokens == 0 ? partition_tokens : -1;
+  int32_t P = auto_partition(batch, num_kv_heads, max_context_len, 0);
+  while (P > 64 && prefix_len % P != 0) P >>= 1;
+  return P;
+}
+
+pa_status_t pa_decode_cascade(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+                              const int32_t* context_lens, int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                              int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq, int32_t num_blocks,
+                              float scale, float softcap, int32_t window, void* out, pa_dtype_t dtype,
+                              int32_t n_sharers, int32_t prefix_len, int32_t partition_tokens,
+                              int32_t max_context_len, void* workspace, size_t workspace_bytes, pa_stream_t stream) {
+  t_last_launches = 0;
+  const Shape s{batch, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks};
+  pa_status_t st = check_decode_args(q, k_cache, v_cache, block_tables, context_lens, s, softcap, out, dtype,
+                                     PA_KERNEL_MMA);
+  if (st != PA_OK) return st;
+  if (n_sharers < 0 || n_sharers > batch || prefix_len < 0 || max_context_len <= 0) return PA_ERR_INVALID;
+  if (partition_tokens < 0 || (partition_tokens > 0 && partition_tokens % 64 != 0)) return PA_ERR_INVALID;
+  if (prefix_len % 64 != 0 || prefix_len % block_size != 0 || prefix_len > max_context_len ||
+      (long long)prefix_len > (long long)max_blocks_per_seq * block_size)
+    return PA_ERR_INVALID;
+  if (n_sharers == 0 || prefix_len == 0)  // nothing shared: the plain split-K call
+    return pa_decode_splitk(q, k_cache, v_cache, block_tables, context_lens, batch, num_q_heads, num_kv_heads,
+                            head_dim, block_size, max_blocks_per_seq, num_blocks, scale, softcap, window, out, dtype,
+                            partition_tokens, max_context_len, workspace, workspace_bytes, PA_KERNEL_MMA, stream);
+  const int32_t P = cascade_partition(batch, num_kv_heads, max_context_len, prefix_len, partition_tokens);
+  if (P <= 0) return PA_ERR_INVALID;
+  const long long parts = splitk_parts(max_context_len, P);
+  if (parts > kMaxPartsPerSeq) return PA_ERR_UNSUPPORTED;
+  const size_t need = workspace_size(batch, num_q_heads, head_dim, max_context_len, P);
+  if (!workspace || !aligned(workspace, 16) || workspace_bytes < need) return PA_ERR_WORKSPACE;
+
+  DecodeParams p = make_params(q, k_cache, v_cache, block_tables, context_lens, s, scale, softcap, window, out);
+  p.partition = P;
+  p.max_parts = (int)parts;
+  p.max_context = max_context_len < p.max_context ? max_context_len : p.max_context;
+  const size_t rows = (size_t)batch * num_q_heads * parts;
+  char* ws = static_cast<char*>(workspace);
+  p.ws_o = reinterpret_cast<float*>(ws + pa::kCounterBytes);
+  p.ws_ml = reinterpret_cast<float*>(ws + pa::kCounterBytes + align256(rows * head_dim * 4));
+  p.n_sharers = n_sharers;
+  p.prefix_len = prefix_len;
+  // 1. The shared prefix, once per (partition, kv head) for up to 64/G sharers per CTA.
+  DecodeParams pp = p;
+  pp.cascade_prefix = 1;
+  pp.q_tile = pa::kMaxMultiColumns / (num_q_heads / num_kv_heads);
+  const unsigned groups = (unsigned)((n_sharers + pp.q_tile - 1) / pp.q_tile);
+  cudaError_t e = launch_multi<true>(pp, dim3((unsigned)(prefix_len / P), num_kv_heads, groups), stream);
+  if (e != cudaSuccess) return PA_ERR_CUDA;
+  // 2. Every sequence's own range (sharers from prefix_len on), split-K.
+  e = launch_decode<true, false>(p, dtype, PA_KERNEL_MMA, dim3((unsigned)parts, num_kv_heads, batch), stream);
+  if (e != cudaSuccess) return PA_ERR_CUDA;
+  // 3. Merge the prefix and suffix partials.
+  e = launch_combine<__nv_bfloat16>(p, stream);
+  if (e != cudaSuccess) return PA_ERR_CUDA;
+  t_last_launches = 3;
+  return PA_OK;
+}
+
+size_t pa_decode_cascade_workspace_size(int32_t batch, int32_t num_q_heads, int32_t head_dim,
+                                        int32_t max_context_len, int32_t prefix_len, int32_t partition_tokens,
+                                        int32_t num_kv_heads) {
+  if (batch <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_context_len <= 0 || prefix_len < 0) return 0;
+  if (prefix_len == 0)
+    return pa_decode_splitk_workspace_size(batch, num_q_heads, head_dim, max_context_len, partition_tokens,
+                                           num_kv_heads);
+  const int32_t P = cascade_partition(batch, num_kv_heads, max_context_len, prefix_len, partition_tokens);
+  if (P <= 0) return 0;
+  return std::max(workspace_size(batch, num_q_heads, head_dim, max_context_len, P),
+                  pa_decode_splitk_workspace_size(batch, num_q_heads, head_dim, max_context_len, partition_tokens,
+                                                  num_kv_heads));
 }
 
 size_t pa_decode_multi_workspace_size(int32_t batch, int32_t q_len, int32_t num_q_heads, int32_t head_dim,

@@ -331,6 +331,34 @@ def make_prefill_inputs(batch: Batch, q_lens, seed: Optional[int] = None, device
             "max_q_len": max(ql) if ql else 0}
 
 
+def order_for_cascade(batch: Batch):
+    """Reorder a prefix-sharing batch for the cascade decode: the sequences
+    whose tables start with all of the shared blocks come first.  Returns
+    ``(batch, n_sharers, prefix_len)``; prefix_len = shared blocks * block_size
+    rounded down to a multiple of 64 (0 when nothing is shared)."""
+    w = batch.workload
+    shared = batch.shared_blocks.tolist()
+    k = len(shared)
+    bs = w.block_size
+    prefix_len = (k * bs) // 64 * 64
+    if k == 0 or prefix_len == 0:
+        return batch, 0, 0
+    nblk = prefix_len // bs
+    tables = batch.block_tables.to("cpu")
+    ref = torch.tensor(shared[:nblk], dtype=torch.int32)
+    is_sharer = [bool(torch.equal(tables[b, :nblk], ref)) for b in range(tables.shape[0])]
+    order = [b for b in range(len(is_sharer)) if is_sharer[b]] + [b for b in range(len(is_sharer)) if not is_sharer[b]]
+    idx = torch.tensor(order, dtype=torch.long)
+    dev = batch.q.device
+    kw = {f: getattr(batch, f) for f in ("workload", "k_cache", "v_cache", "live_per_block", "shared_blocks",
+                                          "prefilled")}
+    kw.update(q=batch.q[idx.to(dev)], k_new=batch.k_new[idx.to(dev)], v_new=batch.v_new[idx.to(dev)],
+              slot_mapping=batch.slot_mapping[idx.to(batch.slot_mapping.device)],
+              block_tables=batch.block_tables[idx.to(batch.block_tables.device)],
+              context_lens=batch.context_lens[idx.to(batch.context_lens.device)])
+    return Batch(**kw), sum(is_sharer), prefix_len
+
+
 def kv_bytes(batch: Batch, unique: bool = False, window: Optional[int] = None) -> int:
     """KV bytes one decode pass must read: sum over sequences of
     ``L_eff * Hkv * 2 * D * elem_bytes`` (``L_eff`` = attended positions).

@@ -31,7 +31,8 @@ def test_header_declares_the_entry_points():
     for n in ["pa_write_kv", "pa_decode", "pa_decode_splitk", "pa_decode_splitk_workspace_size",
               "pa_decode_splitk_partition", "pa_device_errors", "pa_error_string", "pa_last_launch_count",
               "pa_decode_step", "pa_decode_splitk_noalloc", "pa_decode_multi", "pa_decode_multi_workspace_size",
-              "pa_prefill", "pa_copy_blocks", "pa_bm_create", "pa_bm_append_slots", "pa_bm_block_tables"]:
+              "pa_prefill", "pa_copy_blocks", "pa_bm_create", "pa_bm_append_slots", "pa_bm_block_tables",
+              "pa_decode_cascade", "pa_decode_cascade_workspace_size"]:
         assert n in names
 
 
@@ -230,3 +231,36 @@ def test_copy_blocks_host_checks(kw, status):
     assert bnd.lib.pa_copy_blocks(a["k"], a["v"], a["pairs"], a["n"], a["nb"], a["bs"], a["hkv"], a["d"], a["dt"],
                                   None) == status
     assert pa.last_launch_count() == 0
+
+
+def _cascade(**kw):
+    a = dict(B=4, hq=8, hkv=2, d=128, bs=16, mb=128, nb=512, dt=bnd.PA_BF16, nsh=2, plen=1024, P=0, maxL=2048,
+             ws=None, wsb=0)
+    a.update(kw)
+    return bnd.lib.pa_decode_cascade(A, A, A, A, A, a["B"], a["hq"], a["hkv"], a["d"], a["bs"], a["mb"], a["nb"],
+                                     0.1, 0.0, 0, A, a["dt"], a["nsh"], a["plen"], a["P"], a["maxL"], a["ws"],
+                                     a["wsb"], None)
+
+
+@pytest.mark.parametrize(
+    "kw,status",
+    [
+        (dict(nsh=5), bnd.PA_ERR_INVALID),  # more sharers than sequences
+        (dict(plen=1000), bnd.PA_ERR_INVALID),  # not a multiple of 64
+        (dict(plen=4096), bnd.PA_ERR_INVALID),  # beyond max_context_len
+        (dict(P=384), bnd.PA_ERR_INVALID),  # does not divide the prefix
+        (dict(P=100), bnd.PA_ERR_INVALID),
+        (dict(dt=bnd.PA_F32), bnd.PA_ERR_UNSUPPORTED),
+        (dict(), bnd.PA_ERR_WORKSPACE),
+        (dict(B=0, nsh=0), bnd.PA_OK),
+    ],
+)
+def test_cascade_host_checks(kw, status):
+    assert _cascade(**kw) == status
+
+
+def test_cascade_workspace_covers_its_partition():
+    # partition 0: the library's choice halved to divide the prefix; never below the split-K size
+    n = pa.decode_cascade_workspace_size(128, 32, 128, 8192, 1024, 0, 8)
+    assert n >= pa.decode_splitk_workspace_size(128, 32, 128, 8192, 0, 8)
+    assert pa.decode_cascade_workspace_size(128, 32, 128, 8192, 1024, 384, 8) == 0
