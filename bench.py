@@ -391,6 +391,39 @@ class PrefillRunner(Runner):
         self.launches_per_step = n
 
 
+class CascadeRunner(Runner):
+    """The prefix-sharing workload through pa_decode_cascade: the sequences
+    that hold the whole shared prefix go first and read it once per kv head.
+    A step is only that call (the KV already holds every position)."""
+
+    def __init__(self, w: wl.Workload, rank: int):
+        super().__init__(w, rank, "auto", True, 0, fused=True)
+        b = self.batch
+        for kc, vc in self.pools:  # position L-1 live too, as in the decode step after its append
+            self.pa.write_kv(b.k_new, b.v_new, b.slot_mapping, kc, vc)
+        self.batch, self.n_sharers, self.prefix_len = wl.order_for_cascade(b)
+        nbytes = self.pa.decode_cascade_workspace_size(self.B, w.num_q_heads, w.head_dim, self.max_ctx,
+                                                       self.prefix_len, 0, w.num_kv_heads)
+        self.ws = torch.zeros(max(16, nbytes), dtype=torch.uint8, device="cuda")
+        torch.cuda.synchronize()
+
+    def decode(self, r, x):
+        w, b = self.w, self.batch
+        kc, vc = self.pools[r]
+        self.pa.decode_cascade(b.q, kc, vc, b.block_tables, b.context_lens, w.scale, w.softcap, w.window,
+                               n_sharers=self.n_sharers, prefix_len=self.prefix_len, max_context_len=self.max_ctx,
+                               out=self.out, workspace=self.ws)
+        return self.pa.last_launch_count()
+
+    def step(self, r, x=None, ev=None):
+        if ev is not None:
+            ev[0].record()
+        n = self.decode(r, None)
+        if ev is not None:
+            ev[1].record()
+        self.launches_per_step = n
+
+
 def run_timed(runner: Runner, K: int, W: int, world: int, device_index: int):
     """Warm up W steps, then time exactly K graph-replayed steps."""
     for i in range(W):
@@ -616,6 +649,29 @@ def prefill_summary(w: wl.Workload, n_prompts: int, prompt_len: int, rank: int, 
     return res
 
 
+def cascade_summary(w: wl.Workload, rank: int, K: int, W: int, world: int, dev_idx: int, peak: float):
+    """The prefix-sharing workload through the cascade decode: logical and
+    unique KV GB/s (each shared block counted once)."""
+    runner = CascadeRunner(w, rank)
+    total_ms, _, _ = run_timed(runner, K, W, world, dev_idx)
+    ms = total_ms / K
+    res = {
+        "n_sharers": runner.n_sharers,
+        "prefix_len": runner.prefix_len,
+        "tokens_per_s": round(runner.B / (ms * 1e-3), 1),
+        "ms_per_step": round(ms, 5),
+        "decode_gbs": round(runner.kv_bytes / (ms * 1e-3) / 1e9, 1),
+        "decode_gbs_unique": round(runner.kv_bytes_unique / (ms * 1e-3) / 1e9, 1),
+        "decode_frac_unique": round(runner.kv_bytes_unique / (ms * 1e-3) / 1e9 / peak, 4),
+        "launches_per_step": runner.launches_per_step,
+        "kv_bytes": runner.kv_bytes,
+        "kv_bytes_unique": runner.kv_bytes_unique,
+    }
+    del runner
+    torch.cuda.empty_cache()
+    return res
+
+
 def main_ours(args, world, rank, local):
     w = wl.WORKLOADS[args.workload]
     split = not args.no_split
@@ -689,6 +745,9 @@ def main_ours(args, world, rank, local):
         for n, T in MULTI_SHAPES:
             if args.shapes == "auto" or n in names or n == w.name:
                 extra[f"{n}@multi{T}"] = multi_summary(wl.WORKLOADS[n], T, rank, 50, 5, world, local, peak)
+        for n in [n for n in wl.WORKLOADS if wl.WORKLOADS[n].prefix_share > 0]:
+            if args.shapes == "auto" or n in names or n == w.name:
+                extra[f"{n}@cascade"] = cascade_summary(wl.WORKLOADS[n], rank, 50, 5, world, local, peak)
         for n, P_, T in PREFILL_SHAPES:
             if args.shapes == "auto" or n in names or n == w.name:
                 extra[f"{n}@prefill{P_}x{T}"] = prefill_summary(wl.WORKLOADS[n], P_, T, rank, 20, 3, world, local)

@@ -71,6 +71,14 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int& to
 // Partitions of sequence b's attended range [s0, L) (0 when it is empty).
 __device__ __forceinline__ int seq_parts(int L, int s0, int P) { return L > s0 ? (L + P - 1) / P - s0 / P : 0; }
 
+// First position this kernel attends for sequence b: the window start, or
+// (CASCADE) the end of the shared prefix for a sharer.
+template <bool CASCADE>
+__device__ __forceinline__ int seq_start(const DecodeParams& p, int b, int L) {
+  const int s0 = window_start(L, p.window);
+  return (CASCADE && b < p.n_sharers) ? max(s0, p.prefix_len) : s0;
+}
+
 struct Item {
   int b, g, part;  // sequence, kv head, absolute partition index
   int L, lo, hi;   // context length; attended tokens [lo, hi) of this item
@@ -150,8 +158,13 @@ struct DynCfg {
   static __host__ __device__ constexpr int smem_bytes(int B) { return kPrefixOffset + (2 * B + 1) * 4 + 1024; }
 };
 
-template <int D, int NW, int ST, bool APPEND>
-__global__ void __launch_bounds__(NW * 32)
+// Resident CTAs per SM the configurations are sized for (shared memory allows
+// that many): the register budget ptxas may use follows from it.
+template <int D>
+constexpr int dynamic_min_blocks() { return D == 128 ? 3 : 2; }
+
+template <int D, int NW, int ST, bool APPEND, bool CASCADE = false>
+__global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
     decode_dynamic_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                           const DecodeParams p) {
   using Cfg = DynCfg<D, NW, ST>;
@@ -195,7 +208,7 @@ __global__ void __launch_bounds__(NW * 32)
     int items = 0;
     if (b < B) {
       const int L = lens[b];
-      items = Hkv * seq_parts(L, window_start(L, p.window), P);
+      items = Hkv * seq_parts(L, seq_start<CASCADE>(p, b, L), P);
     }
     int total;
     const int ex = block_exclusive_scan(items, scratch, total);
@@ -205,9 +218,11 @@ __global__ void __launch_bounds__(NW * 32)
   if (tid == 0) pre[B] = base;
   __syncthreads();
   const int T = pre[B];
-  // Sequences with nothing to attend (L == 0) get zero rows; no item covers them.
+  // Sequences with nothing to attend (L == 0) get zero rows; no item covers
+  // them.  (A cascade sharer whose range lies inside the shared prefix has no
+  // item either: the prefix pass writes its rows.)
   for (int b = blockIdx.x; b < B; b += gridDim.x) {
-    if (pre[b + 1] != pre[b]) continue;
+    if (pre[b + 1] != pre[b] || (CASCADE && lens[b] != 0)) continue;
     __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + (size_t)b * p.hq * D;
     for (int i = tid; i < p.hq * D; i += blockDim.x) o[i] = __float2bfloat16_rn(0.f);
   }
@@ -225,16 +240,17 @@ __global__ void __launch_bounds__(NW * 32)
     const int r = t - pre[lo];
     it.g = r / parts;
     const int L = lens[lo];
-    const int s0 = window_start(L, p.window);
-    it.pb = s0 / P;
+    const int st = seq_start<CASCADE>(p, lo, L);
+    it.pb = st / P;
     it.parts = parts;
     it.part = it.pb + (r - it.g * parts);
     it.L = L;
-    it.lo = max(s0, it.part * P);
+    it.lo = max(st, it.part * P);
     it.hi = min(L, it.part * P + P);
     it.j0 = it.lo / kSliceTokens;
     it.n = (it.hi + kSliceTokens - 1) / kSliceTokens - it.j0;
-    it.whole = parts == 1;
+    // (a cascade sharer's prefix partials come from the prefix pass)
+    it.whole = parts == 1 && (!CASCADE || st == window_start(L, p.window));
     return it;
   };
 
@@ -429,6 +445,10 @@ __global__ void __launch_bounds__(NW * 32)
       p.queue[1] = 0;
     }
   }
+  // In a cascade this grid is a programmatic dependent of the prefix pass
+  // (which it does not read): it finishes only after that pass has, so the
+  // combine that waits for this grid also sees the prefix partials.
+  if (CASCADE) pdl_wait();
 }
 
 }  // namespace pa

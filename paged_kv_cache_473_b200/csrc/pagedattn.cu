@@ -333,15 +333,15 @@ cudaError_t set_smem_at_least(Kernel k, int bytes, std::atomic<int>* done /* [64
 // (launch, grid drain, L2 round trips) would be a large share of the step;
 // otherwise the combine kernel merges them with full-GPU parallelism after
 // the decode grid, and the merging warps do not stall their loads.
-template <int D, int NW, int ST, bool APPEND>
-cudaError_t launch_dynamic_t(DecodeParams& p, cudaStream_t st) {
+template <int D, int NW, int ST, bool APPEND, bool CASCADE>
+cudaError_t launch_dynamic_t(DecodeParams& p, cudaStream_t st, bool pdl, bool allow_merge) {
   using Cfg = pa::DynCfg<D, NW, ST>;
   CUtensorMap kmap, vmap;
   const long long rows = (long long)p.num_blocks * p.hkv * p.block_size;
   if (!tensor_map_encoder()) return cudaErrorNotSupported;
   if (!encode_cache_map(&kmap, p.k_cache, D, rows) || !encode_cache_map(&vmap, p.v_cache, D, rows))
     return cudaErrorInvalidValue;
-  auto kern = pa::decode_dynamic_kernel<D, NW, ST, APPEND>;
+  auto kern = pa::decode_dynamic_kernel<D, NW, ST, APPEND, CASCADE>;
   const int smem = Cfg::smem_bytes(p.batch);
   static std::atomic<int> smem_done[64];
   cudaError_t e = set_smem_at_least(kern, smem, smem_done);
@@ -352,21 +352,25 @@ cudaError_t launch_dynamic_t(DecodeParams& p, cudaStream_t st) {
   if (occ < 1) return cudaErrorInvalidConfiguration;
   const int grid = occ * sm_count();
   const long long unit_bound = (long long)p.batch * p.hkv * p.max_parts;
-  p.merge_in_kernel = (p.max_parts <= 8 && unit_bound <= 2LL * grid * NW) ? 1 : 0;
-  return launch_ex(kern, dim3(grid), dim3(Cfg::kThreads), smem, st, false, kmap, vmap, p);
+  p.merge_in_kernel = (allow_merge && p.max_parts <= 8 && unit_bound <= 2LL * grid * NW) ? 1 : 0;
+  return launch_ex(kern, dim3(grid), dim3(Cfg::kThreads), smem, st, pdl, kmap, vmap, p);
 }
 
-template <bool APPEND>
+// CASCADE: the cascade's own-range pass (sharers start at the prefix end),
+// launched as a programmatic dependent of the prefix pass, merged by the
+// combine.
+template <bool APPEND, bool CASCADE = false>
 cudaError_t launch_dynamic(DecodeParams& p, cudaStream_t st) {
+  const bool pdl = CASCADE, allow_merge = !CASCADE;
   switch (p.head_dim) {
     // Warps are independent (one work item each); CTAs of a few warps with a
     // 2-6 stage ring each put ~192 KB of loads in flight per SM.
     case 64:
-      return launch_dynamic_t<64, 4, 6, APPEND>(p, st);
+      return launch_dynamic_t<64, 4, 6, APPEND, CASCADE>(p, st, pdl, allow_merge);
     case 128:
-      return launch_dynamic_t<128, 4, 2, APPEND>(p, st);
+      return launch_dynamic_t<128, 4, 2, APPEND, CASCADE>(p, st, pdl, allow_merge);
     default:
-      return launch_dynamic_t<256, 2, 2, APPEND>(p, st);
+      return launch_dynamic_t<256, 2, 2, APPEND, CASCADE>(p, st, pdl, allow_merge);
   }
 }
 
@@ -738,12 +742,22 @@ pa_status_t pa_prefill(const void* q, const void* k_new, const void* v_new, cons
   return PA_OK;
 }
 
+// Whether the cascade's own-range pass runs the dynamic schedule (the library
+// chooses the partition and the shape fits it).
+bool cascade_dynamic(int32_t batch, int32_t num_kv_heads, int32_t partition_tokens) {
+  return partition_tokens == 0 && batch <= pa::kMaxDynamicBatch &&
+         (long long)batch * num_kv_heads <= pa::kMaxDynamicUnits;
+}
+
 // Cascade partition: the requested one (it must divide prefix_len), or the
-// library's choice halved until it divides prefix_len (a multiple of 64).
+// library's choice (the dynamic schedule's, else the grid's) halved until it
+// divides prefix_len (a multiple of 64).
 int32_t cascade_partition(int32_t batch, int32_t num_kv_heads, int32_t max_context_len, int32_t prefix_len,
-                          int32_t partition_tokens) {
+                          int32_t partition_tokens, int32_t head_dim) {
   if (partition_tokens > 0) return prefix_len % partition_tokens == 0 ? partition_tokens : -1;
-  int32_t P = auto_partition(batch, num_kv_heads, max_context_len, 0);
+  int32_t P = cascade_dynamic(batch, num_kv_heads, partition_tokens)
+                  ? dynamic_partition(batch, num_kv_heads, max_context_len, head_dim)
+                  : auto_partition(batch, num_kv_heads, max_context_len, 0);
   while (P > 64 && prefix_len % P != 0) P >>= 1;
   return P;
 }
@@ -768,8 +782,10 @@ pa_status_t pa_decode_cascade(const void* q, const void* k_cache, const void* v_
     return pa_decode_splitk(q, k_cache, v_cache, block_tables, context_lens, batch, num_q_heads, num_kv_heads,
                             head_dim, block_size, max_blocks_per_seq, num_blocks, scale, softcap, window, out, dtype,
                             partition_tokens, max_context_len, workspace, workspace_bytes, PA_KERNEL_MMA, stream);
-  const int32_t P = cascade_partition(batch, num_kv_heads, max_context_len, prefix_len, partition_tokens);
+  const int32_t P =
+      cascade_partition(batch, num_kv_heads, max_context_len, prefix_len, partition_tokens, head_dim);
   if (P <= 0) return PA_ERR_INVALID;
+  const bool dynamic = cascade_dynamic(batch, num_kv_heads, partition_tokens);
   const long long parts = splitk_parts(max_context_len, P);
   if (parts > kMaxPartsPerSeq) return PA_ERR_UNSUPPORTED;
   const size_t need = workspace_size(batch, num_q_heads, head_dim, max_context_len, P);
@@ -792,8 +808,17 @@ pa_status_t pa_decode_cascade(const void* q, const void* k_cache, const void* v_
   const unsigned groups = (unsigned)((n_sharers + pp.q_tile - 1) / pp.q_tile);
   cudaError_t e = launch_multi<true>(pp, dim3((unsigned)(prefix_len / P), num_kv_heads, groups), stream);
   if (e != cudaSuccess) return PA_ERR_CUDA;
-  // 2. Every sequence's own range (sharers from prefix_len on), split-K.
-  e = launch_decode<true, false>(p, dtype, PA_KERNEL_MMA, dim3((unsigned)parts, num_kv_heads, batch), stream);
+  // 2. Every sequence's own range (sharers from prefix_len on), split-K: the
+  // dynamic schedule as a programmatic dependent of the prefix pass (the two
+  // overlap; it waits for the prefix pass only before it exits), merged by
+  // the combine; or the grid schedule after it.
+  if (dynamic) {
+    p.queue = reinterpret_cast<int*>(ws);
+    p.unit_count = p.queue + 2;
+    e = launch_dynamic<false, true>(p, stream);
+  } else {
+    e = launch_decode<true, false>(p, dtype, PA_KERNEL_MMA, dim3((unsigned)parts, num_kv_heads, batch), stream);
+  }
   if (e != cudaSuccess) return PA_ERR_CUDA;
   // 3. Merge the prefix and suffix partials.
   e = launch_combine<__nv_bfloat16>(p, stream);
@@ -809,7 +834,8 @@ size_t pa_decode_cascade_workspace_size(int32_t batch, int32_t num_q_heads, int3
   if (prefix_len == 0)
     return pa_decode_splitk_workspace_size(batch, num_q_heads, head_dim, max_context_len, partition_tokens,
                                            num_kv_heads);
-  const int32_t P = cascade_partition(batch, num_kv_heads, max_context_len, prefix_len, partition_tokens);
+  const int32_t P =
+      cascade_partition(batch, num_kv_heads, max_context_len, prefix_len, partition_tokens, head_dim);
   if (P <= 0) return 0;
   return std::max(workspace_size(batch, num_q_heads, head_dim, max_context_len, P),
                   pa_decode_splitk_workspace_size(batch, num_q_heads, head_dim, max_context_len, partition_tokens,
