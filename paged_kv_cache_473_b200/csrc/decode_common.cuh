@@ -36,6 +36,7 @@ struct DecodeParams {
   int* queue;                   // dynamic schedule: [0] work-item counter, [1] CTAs finished (zero between calls)
   int* unit_count;              // dynamic schedule: partials stored per (sequence, kv head) (zero between calls)
   int merge_in_kernel;          // dynamic schedule: the last partial of a unit merges it (else the combine kernel)
+  int static_items;             // dynamic schedule: items per warp fixed by its index (1 or 2) before claims
   int batch, hq, hkv, group, head_dim;
   int q_len;        // query tokens per sequence (1 for decode; T for the multi-query rows [B][T][Hq][D])
   const int32_t* cu_q;  // prefill: sequence b's query rows are [cu_q[b], cu_q[b+1]) of [total][Hq][D] (else null)

@@ -254,11 +254,33 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
     return it;
   };
 
+  // The first p.static_items (1 or 2) items of a warp are fixed by its index
+  // (wg, W + wg); later ones are claimed from the counter, offset by
+  // static_items * W.  One claim is always in flight ahead of use and is read
+  // only when its item is needed, so no warp waits on the counter at launch.
+  const int n_static = p.static_items;
+  const int claim_base = n_static * W;
   int t_cur = wg;       // item being computed
-  int t_next = W + wg;  // item after it
+  int t_next = W + wg;  // item after it, valid when next_known
+  bool next_known = n_static >= 2;
   if (t_cur < T) {  // else this warp has no item; it still joins the final barrier
-    int t_claim = 0;         // lane 0: the claim after t_next, in flight
-    if (lane == 0 && t_next < T) t_claim = 2 * W + atomicAdd(p.queue, 1);
+    int t_claim = 0;       // lane 0: the claim in flight (for t_next when !next_known, else the item after)
+    bool pending = false;  // a claim is in flight (warp-uniform)
+    if (n_static < 2 || t_next < T) {
+      if (lane == 0) t_claim = (n_static < 2 ? W : claim_base) + atomicAdd(p.queue, 1);
+      pending = true;
+    }
+    // Make t_next known (read the claim in flight) and put the next claim in flight.
+    auto resolve_next = [&]() {
+      if (next_known) return;
+      t_next = pending ? __shfl_sync(FULL, t_claim, 0) : T;
+      next_known = true;
+      pending = false;
+      if (t_next < T) {
+        if (lane == 0) t_claim = claim_base + atomicAdd(p.queue, 1);
+        pending = true;
+      }
+    };
 
     Item ci = decode(t_cur);
     // Load cursor: slice ik of item ii (ii == ci, or the next item once ci is fully issued).
@@ -285,7 +307,9 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
     auto fill = [&]() {
       while (gi - gc < ST) {
         if (ik >= ii.n) {
-          if (i_in_next || t_next >= T) return;
+          if (i_in_next) return;
+          resolve_next();
+          if (t_next >= T) return;
           ii = decode(t_next);
           ik = 0;
           i_in_next = true;
@@ -406,10 +430,10 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
       st.reset();
 
       // ---- next item ------------------------------------------------------------------
+      resolve_next();
       t_cur = t_next;
       if (t_cur >= T) break;
-      t_next = __shfl_sync(FULL, t_claim, 0);
-      if (lane == 0 && t_next < T) t_claim = 2 * W + atomicAdd(p.queue, 1);
+      next_known = false;  // the claim in flight is for the item after t_cur
       if (i_in_next) {
         ci = ii;
 #pragma unroll
@@ -427,6 +451,7 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
       }
     }
 
+    if (pending) t_claim = __shfl_sync(FULL, t_claim, 0);  // every claim lands before the CTA counts out
     if (aborted) {
       if (lane == 0) raise_error(PA_DEVERR_TIMEOUT);
       // Give this warp's loads still in flight a bounded time to land before the
