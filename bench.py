@@ -61,6 +61,12 @@ def parse():
     ap.add_argument("--shapes", default="auto", help="comma list of extra workloads to time, 'none', or 'auto'")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="bound on the CPU-oracle sample")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--op", default="decode", choices=["decode", "multi", "cascade", "prefill"],
+                    help="the timed op: the decode step (default), multi-query rows, the cascade decode of the "
+                         "prefix-sharing shape, or a paged prefill of whole prompts")
+    ap.add_argument("--q-len", type=int, default=4, help="--op multi: query tokens per sequence")
+    ap.add_argument("--prompts", type=int, default=16, help="--op prefill: prompts per step")
+    ap.add_argument("--prompt-len", type=int, default=1024, help="--op prefill: tokens per prompt")
     return ap.parse_args()
 
 
@@ -674,6 +680,8 @@ def cascade_summary(w: wl.Workload, rank: int, K: int, W: int, world: int, dev_i
 
 def main_ours(args, world, rank, local):
     w = wl.WORKLOADS[args.workload]
+    if args.op != "decode":
+        return main_op(args, world, rank, local)
     split = not args.no_split
     runner = Runner(w, rank, args.kernel, split, args.partition, fused=not args.unfused)
     l2 = torch.cuda.get_device_properties(local).L2_cache_size
@@ -758,6 +766,51 @@ def main_ours(args, world, rank, local):
         info = OracleSample(w, b).run(args.cpu_seconds)
         info["value"] = round(info["value"], 2)
         line["cpu_baseline"] = info
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main_op(args, world, rank, local):
+    """One of the other ops as the timed line (multi-query rows, cascade,
+    prefill): the same timing and JSON keys as the decode line; the roofline is
+    HBM for the attention ops and the tensor pipe for the prefill.  No
+    end-to-end leg or CPU baseline (those belong to the decode step)."""
+    w = wl.WORKLOADS[args.workload]
+    if args.op == "multi":
+        runner = MultiRunner(w, rank, args.q_len)
+        per_step, what = runner.B * args.q_len, f"pa_decode_multi, T={args.q_len}"
+    elif args.op == "cascade":
+        runner = CascadeRunner(w, rank)
+        per_step, what = runner.B, f"pa_decode_cascade, {runner.n_sharers} sharers of {runner.prefix_len} positions"
+    else:
+        runner = PrefillRunner(w, rank, args.prompts, args.prompt_len)
+        per_step, what = args.prompts * args.prompt_len, f"pa_prefill, {args.prompts} x {args.prompt_len} tokens"
+    K, W = args.steps, args.warmup
+    total_ms, dec_ms, clocks = run_timed(runner, K, W, world, local)
+    total_ms = max_over_ranks(total_ms, world)
+    ms = total_ms / K
+    value = sum_over_ranks(per_step * K, world) / (total_ms * 1e-3)
+    if args.op == "prefill":
+        peak, kind = tensor_peak(), "measured bf16 burst"
+        achieved = runner.flops / (ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "peak_kind": kind,
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                "algorithmic_flops_per_launch": runner.flops}
+    else:
+        peak, kind = measured_peaks()
+        nbytes = runner.kv_bytes_unique if args.op == "cascade" else runner.kv_bytes
+        achieved = nbytes / (ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "peak_kind": kind, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": None, "algorithmic_bytes_per_launch": nbytes}
+    roof.update(kernel=what, launch_ms=round(ms, 5),
+                launch_timing=f"whole timed region / {K}: each step is only the op's launches, in a CUDA graph")
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w.dtype, "data": "synthetic (seeded; q/k/v ~ N(0,1), shuffled physical blocks)",
+        "config": {"workload": w.name, "op": args.op, "batch": runner.B, "seed": "workload seed + 7919 * rank"},
+        "roofline": roof, "e2e": None, "gpu_launches": K * runner.launches_per_step, "clocks": clocks,
+    }
     if rank == 0:
         print(json.dumps(line), flush=True)
 
