@@ -245,4 +245,149 @@ __device__ __forceinline__ void attend_slice(WarpAttn<D>& st, const uint32_t (&q
   }
 }
 
+// ---- query rows as the MMA M dimension -------------------------------------------
+//
+// For several query tokens per sequence (multi-query rows) with R = T*G <= 16
+// query rows per kv head, the rows fill the 16-row M dimension of the MMA:
+//   S[16 rows x 16 tok] = Q[16 x D] . K^T          (2 n-tiles x D/16 MMAs)
+//   online softmax per row (fp32, log2 domain, quad shuffles)
+//   O[16 x D]          += P[16 x 16] . V[16 x D]     (D/8 n-tiles, one k-step)
+// P goes from the S accumulators straight into the A operand of the second
+// product (the accumulator and A-operand layouts of m16n8k16 line up), K^T
+// is read with ldmatrix and V with ldmatrix.trans from the same swizzled
+// stage as the head-column form.  Lane holds rows r0 = lane/4 and r1 = r0 + 8,
+// and for each 8-column n-tile the columns 2*(lane%4) and +1.
+template <int D>
+struct WarpRows {
+  float m0, m1, l0, l1;
+  float o[D / 8][4];
+
+  __device__ __forceinline__ void reset() {
+    m0 = m1 = -CUDART_INF_F;
+    l0 = l1 = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < D / 8; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+  }
+
+  // Lane partial sums -> row sums (the four lanes of a row share lane / 4).
+  __device__ __forceinline__ void reduce_sums() {
+#pragma unroll
+    for (int off = 1; off < 4; off <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+    }
+  }
+};
+
+// Q as the A operand: rows r0, r1 of the 16 (rows >= R are zero); qrow0/qrow1
+// point at the rows' query vectors.
+template <int D>
+__device__ __forceinline__ void load_q_rows(uint32_t (&qa)[D / 16][4], const __nv_bfloat16* qrow0, bool ok0,
+                                            const __nv_bfloat16* qrow1, bool ok1, int lane) {
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const int c = kk * 16 + 2 * (lane & 3);
+    qa[kk][0] = ok0 ? *reinterpret_cast<const uint32_t*>(qrow0 + c) : 0u;
+    qa[kk][1] = ok1 ? *reinterpret_cast<const uint32_t*>(qrow1 + c) : 0u;
+    qa[kk][2] = ok0 ? *reinterpret_cast<const uint32_t*>(qrow0 + c + 8) : 0u;
+    qa[kk][3] = ok1 ? *reinterpret_cast<const uint32_t*>(qrow1 + c + 8) : 0u;
+  }
+}
+
+// Attend the slice of tokens [t0, t0+16) at kbase/vbase for the lane's rows:
+// row r0 counts tokens in [cr.lo0, cr.hi0), row r1 in [cr.lo1, cr.hi1); V rows
+// outside [lo, hi) (the union) are zeroed.  A row may see no token of the
+// slice; the safe reference maximum keeps its weights at zero.
+template <int D>
+__device__ __forceinline__ void attend_slice_rows(WarpRows<D>& st, const uint32_t (&qa)[D / 16][4], uint32_t kbase,
+                                                  uint32_t vbase, int t0, int lo, int hi, const ColRange& cr,
+                                                  float qk_scale, const DecodeParams& p, int lane) {
+  constexpr uint32_t FULL = 0xffffffffu;
+  const int mi = lane >> 3, mj = lane & 7;  // the ldmatrix row this lane addresses: matrix mi, row mj
+  const int tq = lane & 3;
+
+  // ---- S = Q K^T: n-tiles 0 (tokens 0-7) and 1 (tokens 8-15) -------------------------
+  float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  {
+    // matrix mi: tokens (mi >> 1) * 8 + mj, 16-byte chunk 2*kk + (mi & 1)
+    const int tok = ((mi >> 1) << 3) | mj;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const int chunk = 2 * kk + (mi & 1);
+      const uint32_t addr =
+          kbase + (chunk >> 3) * kPanelBytes + tok * 128 + ((((chunk & 7) ^ (tok & 7))) << 4);
+      uint32_t b00, b01, b10, b11;
+      ldsm_x4(addr, b00, b01, b10, b11);
+      mma_bf16_16816(s[0], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b00, b01);
+      mma_bf16_16816(s[1], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b10, b11);
+    }
+  }
+  // s[nt][0..1]: row r0, tokens t0 + 8 nt + 2 tq (+1); s[nt][2..3]: row r1.
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float v = s[nt][e] * qk_scale;
+      if (p.use_softcap) v = p.softcap * tanhf(v * p.inv_softcap) * kLog2e;
+      const int t = t0 + 8 * nt + 2 * tq + (e & 1);
+      const bool ok = e < 2 ? (t >= cr.lo0 && t < cr.hi0) : (t >= cr.lo1 && t < cr.hi1);
+      s[nt][e] = ok ? v : -CUDART_INF_F;
+    }
+
+  // ---- online softmax per row -----------------------------------------------------
+  float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+  float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
+#pragma unroll
+  for (int off = 1; off < 4; off <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, off));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, off));
+  }
+  const float mn0 = fmaxf(st.m0, mx0), mn1 = fmaxf(st.m1, mx1);
+  const float r0 = mn0 == -CUDART_INF_F ? 0.f : mn0;
+  const float r1 = mn1 == -CUDART_INF_F ? 0.f : mn1;
+  const float al0 = exp2f(st.m0 - r0), al1 = exp2f(st.m1 - r1);
+  st.m0 = mn0;
+  st.m1 = mn1;
+  // P as the A operand of P V (16 rows x 16 tokens).
+  const uint32_t a0 = pack_bf16x2(exp2f(s[0][0] - r0), exp2f(s[0][1] - r0));
+  const uint32_t a1 = pack_bf16x2(exp2f(s[0][2] - r1), exp2f(s[0][3] - r1));
+  const uint32_t a2 = pack_bf16x2(exp2f(s[1][0] - r0), exp2f(s[1][1] - r0));
+  const uint32_t a3 = pack_bf16x2(exp2f(s[1][2] - r1), exp2f(s[1][3] - r1));
+  st.l0 = st.l0 * al0 + bf16_lo(a0) + bf16_hi(a0) + bf16_lo(a2) + bf16_hi(a2);
+  st.l1 = st.l1 * al1 + bf16_lo(a1) + bf16_hi(a1) + bf16_lo(a3) + bf16_hi(a3);
+#pragma unroll
+  for (int nt = 0; nt < D / 8; ++nt) {
+    st.o[nt][0] *= al0;
+    st.o[nt][1] *= al0;
+    st.o[nt][2] *= al1;
+    st.o[nt][3] *= al1;
+  }
+
+  // V rows outside [lo, hi) may hold anything (NaN canaries): zero them.  This
+  // lane's B fragments hold tokens 2 tq, 2 tq + 1 (b0) and 8 + 2 tq, + 1 (b1).
+  uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;
+  if (t0 < lo || t0 + kSliceTokens > hi) {
+    const int tc = t0 + 2 * tq;
+    auto ok = [&](int t) { return t >= lo && t < hi; };
+    keep_lo = (ok(tc) ? 0x0000ffffu : 0u) | (ok(tc + 1) ? 0xffff0000u : 0u);
+    keep_hi = (ok(tc + 8) ? 0x0000ffffu : 0u) | (ok(tc + 9) ? 0xffff0000u : 0u);
+  }
+
+  // ---- O += P V: d n-tiles in pairs (2c, 2c+1) ------------------------------------------
+  {
+    // matrix mi: tokens (mi & 1) * 8 + mj, 16-byte chunk 2c + (mi >> 1)
+    const int tok = ((mi & 1) << 3) | mj;
+#pragma unroll
+    for (int c = 0; c < D / 16; ++c) {
+      const int chunk = 2 * c + (mi >> 1);
+      const uint32_t addr =
+          vbase + (chunk >> 3) * kPanelBytes + tok * 128 + ((((chunk & 7) ^ (tok & 7))) << 4);
+      uint32_t v0, v1, v2, v3;
+      ldsm_x4_trans(addr, v0, v1, v2, v3);
+      mma_bf16_16816(st.o[2 * c], a0, a1, a2, a3, v0 & keep_lo, v1 & keep_hi);
+      mma_bf16_16816(st.o[2 * c + 1], a0, a1, a2, a3, v2 & keep_lo, v3 & keep_hi);
+    }
+  }
+}
+
 }  // namespace pa

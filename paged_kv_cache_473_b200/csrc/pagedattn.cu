@@ -20,6 +20,7 @@
 #include "decode_simt.cuh"
 #include "decode_dynamic.cuh"
 #include "decode_multi.cuh"
+#include "decode_rows.cuh"
 
 namespace {
 
@@ -375,6 +376,35 @@ cudaError_t launch_dynamic(DecodeParams& p, cudaStream_t st) {
   }
 }
 
+// Multi-query rows with T*G <= 16 on the dynamic warp-per-item schedule (the
+// combine merges the partials).
+template <int D, int NW, int ST>
+cudaError_t launch_rows_t(DecodeParams& p, cudaStream_t st) {
+  using Cfg = pa::DynCfg<D, NW, ST>;
+  CUtensorMap kmap, vmap;
+  const long long rows = (long long)p.num_blocks * p.hkv * p.block_size;
+  if (!tensor_map_encoder()) return cudaErrorNotSupported;
+  if (!encode_cache_map(&kmap, p.k_cache, D, rows) || !encode_cache_map(&vmap, p.v_cache, D, rows))
+    return cudaErrorInvalidValue;
+  auto kern = pa::decode_rows_kernel<D, NW, ST>;
+  const int smem = Cfg::smem_bytes(p.batch);
+  static std::atomic<int> smem_done[64];
+  cudaError_t e = set_smem_at_least(kern, smem, smem_done);
+  if (e != cudaSuccess) return e;
+  int occ = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, Cfg::kThreads, smem);
+  if (e != cudaSuccess) return e;
+  if (occ < 1) return cudaErrorInvalidConfiguration;
+  p.merge_in_kernel = 0;
+  p.static_items = 2;
+  return launch_ex(kern, dim3(occ * sm_count()), dim3(Cfg::kThreads), smem, st, false, kmap, vmap, p);
+}
+
+cudaError_t launch_rows(DecodeParams& p, cudaStream_t st) {
+  return p.head_dim == 64 ? launch_rows_t<64, 4, 6>(p, st) : launch_rows_t<128, 4, 2>(p, st);
+}
+
+
 int32_t auto_partition(int32_t batch, int32_t num_kv_heads, int32_t max_context_len, int32_t partition_tokens) {
   if (partition_tokens > 0) return partition_tokens;
   const long long work = (long long)(batch > 0 ? batch : 1) * (num_kv_heads > 0 ? num_kv_heads : 1) *
@@ -654,6 +684,24 @@ pa_status_t pa_decode_step(const void* q, const void* k_new, const void* v_new, 
   return run_decode(c);
 }
 
+// Whether multi-query rows run on the dynamic warp-per-item schedule: at most
+// 16 query rows (T * G) per kv head, head_dim <= 128, and a batch the schedule
+// takes.
+bool multi_rows_path(int32_t batch, int32_t q_len, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim) {
+  return head_dim <= 128 && (long long)q_len * (num_q_heads / num_kv_heads) <= pa::kMaxRowsPerWarp &&
+         batch <= pa::kMaxDynamicBatch && (long long)batch * num_kv_heads <= pa::kMaxDynamicUnits;
+}
+
+// Multi-query partition: the requested one; else the dynamic schedule's choice
+// on that path, the grid schedule's otherwise.
+int32_t multi_partition(int32_t batch, int32_t q_len, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                        int32_t max_context_len, int32_t partition_tokens) {
+  if (partition_tokens > 0) return partition_tokens;
+  return multi_rows_path(batch, q_len, num_q_heads, num_kv_heads, head_dim)
+             ? dynamic_partition(batch, num_kv_heads, max_context_len, head_dim)
+             : auto_partition(batch, num_kv_heads, max_context_len, 0);
+}
+
 pa_status_t pa_decode_multi(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
                             const int32_t* context_lens, int32_t batch, int32_t q_len, int32_t num_q_heads,
                             int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq,
@@ -668,12 +716,13 @@ pa_status_t pa_decode_multi(const void* q, const void* k_cache, const void* v_ca
   if (q_len <= 0) return PA_ERR_INVALID;
   if ((long long)q_len * (num_q_heads / num_kv_heads) > pa::kMaxMultiColumns) return PA_ERR_UNSUPPORTED;
   const bool split = partition_tokens >= 0;
+  const bool rows_path = split && multi_rows_path(batch, q_len, num_q_heads, num_kv_heads, head_dim);
   int P = kNoSplitPartition;
   long long parts = 1;
   if (split) {
     if (partition_tokens > 0 && partition_tokens % 64 != 0) return PA_ERR_INVALID;
     if (max_context_len <= 0) return PA_ERR_INVALID;
-    P = auto_partition(batch, num_kv_heads, max_context_len, partition_tokens);
+    P = multi_partition(batch, q_len, num_q_heads, num_kv_heads, head_dim, max_context_len, partition_tokens);
     parts = splitk_parts(max_context_len, P);
     if (parts > kMaxPartsPerSeq) return PA_ERR_UNSUPPORTED;
     const size_t need = workspace_size(batch, num_q_heads, head_dim, max_context_len, P, q_len);
@@ -691,7 +740,13 @@ pa_status_t pa_decode_multi(const void* q, const void* k_cache, const void* v_ca
     char* ws = static_cast<char*>(workspace);
     p.ws_o = reinterpret_cast<float*>(ws + pa::kCounterBytes);
     p.ws_ml = reinterpret_cast<float*>(ws + pa::kCounterBytes + align256(rows * head_dim * 4));
-    e = launch_multi<true>(p, dim3((unsigned)parts, num_kv_heads, batch), stream);
+    if (rows_path) {  // one warp per (sequence, kv head, partition) item, dynamic schedule
+      p.queue = reinterpret_cast<int*>(ws);
+      p.unit_count = p.queue + 2;
+      e = launch_rows(p, stream);
+    } else {
+      e = launch_multi<true>(p, dim3((unsigned)parts, num_kv_heads, batch), stream);
+    }
     if (e != cudaSuccess) return PA_ERR_CUDA;
     t_last_launches = 1;
     if (parts > 1) {
@@ -846,7 +901,9 @@ size_t pa_decode_cascade_workspace_size(int32_t batch, int32_t num_q_heads, int3
 size_t pa_decode_multi_workspace_size(int32_t batch, int32_t q_len, int32_t num_q_heads, int32_t head_dim,
                                       int32_t max_context_len, int32_t partition_tokens, int32_t num_kv_heads) {
   if (batch <= 0 || q_len <= 0 || num_q_heads <= 0 || head_dim <= 0 || partition_tokens < 0) return 0;
-  const int P = auto_partition(batch, num_kv_heads, max_context_len, partition_tokens);
+  if (num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0) return 0;
+  const int P =
+      multi_partition(batch, q_len, num_q_heads, num_kv_heads, head_dim, max_context_len, partition_tokens);
   if (P <= 0) return 0;
   return workspace_size(batch, num_q_heads, head_dim, max_context_len, P, q_len);
 }

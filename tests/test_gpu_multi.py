@@ -33,6 +33,9 @@ def _case(name, T, **extra):
     w = wl.WORKLOADS[name]
     kw = dict(REDUCED[name])
     kw.update(extra)
+    if "lengths" in kw:
+        kw.pop("batch", None)
+    kw = {k: v for k, v in kw.items() if v is not None}
     b_cpu = wl.make_batch(w, prefilled=True, **kw)
     mq = wl.make_multi_queries(b_cpu, T)
     return w, b_cpu, to_dev(b_cpu), mq
@@ -55,9 +58,9 @@ def _ref(w, b_cpu, q, window=None, softcap=None, rows=None):
                                cap, win, rows=rows)
 
 
-@pytest.mark.parametrize("name,T", [("tinyllama_1b", 1), ("tinyllama_1b", 4), ("tinyllama_1b", 8),
-                                    ("gemma2_2b", 5), ("gemma2_2b", 32), ("llama3_8b", 3), ("llama3_8b", 16),
-                                    ("long_splitk", 6)])
+@pytest.mark.parametrize("name,T", [("tinyllama_1b", 1), ("tinyllama_1b", 2), ("tinyllama_1b", 4),
+                                    ("tinyllama_1b", 8), ("gemma2_2b", 5), ("gemma2_2b", 32), ("llama3_8b", 3),
+                                    ("llama3_8b", 4), ("llama3_8b", 16), ("long_splitk", 4), ("long_splitk", 6)])
 @pytest.mark.parametrize("split,partition", [(False, 0), (True, 0), (True, 64)])
 def test_multi_parity(name, T, split, partition):
     w, b_cpu, b, mq = _case(name, T)
@@ -69,25 +72,30 @@ def test_multi_parity(name, T, split, partition):
 
 @pytest.mark.parametrize("window", [1, 3, 17, 200])
 @pytest.mark.parametrize("split", [False, True])
-def test_multi_window_per_query_token(window, split):
-    """Each query token has its own window start."""
-    w, b_cpu, b, mq = _case("llama3_8b", 6)
+@pytest.mark.parametrize("T", [4, 6])
+def test_multi_window_per_query_token(window, split, T):
+    """Each query token has its own window start (T = 4: 16 query rows per kv
+    head, the warp-per-item path when split; T = 6: the CTA-shared path)."""
+    w, b_cpu, b, mq = _case("llama3_8b", T)
     out = _run(w, b, mq["q"], split, 64, window=window)
     ref = _ref(w, b_cpu, mq["q"], window=window)
     assert_close(out, ref, torch.bfloat16, f"multi window={window} split={split}")
 
 
 @pytest.mark.parametrize("split", [False, True])
-def test_multi_short_and_empty_sequences(split):
+@pytest.mark.parametrize("name,T", [("tinyllama_1b", 5), ("tinyllama_1b", 2), ("llama3_8b", 4)])
+def test_multi_short_and_empty_sequences(split, name, T):
     """L = 0 rows, L < T (early query tokens see nothing: zero rows), L = T,
     ranges inside one slice and across block edges."""
     lengths = [0, 2, 5, 1, 17, 33, 64]
-    w, b_cpu, b, mq = _case("tinyllama_1b", 5, lengths=lengths)
+    w, b_cpu, b, mq = _case(name, T, lengths=lengths, max_len=None)
     out = _run(w, b, mq["q"], split, 64, max_ctx=64)
     ref = _ref(w, b_cpu, mq["q"])
-    assert_close(out, ref, torch.bfloat16, f"multi short split={split}")
+    assert_close(out, ref, torch.bfloat16, f"multi short {name} T={T} split={split}")
     assert torch.count_nonzero(out[0]).item() == 0
-    assert torch.count_nonzero(out[1, :3]).item() == 0 and torch.count_nonzero(out[3, :4]).item() == 0
+    for i, L in enumerate(lengths):
+        if L < T:  # query tokens before the first position
+            assert torch.count_nonzero(out[i, : T - L]).item() == 0
 
 
 def test_multi_softcap_and_verify_flow():
