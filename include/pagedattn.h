@@ -85,7 +85,8 @@ enum {
   PA_DEVERR_BLOCK = 2u,      /* decode: block id outside [0, num_blocks) (tile skipped) */
   PA_DEVERR_CONTEXT = 4u,    /* decode: context_lens[b] < 0 or > max_blocks_per_seq * block_size,
                                 or > max_context_len in split-K (length clamped) */
-  PA_DEVERR_TIMEOUT = 8u     /* a bounded wait on a tile load gave up (output row not written) */
+  PA_DEVERR_TIMEOUT = 8u,    /* a bounded wait on a tile load gave up (output row not written) */
+  PA_DEVERR_LAYOUT = 16u     /* prefill: shared memory was not 1024-byte aligned (tile not computed) */
 };
 
 /*

@@ -10,6 +10,7 @@ from ._binding import (  # noqa: F401
     copy_blocks,
     DEVERR_BLOCK,
     DEVERR_CONTEXT,
+    DEVERR_LAYOUT,
     DEVERR_SLOT,
     DEVERR_TIMEOUT,
     KERNELS,

@@ -16,11 +16,9 @@
 // the normalised rows when the sequence's range is one partition, else the
 // partial state for the combine kernel.
 //
-// Prefill (p.cu_q set): the same kernel over variable-length query blocks.
-// Sequence b's new tokens are rows [cu_q[b], cu_q[b+1]) of q and out, T_b of
-// them, the last T_b positions of its context; CTA x takes the query tile of
-// tokens [x*q_tile, x*q_tile + q_tile) (q_tile*G <= 64 columns) and attends,
-// without split, the union of its tokens' causal ranges.
+// Cascade prefix pass (p.cascade_prefix): the same kernel with sharer columns
+// (sequence x head) over the shared prefix, addressed through sequence 0's
+// table.
 #pragma once
 
 #include "decode_common.cuh"
@@ -66,7 +64,6 @@ __global__ void __launch_bounds__(kMaxMultiColumns / 8 * 32)
   const int g = blockIdx.y;
   const int G = p.group, P = p.partition;
   const bool cascade = p.cascade_prefix != 0;
-  const bool varlen = p.cu_q != nullptr;
 
   // ---- the CTA's K/V range and its query columns ---------------------------------------
   // kv_seq: the sequence whose block table addresses the K/V; [pl, ph): the
@@ -87,21 +84,9 @@ __global__ void __launch_bounds__(kMaxMultiColumns / 8 * 32)
     uhi = min(ulo + P, p.prefix_len);
   } else {
     kv_seq = blockIdx.z;
-    if (varlen) {
-      const int a = p.cu_q[kv_seq], e = p.cu_q[kv_seq + 1];
-      if (a < 0 || e < a || e > p.total_q || e - a > p.max_q_len) {  // malformed offsets: report, write nothing
-        if (blockIdx.x == 0 && g == 0 && threadIdx.x == 0) raise_error(PA_DEVERR_CONTEXT);
-        return;
-      }
-      T = e - a;
-      part = 0;
-      j0 = blockIdx.x * p.q_tile;
-      row0 = (size_t)a + j0;
-    } else {
-      T = p.q_len;
-      row0 = (size_t)kv_seq * T;
-    }
-    const int ntok = min(varlen ? p.q_tile : T, T - j0);
+    T = p.q_len;
+    row0 = (size_t)kv_seq * T;
+    const int ntok = T;
     if (ntok <= 0) return;
     ncols = ntok * G;
     L = clamp_context(p, kv_seq, threadIdx.x == 0 && part == 0 && j0 == 0);

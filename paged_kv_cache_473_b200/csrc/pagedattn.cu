@@ -21,6 +21,7 @@
 #include "decode_dynamic.cuh"
 #include "decode_multi.cuh"
 #include "decode_rows.cuh"
+#include "prefill_umma.cuh"
 
 namespace {
 
@@ -200,6 +201,34 @@ cudaError_t launch_mma(const DecodeParams& p, dim3 grid, cudaStream_t st) {
   }
 }
 
+// Paged prefill attention on tcgen05: one CTA per 128 query rows (128 / G
+// tokens) of one sequence and kv head.
+template <int D>
+cudaError_t launch_prefill_t(const DecodeParams& p, dim3 grid, cudaStream_t st) {
+  using Cfg = pa::PrefillCfg<D>;
+  CUtensorMap kmap, vmap;
+  const long long rows = (long long)p.num_blocks * p.hkv * p.block_size;
+  if (!tensor_map_encoder()) return cudaErrorNotSupported;
+  if (!encode_cache_map(&kmap, p.k_cache, D, rows) || !encode_cache_map(&vmap, p.v_cache, D, rows))
+    return cudaErrorInvalidValue;
+  auto kern = pa::prefill_umma_kernel<D>;
+  static std::atomic<uint64_t> smem_done{0};
+  cudaError_t e = set_smem(kern, Cfg::kSmemBytes, smem_done);
+  if (e != cudaSuccess) return e;
+  return launch_ex(kern, grid, dim3(Cfg::kThreads), Cfg::kSmemBytes, st, false, kmap, vmap, p);
+}
+
+cudaError_t launch_prefill(const DecodeParams& p, dim3 grid, cudaStream_t st) {
+  switch (p.head_dim) {
+    case 64:
+      return launch_prefill_t<64>(p, grid, st);
+    case 128:
+      return launch_prefill_t<128>(p, grid, st);
+    default:
+      return launch_prefill_t<256>(p, grid, st);
+  }
+}
+
 template <int D, int ST, bool SPLIT>
 cudaError_t launch_multi_t(const DecodeParams& p, dim3 grid, int warps, cudaStream_t st) {
   using Cfg = pa::MultiCfg<D, ST>;
@@ -216,12 +245,11 @@ cudaError_t launch_multi_t(const DecodeParams& p, dim3 grid, int warps, cudaStre
 }
 
 // Multi-query rows: one warp per 8 of the T*G query columns of a kv head (or
-// of the q_tile*G columns of a prefill tile); the CTA's shared ring holds
-// 32-64 KB of K/V slices.
+// of the q_tile*G columns of a cascade sharer group); the CTA's shared ring
+// holds 32-64 KB of K/V slices.
 template <bool SPLIT>
 cudaError_t launch_multi(const DecodeParams& p, dim3 grid, cudaStream_t st) {
-  // Columns per CTA: a prefill tile's or a cascade group's q_tile x G, else T x G.
-  const int warps = (((p.cu_q || p.cascade_prefix) ? p.q_tile : p.q_len) * p.group + 7) / 8;
+  const int warps = ((p.cascade_prefix ? p.q_tile : p.q_len) * p.group + 7) / 8;
   switch (p.head_dim) {
     case 64:
       return launch_multi_t<64, 8, SPLIT>(p, grid, warps, st);
@@ -784,7 +812,7 @@ pa_status_t pa_prefill(const void* q, const void* k_new, const void* v_new, cons
     if (st != PA_OK) return st;
   }
   const int G = num_q_heads / num_kv_heads;
-  const int q_tile = pa::kMaxMultiColumns / G;  // G <= 8: 8 .. 64 tokens per CTA
+  const int q_tile = 128 / G;  // one CTA: 128 query rows = q_tile tokens x G heads
   const long long tiles = ((long long)max_q_len + q_tile - 1) / q_tile;
   if (tiles > INT_MAX) return PA_ERR_UNSUPPORTED;
   DecodeParams p = make_params(q, k_cache, v_cache, block_tables, context_lens, s, scale, softcap, window, out);
@@ -792,7 +820,7 @@ pa_status_t pa_prefill(const void* q, const void* k_new, const void* v_new, cons
   p.q_tile = q_tile;
   p.max_q_len = max_q_len;
   p.total_q = total_q;
-  cudaError_t e = launch_multi<false>(p, dim3((unsigned)tiles, num_kv_heads, batch), stream);
+  cudaError_t e = launch_prefill(p, dim3((unsigned)tiles, num_kv_heads, batch), stream);
   if (e != cudaSuccess) return PA_ERR_CUDA;
   t_last_launches = append ? 2 : 1;
   return PA_OK;

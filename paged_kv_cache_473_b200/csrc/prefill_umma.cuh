@@ -1,0 +1,362 @@
+// Paged prefill attention on the 5th-generation tensor cores (tcgen05 / UMMA,
+// accumulators in tensor memory).
+//
+// One CTA takes 128 query rows of one sequence and kv head: TQ = 128 / G query
+// tokens x G heads, row r = (token j0 + r / G, head r % G), the token at
+// position p = L - T + j attending the positions [s0(p + 1), p] of its
+// sequence (causal, sliding window).  The K/V of the union of those ranges
+// stream through a 2-stage ring of 64-token tiles (2-D TMA boxes of 16 rows
+// per physical block, SWIZZLE_128B, which is the canonical K-major layout for
+// K and the MN-major layout for V).  Per tile:
+//   S = Q K^T        UMMA M=128, N=64, K=D     into one of two TMEM S buffers
+//   softmax          warps 0-3: each thread owns one query row (its TMEM lane):
+//                    tcgen05.ld of its 64 scores, scale / softcap / masks,
+//                    online max and sum, O rescale in TMEM when the max moved,
+//                    P (bf16) to shared memory in the canonical K-major layout
+//   O += P V         UMMA M=128, N=D, K=64                into TMEM
+// Warp 4 issues the TMA loads (one box per lane) and, from lane 0, the MMAs;
+// it issues S for the next tile before waiting for this tile's P, so the
+// tensor core computes S(i+1) while the softmax warps work on S(i).  Completion
+// travels through mbarriers (TMA bytes, tcgen05.commit); every wait is
+// bounded.  V rows of a tile outside the union range are zeroed in shared
+// memory before P V (P is 0 there, and a NaN canary would still poison it).
+#pragma once
+
+#include "decode_common.cuh"
+#include "ptx.cuh"
+#include "umma.cuh"
+
+namespace pa {
+
+template <int D>
+struct PrefillCfg {
+  static constexpr int kPanels = D / 64;         // 64-element (128-byte) column panels
+  static constexpr int kTile = 64;               // K/V tokens per stage
+  static constexpr int kStages = D <= 64 ? 4 : 2;
+  static constexpr int kRows = 128;              // query rows per CTA (UMMA M)
+  static constexpr int kQPanelBytes = kRows * 128;
+  static constexpr int kKVPanelBytes = kTile * 128;
+  static constexpr int kKBytes = kPanels * kKVPanelBytes;
+  static constexpr int kStageBytes = 2 * kKBytes;  // K then V
+  static constexpr int kPBytes = kRows * 128;      // 128 rows x 64 bf16
+  static constexpr int kQOff = 0;
+  static constexpr int kStageOff = kPanels * kQPanelBytes;
+  static constexpr int kPOff = kStageOff + kStages * kStageBytes;
+  static constexpr int kBarOff = kPOff + kPBytes;
+  // Exactly the layout plus the barrier area (the dynamic shared-memory base is
+  // 1024-byte aligned; the kernel checks it), and at least 80 KB so that no more
+  // CTAs share an SM than its 512 tensor-memory columns hold (kTmemCols each):
+  // two CTAs per SM for head_dim 64 and 128, one for 256.
+  static constexpr int kSmemBytes = (kBarOff + 128) > 80 * 1024 ? (kBarOff + 128) : 80 * 1024;
+  static_assert(16 * kStages + 40 <= 128, "barrier area");
+  static constexpr int kSCol = 0;                // two S buffers: columns [0, 64) and [64, 128)
+  static constexpr int kOCol = 2 * kTile;        // O: columns [128, 128 + D)
+  static constexpr int kTmemCols = (2 * kTile + D) <= 256 ? 256 : 512;
+  static constexpr int kThreads = 160;           // 4 softmax warps + the TMA / MMA warp
+};
+
+template <int D>
+__global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
+    prefill_umma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                        const DecodeParams p) {
+  using C = PrefillCfg<D>;
+  constexpr uint32_t FULL = 0xffffffffu;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+  const int g = blockIdx.y, b = blockIdx.z, G = p.group;
+  const int TQ = C::kRows / G;
+  if (smem_addr(smem) & 1023) {  // the swizzled tiles need 1024-byte alignment
+    if (tid == 0) raise_error(PA_DEVERR_LAYOUT);
+    return;
+  }
+
+  // ---- this CTA's query tokens and K/V range ------------------------------------------
+  const int a = p.cu_q[b], e = p.cu_q[b + 1];
+  if (a < 0 || e < a || e > p.total_q || e - a > p.max_q_len) {  // malformed offsets: report, write nothing
+    if (blockIdx.x == 0 && g == 0 && tid == 0) raise_error(PA_DEVERR_CONTEXT);
+    return;
+  }
+  const int T = e - a;
+  const int j0 = blockIdx.x * TQ;
+  const int ntok = min(TQ, T - j0);
+  if (ntok <= 0) return;
+  const int L = clamp_context(p, b, blockIdx.x == 0 && g == 0 && tid == 0);
+  const int ulo = window_start(max(L - T + j0 + 1, 0), p.window);
+  const int uhi = min(L, L - T + j0 + ntok);
+  const size_t row0 = (size_t)a + j0;  // q / out row of token j0
+  if (ulo >= uhi) {  // no token of the tile has a position: zero rows
+    for (int idx = tid; idx < ntok * G * D; idx += blockDim.x) {
+      const int r = idx / D;
+      static_cast<__nv_bfloat16*>(p.out)[((row0 + r / G) * p.hq + (size_t)g * G + r % G) * D + idx % D] =
+          __float2bfloat16_rn(0.f);
+    }
+    return;
+  }
+  const int kt0 = (ulo / C::kTile) * C::kTile;
+  const int n_kv = (uhi - kt0 + C::kTile - 1) / C::kTile;
+
+  const uint32_t s_base = smem_addr(smem);
+  const uint32_t q_s = s_base + C::kQOff, st_s = s_base + C::kStageOff, p_s = s_base + C::kPOff;
+  const uint32_t bar = s_base + C::kBarOff;
+  // Barrier area: full[kStages], empty[kStages], sfull[2], pready, odone, the
+  // TMEM address slot and the abort flag (at most 16*4 + 40 bytes of the 128).
+  const uint32_t full_b = bar, empty_b = bar + 8 * C::kStages, sfull_b = bar + 16 * C::kStages;
+  const uint32_t pready_b = sfull_b + 16, odone_b = sfull_b + 24;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + 16 * C::kStages + 32);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kBarOff + 16 * C::kStages + 36);
+
+  if (tid == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(full_b + 8 * s, 1);
+      mbar_init(empty_b + 8 * s, 1);
+    }
+    mbar_init(sfull_b, 1);
+    mbar_init(sfull_b + 8, 1);
+    mbar_init(pready_b, 4);
+    mbar_init(odone_b, 1);
+    *abort_flag = 0;
+    mbar_init_fence();
+    prefetch_tensormap(&kmap);
+    prefetch_tensormap(&vmap);
+  }
+  if (warp == 0) umma::alloc(smem_addr(tmem_slot), C::kTmemCols);
+
+  // ---- Q tile into shared memory (canonical K-major SWIZZLE_128B) ------------------------
+  if (tid < C::kRows) {
+    const int r = tid;
+    const bool real = r / G < ntok;
+    const __nv_bfloat16* qrow =
+        static_cast<const __nv_bfloat16*>(p.q) + ((row0 + r / G) * p.hq + (size_t)g * G + r % G) * D;
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+      const uint4 v = real ? *reinterpret_cast<const uint4*>(qrow + c * 8) : make_uint4(0, 0, 0, 0);
+      const uint32_t dst = q_s + (c >> 3) * C::kQPanelBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                   : "memory");
+    }
+  }
+  fence_proxy_async_smem();
+  umma::fence_before();
+  __syncthreads();
+  umma::fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const float qk_scale = p.use_softcap ? p.scale : p.scale * kLog2e;
+  const int32_t* table = p.block_tables + (size_t)b * p.max_blocks;
+
+  if (warp == 4) {
+    // ================= TMA producer and MMA issuer =================
+    // Tile i: one 2-D box per lane (slice s = lane / (2*panels), K or V, panel).
+    auto issue_tile = [&](int i) {
+      const int stage = i % C::kStages;
+      const int kt = kt0 + i * C::kTile;
+      const int box = lane;
+      const int s = box / (2 * C::kPanels), kv = (box / C::kPanels) & 1, pn = box % C::kPanels;
+      const int t = kt + s * kSliceTokens;
+      bool valid = false;
+      int y = -1;
+      if (box < 8 * C::kPanels && t + kSliceTokens > ulo && t < uhi) {
+        const int phys = table[t >> p.log2_bs];
+        if (phys >= 0 && phys < p.num_blocks) {
+          valid = true;
+          y = cache_row(p, phys, g, t);
+        } else if (kv == 0 && pn == 0) {
+          raise_error(PA_DEVERR_BLOCK);
+        }
+      }
+      const uint32_t nvalid = __popc(__ballot_sync(FULL, valid));
+      if (lane == 0) {
+        if (nvalid) mbar_arrive_expect_tx(full_b + 8 * stage, nvalid * kSliceTokens * 128);
+        else mbar_arrive(full_b + 8 * stage);
+      }
+      __syncwarp();
+      if (valid) {
+        const uint32_t dst = st_s + stage * C::kStageBytes + kv * C::kKBytes + pn * C::kKVPanelBytes + s * kSliceTokens * 128;
+        tma_load_2d(dst, kv ? &vmap : &kmap, full_b + 8 * stage, pn * 64, y);
+      }
+    };
+    const uint32_t idesc_s = umma::idesc_bf16(128, C::kTile, 0, 0);
+    const uint32_t idesc_o = umma::idesc_bf16(128, D, 0, 1);
+    auto issue_s = [&](int i) {  // lane 0: S(i) = Q K(i)^T into buffer i % 2
+      const uint32_t kst = st_s + (i % C::kStages) * C::kStageBytes;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t ad = umma::desc_sw128(q_s + (kk >> 2) * C::kQPanelBytes + (kk & 3) * 32, 16, 1024);
+        const uint64_t bd = umma::desc_sw128(kst + (kk >> 2) * C::kKVPanelBytes + (kk & 3) * 32, 16, 1024);
+        umma::mma_f16(tmem + C::kSCol + (i & 1) * C::kTile, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+      }
+      umma::commit(sfull_b + 8 * (i & 1));
+    };
+    auto issue_o = [&](int i) {  // lane 0: O += P V(i)
+      const uint32_t vst = st_s + (i % C::kStages) * C::kStageBytes + C::kKBytes;
+#pragma unroll
+      for (int k = 0; k < C::kTile / 16; ++k) {
+        const uint64_t ad = umma::desc_sw128(p_s + k * 32, 16, 1024);
+        const uint64_t bd = umma::desc_sw128(vst + k * 16 * 128, C::kKVPanelBytes, 1024);
+        umma::mma_f16(tmem + C::kOCol, ad, bd, idesc_o, (i > 0 || k > 0) ? 1u : 0u);
+      }
+      umma::commit(odone_b);
+      umma::commit(empty_b + 8 * (i % C::kStages));
+    };
+    bool ok = true;
+    for (int i = 0; i < C::kStages && i < n_kv; ++i) issue_tile(i);
+    ok = __all_sync(FULL, mbar_wait_bounded(full_b, 0, kWaitLimitNs));
+    if (ok && lane == 0) issue_s(0);
+    for (int i = 0; ok && i < n_kv; ++i) {
+      if (i + 1 < n_kv) {
+        const int st = (i + 1) % C::kStages;
+        ok = __all_sync(FULL, mbar_wait_bounded(full_b + 8 * st, ((i + 1) / C::kStages) & 1, kWaitLimitNs));
+        if (!ok) break;
+        umma::fence_after();
+        if (lane == 0) issue_s(i + 1);
+      }
+      ok = __all_sync(FULL, mbar_wait_bounded(pready_b, i & 1, kWaitLimitNs));
+      if (!ok || *abort_flag) break;
+      umma::fence_after();
+      if (lane == 0) issue_o(i);
+      __syncwarp();
+      // Refill a released stage with tile jr + kStages.  With more than two
+      // stages it is the one P V(i-1) released (it has had a tile's time to
+      // complete), which keeps the loads kStages - 1 tiles ahead of S; with two
+      // stages S(i+1) needs tile i+2 next, so it is the stage P V(i) releases.
+      constexpr int kLag = C::kStages > 2 ? 1 : 0;
+      const int jr = i - kLag;
+      if (jr >= 0 && jr + C::kStages < n_kv) {
+        ok = __all_sync(FULL, mbar_wait_bounded(empty_b + 8 * (jr % C::kStages), (jr / C::kStages) & 1,
+                                                kWaitLimitNs));
+        if (!ok) break;
+        issue_tile(jr + C::kStages);
+      }
+    }
+    if (!ok) {
+      if (lane == 0) raise_error(PA_DEVERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+  } else {
+    // ================= softmax warps: one query row per thread =================
+    const int r = tid;  // TMEM lane = row
+    const bool real = r / G < ntok;
+    const int end_r = L - T + j0 + r / G + 1;  // p + 1
+    const int lo_r = real ? max(window_start(max(end_r, 0), p.window), 0) : ulo;
+    const int hi_r = real ? min(end_r, L) : uhi;
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
+    float m = -CUDART_INF_F, l = 0.f;
+    bool ok = true;
+    for (int i = 0; i < n_kv; ++i) {
+      ok = __all_sync(FULL, mbar_wait_bounded(sfull_b + 8 * (i & 1), (i >> 1) & 1, kWaitLimitNs));
+      if (!ok || *abort_flag) break;
+      umma::fence_after();
+      const int kt = kt0 + i * C::kTile;
+      float x[C::kTile];
+#pragma unroll
+      for (int c = 0; c < C::kTile / 16; ++c) {
+        float v[16];
+        umma::ld16(lane_base + C::kSCol + (i & 1) * C::kTile + c * 16, v);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) x[c * 16 + k] = v[k];
+      }
+      float mt = -CUDART_INF_F;
+#pragma unroll
+      for (int k = 0; k < C::kTile; ++k) {
+        float v = x[k] * qk_scale;
+        if (p.use_softcap) v = p.softcap * tanhf(v * p.inv_softcap) * kLog2e;
+        const int t = kt + k;
+        v = (t >= lo_r && t < hi_r) ? v : -CUDART_INF_F;
+        x[k] = v;
+        mt = fmaxf(mt, v);
+      }
+      // Lazy rescaling: keep the reference m while the tile's maximum exceeds
+      // it by at most 8 (log2 units): the weights stay <= 256 and the sum and
+      // output share the reference, so the result is exact; O is rescaled only
+      // when the reference moves.
+      const float mn = (m == -CUDART_INF_F || mt > m + 8.f) ? mt : m;
+      const float ref = mn == -CUDART_INF_F ? 0.f : mn;
+      const float alpha = exp2f(m - ref);
+      m = mn;
+      float psum = 0.f;
+      uint32_t pk[C::kTile / 2];
+#pragma unroll
+      for (int k = 0; k < C::kTile / 2; ++k) {
+        pk[k] = pack_bf16x2(exp2f(x[2 * k] - ref), exp2f(x[2 * k + 1] - ref));
+        psum += bf16_lo(pk[k]) + bf16_hi(pk[k]);
+      }
+      l = l * alpha + psum;
+      if (i > 0) {  // P V(i-1) must be done: it reads the P buffer, and O is rescaled below
+        ok = __all_sync(FULL, mbar_wait_bounded(odone_b, (i - 1) & 1, kWaitLimitNs));
+        if (!ok) break;
+        umma::fence_after();
+        if (__any_sync(FULL, alpha != 1.f)) {
+#pragma unroll 1
+          for (int c = 0; c < D / 16; ++c) {
+            float v[16];
+            umma::ld16(lane_base + C::kOCol + c * 16, v);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) v[k] *= alpha;
+            umma::st16(lane_base + C::kOCol + c * 16, v);
+          }
+        }
+      }
+      // P row r (64 bf16 = 8 chunks) in the canonical K-major SWIZZLE_128B layout.
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint32_t dst = p_s + r * 128 + ((c ^ (r & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pk[4 * c]), "r"(pk[4 * c + 1]),
+                     "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
+                     : "memory");
+      }
+      // V rows of this tile outside [ulo, uhi): zero (stale or canary data, P = 0 there).
+      if (kt < ulo || kt + C::kTile > uhi) {
+        const uint32_t vst = st_s + (i % C::kStages) * C::kStageBytes + C::kKBytes;
+        for (int idx = tid; idx < C::kTile * C::kPanels * 8; idx += C::kRows) {
+          const int row = idx / (C::kPanels * 8), rem = idx % (C::kPanels * 8);
+          const int t = kt + row;
+          if (t < ulo || t >= uhi) {
+            const uint32_t dst = vst + (rem >> 3) * C::kKVPanelBytes + row * 128 + ((rem & 7) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      umma::fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(pready_b);
+    }
+    // ---- epilogue: O / l to the output rows ---------------------------------------------
+    if (ok && !*abort_flag) ok = __all_sync(FULL, mbar_wait_bounded(odone_b, (n_kv - 1) & 1, kWaitLimitNs));
+    if (ok && !*abort_flag) {
+      umma::fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* orow =
+          static_cast<__nv_bfloat16*>(p.out) + ((row0 + r / G) * p.hq + (size_t)g * G + r % G) * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 16; ++c) {
+        float v[16];
+        umma::ld16(lane_base + C::kOCol + c * 16, v);
+        if (real) {
+          uint4 lo, hi;
+          lo.x = pack_bf16x2(v[0] * inv, v[1] * inv);
+          lo.y = pack_bf16x2(v[2] * inv, v[3] * inv);
+          lo.z = pack_bf16x2(v[4] * inv, v[5] * inv);
+          lo.w = pack_bf16x2(v[6] * inv, v[7] * inv);
+          hi.x = pack_bf16x2(v[8] * inv, v[9] * inv);
+          hi.y = pack_bf16x2(v[10] * inv, v[11] * inv);
+          hi.z = pack_bf16x2(v[12] * inv, v[13] * inv);
+          hi.w = pack_bf16x2(v[14] * inv, v[15] * inv);
+          reinterpret_cast<uint4*>(orow + c * 16)[0] = lo;
+          reinterpret_cast<uint4*>(orow + c * 16)[1] = hi;
+        }
+      }
+    } else if (lane == 0) {
+      raise_error(PA_DEVERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+  }
+  // Every tcgen05 access is complete (waited); free the tensor memory.
+  umma::fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    umma::fence_after();
+    umma::dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace pa

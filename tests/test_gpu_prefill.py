@@ -44,11 +44,11 @@ def _run(name, lengths, q_lens, window=None, softcap=None, append=True):
 def test_prefill_prompts_from_scratch(name):
     """Whole prompts: every context position is new (T_b = L_b), ragged lengths
     spanning several query tiles and a partial last tile."""
-    lengths = [1, 9, 64, 130, 257]
+    lengths = [1, 9, 64, 130, 257, 700]
     w, out, ref, (kc, vc), (kc_ref, vc_ref) = _run(name, lengths, lengths)
+    assert pa.device_errors() == 0
     assert torch.equal(bits(kc), bits(kc_ref)) and torch.equal(bits(vc), bits(vc_ref))
     assert_close(out, ref, torch.bfloat16, f"prefill {name}")
-    assert pa.device_errors() == 0
 
 
 @pytest.mark.parametrize("name", ["tinyllama_1b", "llama3_8b"])
