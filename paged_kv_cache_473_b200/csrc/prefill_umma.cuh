@@ -239,6 +239,9 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
     const int lo_r = real ? max(window_start(max(end_r, 0), p.window), 0) : ulo;
     const int hi_r = real ? min(end_r, L) : uhi;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
+    // Tiles that need no mask for any row of this warp: [w_lo, w_hi) is valid
+    // for all of them.
+    const int w_lo = __reduce_max_sync(FULL, lo_r), w_hi = __reduce_min_sync(FULL, hi_r);
     float m = -CUDART_INF_F, l = 0.f;
     bool ok = true;
     for (int i = 0; i < n_kv; ++i) {
@@ -247,23 +250,36 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
       umma::fence_after();
       const int kt = kt0 + i * C::kTile;
       float x[C::kTile];
+      {
+        uint32_t u[C::kTile / 16][16];
 #pragma unroll
-      for (int c = 0; c < C::kTile / 16; ++c) {
-        float v[16];
-        umma::ld16(lane_base + C::kSCol + (i & 1) * C::kTile + c * 16, v);
+        for (int c = 0; c < C::kTile / 16; ++c)
+          umma::ld16_nowait(lane_base + C::kSCol + (i & 1) * C::kTile + c * 16, u[c]);
+        umma::wait_ld();
 #pragma unroll
-        for (int k = 0; k < 16; ++k) x[c * 16 + k] = v[k];
+        for (int c = 0; c < C::kTile / 16; ++c)
+#pragma unroll
+          for (int k = 0; k < 16; ++k) x[c * 16 + k] = __uint_as_float(u[c][k]);
       }
+      // x becomes the log2-domain score (scaled, softcapped) in place; the
+      // masks apply only where some row of the warp needs them.
       float mt = -CUDART_INF_F;
+      const bool masked = kt < w_lo || kt + C::kTile > w_hi;
+      if (p.use_softcap) {
 #pragma unroll
-      for (int k = 0; k < C::kTile; ++k) {
-        float v = x[k] * qk_scale;
-        if (p.use_softcap) v = p.softcap * tanhf(v * p.inv_softcap) * kLog2e;
-        const int t = kt + k;
-        v = (t >= lo_r && t < hi_r) ? v : -CUDART_INF_F;
-        x[k] = v;
-        mt = fmaxf(mt, v);
+        for (int k = 0; k < C::kTile; ++k) x[k] = p.softcap * tanhf(x[k] * qk_scale * p.inv_softcap) * kLog2e;
       }
+      const float xs = p.use_softcap ? 1.f : qk_scale;  // scale still to apply to x
+      if (masked) {
+#pragma unroll
+        for (int k = 0; k < C::kTile; ++k) {
+          const int t = kt + k;
+          x[k] = (t >= lo_r && t < hi_r) ? x[k] : -CUDART_INF_F;
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < C::kTile; ++k) mt = fmaxf(mt, x[k]);
+      mt *= xs;  // xs > 0: the maximum of the scaled scores
       // Lazy rescaling: keep the reference m while the tile's maximum exceeds
       // it by at most 8 (log2 units): the weights stay <= 256 and the sum and
       // output share the reference, so the result is exact; O is rescaled only
@@ -272,14 +288,19 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
       const float ref = mn == -CUDART_INF_F ? 0.f : mn;
       const float alpha = exp2f(m - ref);
       m = mn;
-      float psum = 0.f;
+      // p = 2^(xs x - ref) (one FMA and one ex2 each); the row sum in four
+      // independent chains.
+      float ps[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t pk[C::kTile / 2];
 #pragma unroll
       for (int k = 0; k < C::kTile / 2; ++k) {
-        pk[k] = pack_bf16x2(exp2f(x[2 * k] - ref), exp2f(x[2 * k + 1] - ref));
-        psum += bf16_lo(pk[k]) + bf16_hi(pk[k]);
+        float e0, e1;
+        asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e0) : "f"(fmaf(x[2 * k], xs, -ref)));
+        asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e1) : "f"(fmaf(x[2 * k + 1], xs, -ref)));
+        ps[k & 3] += e0 + e1;
+        pk[k] = pack_bf16x2(e0, e1);
       }
-      l = l * alpha + psum;
+      l = l * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
       if (i > 0) {  // P V(i-1) must be done: it reads the P buffer, and O is rescaled below
         ok = __all_sync(FULL, mbar_wait_bounded(odone_b, (i - 1) & 1, kWaitLimitNs));
         if (!ok) break;
