@@ -215,6 +215,11 @@ cudaError_t launch_prefill_t(const DecodeParams& p, dim3 grid, cudaStream_t st) 
   static std::atomic<uint64_t> smem_done{0};
   cudaError_t e = set_smem(kern, Cfg::kSmemBytes, smem_done);
   if (e != cudaSuccess) return e;
+  // The whole shared-memory carveout, so that kMinBlocks CTAs fit per SM.
+  static std::once_flag carveout_once;
+  std::call_once(carveout_once, [&] {
+    (void)cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  });
   return launch_ex(kern, grid, dim3(Cfg::kThreads), Cfg::kSmemBytes, st, false, kmap, vmap, p);
 }
 

@@ -53,10 +53,15 @@ struct PrefillCfg {
   static constexpr int kOCol = 2 * kTile;        // O: columns [128, 128 + D)
   static constexpr int kTmemCols = (2 * kTile + D) <= 256 ? 256 : 512;
   static constexpr int kThreads = 160;           // 4 softmax warps + the TMA / MMA warp
+  // Register budget: two resident CTAs per SM for head_dim <= 128.  The bound
+  // is stated for 192 threads because registers are allotted to a CTA's warps
+  // in pairs (five warps take six warps' registers).
+  static constexpr int kBoundThreads = 192;
+  static constexpr int kMinBlocks = D <= 128 ? 2 : 1;
 };
 
 template <int D>
-__global__ void __launch_bounds__(PrefillCfg<D>::kThreads, 1)
+__global__ void __launch_bounds__(PrefillCfg<D>::kBoundThreads, PrefillCfg<D>::kMinBlocks)
     prefill_umma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                         const DecodeParams p) {
   using C = PrefillCfg<D>;
