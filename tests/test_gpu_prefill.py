@@ -87,3 +87,33 @@ def test_prefill_bad_offsets_are_reported_not_written():
     torch.cuda.synchronize()
     assert pa.device_errors() & pa.DEVERR_CONTEXT
     assert torch.all(out[10:] == 7.0)  # the malformed sequence's rows are untouched
+
+
+@pytest.mark.parametrize("name,lengths", [("llama3_8b", [1024] * 16), ("tinyllama_1b", [37, 2047, 512, 1300, 64, 999]),
+                                          ("gemma2_2b", [1024, 333, 700])])
+def test_prefill_full_size_sampled_rows(name, lengths):
+    """The measured prefill workload (16 prompts x 1024 tokens) and ragged long
+    prompts: sampled rows against the oracle (each row is a causal attention
+    over up to 2047 positions)."""
+    w = wl.WORKLOADS[name].replace(prefix_share=0.0)
+    b = wl.make_batch(w, lengths=lengths, device="cuda")
+    x = wl.make_prefill_inputs(b, lengths)
+    kc, vc = b.k_cache.clone(), b.v_cache.clone()
+    out = pa.prefill(x["q"], x["k_new"], x["v_new"], x["slot_mapping"], x["cu_q_lens"], kc, vc, b.block_tables,
+                     b.context_lens, w.scale, w.softcap, w.window, max_q_len=x["max_q_len"])
+    torch.cuda.synchronize()
+    assert pa.device_errors() == 0
+    cu = x["cu_q_lens"].tolist()
+    g = torch.Generator().manual_seed(17)
+    picks = []
+    for bi, L in enumerate(lengths):
+        for j in sorted(set([0, L - 1] + torch.randint(0, L, (4,), generator=g).tolist())):
+            picks.append((bi, j, int(torch.randint(0, w.num_q_heads, (1,), generator=g))))
+    # oracle: each picked row is a decode over its own prefix of the appended cache
+    kc_cpu, vc_cpu = kc.cpu(), vc.cpu()
+    tables, q = b.block_tables.cpu(), x["q"].cpu()
+    for bi, j, h in picks:
+        lens = torch.tensor([j + 1], dtype=torch.int32)
+        ref = oracle.decode(q[cu[bi] + j].unsqueeze(0), kc_cpu, vc_cpu, tables[bi:bi + 1], lens, w.scale, w.softcap,
+                            w.window, rows=[(0, h)])
+        assert_close(out[cu[bi] + j, h].unsqueeze(0), ref, torch.bfloat16, f"{name} prompt {bi} token {j} head {h}")
