@@ -730,9 +730,18 @@ bool multi_rows_path(int32_t batch, int32_t q_len, int32_t num_q_heads, int32_t 
 int32_t multi_partition(int32_t batch, int32_t q_len, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                         int32_t max_context_len, int32_t partition_tokens) {
   if (partition_tokens > 0) return partition_tokens;
-  return multi_rows_path(batch, q_len, num_q_heads, num_kv_heads, head_dim)
-             ? dynamic_partition(batch, num_kv_heads, max_context_len, head_dim)
-             : auto_partition(batch, num_kv_heads, max_context_len, 0);
+  if (!multi_rows_path(batch, q_len, num_q_heads, num_kv_heads, head_dim))
+    return auto_partition(batch, num_kv_heads, max_context_len, 0);
+  // The rows path writes T*G partial rows per item, twice the decode's at
+  // T*G = 16: at head_dim 128 512-token partitions keep the partials and the
+  // combine small (a sweep on B200: Llama-3 T=4, 0.76 -> 0.89 of HBM peak);
+  // halved, as for decode, while there are fewer items than resident warps.
+  const long long work = (long long)(batch > 0 ? batch : 1) * (num_kv_heads > 0 ? num_kv_heads : 1) *
+                         (max_context_len > 0 ? max_context_len : 1);
+  int P = head_dim <= 64 ? 256 : 512;
+  const int warps_per_sm = head_dim <= 64 ? 8 : 12;
+  while (P > 64 && work / P < (long long)warps_per_sm * 148) P >>= 1;
+  return P;
 }
 
 pa_status_t pa_decode_multi(const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
