@@ -87,24 +87,31 @@ struct Item {
   bool whole;      // the item is the sequence's only partition
 };
 
-// Log-sum-exp merge of the `n` partials [pb, pb + n) of unit (b, g) into the
-// normalised output rows of its G query heads:
+// In-kernel merges take at most this many partials per unit (the host merges
+// larger splits with the combine kernel).
+constexpr int kMaxMergeParts = 8;
+
+// Log-sum-exp merge of the `n` <= kMaxMergeParts partials [pb, pb + n) of unit
+// (b, g) into the normalised output rows of its G query heads:
 //   M = max_p m_p,  out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p
 // (m in the log2 domain, o unnormalised relative to m).  lph lanes per head (a
 // power of two), each covering D / lph dims in chunks of 16; the partials are
-// read through L2 (other SMs wrote them).
+// read through L2 (other SMs wrote them).  The merge runs after the unit's
+// last partition, on the critical path of the call's tail, so every load of a
+// chunk is issued before any is used: one L2 round trip instead of one per
+// few partials (kBatch partials at a time where registers are tight).
 template <int D>
 __device__ __forceinline__ void merge_unit(const DecodeParams& p, int b, int g, int pb, int n, int lane) {
-  constexpr uint32_t FULL = 0xffffffffu;
+  constexpr int kBatch = D == 128 ? 4 : kMaxMergeParts;  // head_dim 128 runs with a 170-register cap
   const int G = p.group;
   const int lph = min(G == 1 ? 32 : G == 2 ? 16 : G <= 4 ? 8 : 4, D / 16);
   const int h = lane / lph, s = lane & (lph - 1);
   const bool active = h < G;
   const size_t row = (size_t)b * p.hq + (size_t)g * G + (active ? h : 0);
   const float2* ml = reinterpret_cast<const float2*>(p.ws_ml) + row * p.max_parts + pb;
-  float M = -CUDART_INF_F;
-  for (int i = s; i < n; i += lph) M = fmaxf(M, __ldcg(ml + i).x);
-  for (int off = 1; off < lph; off <<= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, off));
+  float2 mlv[kMaxMergeParts];
+#pragma unroll
+  for (int i = 0; i < kMaxMergeParts; ++i) mlv[i] = i < n ? __ldcg(ml + i) : make_float2(-CUDART_INF_F, 0.f);
   const int E = D / lph;
   const float* po = p.ws_o + (row * p.max_parts + pb) * D + s * E;
   __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row * D + s * E;
@@ -113,19 +120,31 @@ __device__ __forceinline__ void merge_unit(const DecodeParams& p, int b, int g, 
 #pragma unroll
     for (int k = 0; k < 16; ++k) acc[k] = 0.f;
     float den = 0.f;
-#pragma unroll 4
-    for (int i = 0; i < n; ++i) {
-      const float2 v = __ldcg(ml + i);
-      const float w = v.x == -CUDART_INF_F ? 0.f : exp2f(v.x - M);
-      den = fmaf(w, v.y, den);
-      const float4* src = reinterpret_cast<const float4*>(po + (size_t)i * D + c0);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float4 x = __ldcg(src + k);
-        acc[4 * k + 0] = fmaf(w, x.x, acc[4 * k + 0]);
-        acc[4 * k + 1] = fmaf(w, x.y, acc[4 * k + 1]);
-        acc[4 * k + 2] = fmaf(w, x.z, acc[4 * k + 2]);
-        acc[4 * k + 3] = fmaf(w, x.w, acc[4 * k + 3]);
+    for (int i0 = 0; i0 < kMaxMergeParts; i0 += kBatch) {
+      if (i0 >= n) break;
+      float4 x[kBatch][4];
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        const float4* src = reinterpret_cast<const float4*>(po + (size_t)(i0 + i) * D + c0);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) x[i][k] = i0 + i < n ? __ldcg(src + k) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      float M = -CUDART_INF_F;
+#pragma unroll
+      for (int i = 0; i < kMaxMergeParts; ++i) M = fmaxf(M, mlv[i].x);
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        const float2 v = mlv[i0 + i];
+        const float w = v.x == -CUDART_INF_F ? 0.f : exp2f(v.x - M);  // empty or absent partial: weight 0
+        den = fmaf(w, v.y, den);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          acc[4 * k + 0] = fmaf(w, x[i][k].x, acc[4 * k + 0]);
+          acc[4 * k + 1] = fmaf(w, x[i][k].y, acc[4 * k + 1]);
+          acc[4 * k + 2] = fmaf(w, x[i][k].z, acc[4 * k + 2]);
+          acc[4 * k + 3] = fmaf(w, x[i][k].w, acc[4 * k + 3]);
+        }
       }
     }
     if (active) {
@@ -260,13 +279,17 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
   // only when its item is needed, so no warp waits on the counter at launch.
   const int n_static = p.static_items;
   const int claim_base = n_static * W;
+  // Claims are needed only when there are more items than the warps' fixed
+  // ones; otherwise no warp touches the counter and no CTA counts out, so a
+  // CTA ends with its last warp.
+  const bool claims = T > claim_base;
   int t_cur = wg;       // item being computed
   int t_next = W + wg;  // item after it, valid when next_known
   bool next_known = n_static >= 2;
   if (t_cur < T) {  // else this warp has no item; it still joins the final barrier
     int t_claim = 0;       // lane 0: the claim in flight (for t_next when !next_known, else the item after)
     bool pending = false;  // a claim is in flight (warp-uniform)
-    if (n_static < 2 || t_next < T) {
+    if (claims && (n_static < 2 || t_next < T)) {
       if (lane == 0) t_claim = (n_static < 2 ? W : claim_base) + atomicAdd(p.queue, 1);
       pending = true;
     }
@@ -276,7 +299,7 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
       t_next = pending ? __shfl_sync(FULL, t_claim, 0) : T;
       next_known = true;
       pending = false;
-      if (t_next < T) {
+      if (claims && t_next < T) {
         if (lane == 0) t_claim = claim_base + atomicAdd(p.queue, 1);
         pending = true;
       }
@@ -414,14 +437,15 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
           }
         }
         if (p.merge_in_kernel) {
-          // Publish the partial, then count it; the unit's last partial merges them all.
-          __threadfence();
+          // Publish the partial, then count it (release); the unit's last
+          // partial merges them all (acquire).
+          fence_acq_rel_gpu();
           __syncwarp();
           int* cnt = p.unit_count + (size_t)ci.b * Hkv + ci.g;
           int last = 0;
           if (lane == 0) last = atomicAdd(cnt, 1) == ci.parts - 1;
           if (__shfl_sync(FULL, last, 0)) {
-            __threadfence();
+            fence_acq_rel_gpu();
             merge_unit<D>(p, ci.b, ci.g, ci.pb, ci.parts, lane);
             if (lane == 0) *cnt = 0;  // every partial of the unit has arrived: ready for the next call
           }
@@ -462,12 +486,14 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
 
   // Every claim of this CTA's warps has returned: count the CTA out; the last
   // CTA returns the work counter (and this count) to zero for the next call.
-  __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    if (atomicAdd(p.queue + 1, 1) == (int)gridDim.x - 1) {
-      p.queue[0] = 0;
-      p.queue[1] = 0;
+  if (claims) {
+    __syncthreads();
+    if (tid == 0) {
+      __threadfence();
+      if (atomicAdd(p.queue + 1, 1) == (int)gridDim.x - 1) {
+        p.queue[0] = 0;
+        p.queue[1] = 0;
+      }
     }
   }
   // In a cascade this grid is a programmatic dependent of the prefix pass

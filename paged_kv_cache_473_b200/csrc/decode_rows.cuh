@@ -131,13 +131,17 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
 
   const int n_static = p.static_items;
   const int claim_base = n_static * W;
+  // Claims are needed only when there are more items than the warps' fixed
+  // ones; otherwise no warp touches the counter and no CTA counts out, so a
+  // CTA ends with its last warp.
+  const bool claims = T_items > claim_base;
   int t_cur = wg;
   int t_next = W + wg;
   bool next_known = n_static >= 2;
   if (t_cur < T_items) {
     int t_claim = 0;
     bool pending = false;
-    if (n_static < 2 || t_next < T_items) {
+    if (claims && (n_static < 2 || t_next < T_items)) {
       if (lane == 0) t_claim = (n_static < 2 ? W : claim_base) + atomicAdd(p.queue, 1);
       pending = true;
     }
@@ -146,7 +150,7 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
       t_next = pending ? __shfl_sync(FULL, t_claim, 0) : T_items;
       next_known = true;
       pending = false;
-      if (t_next < T_items) {
+      if (claims && t_next < T_items) {
         if (lane == 0) t_claim = claim_base + atomicAdd(p.queue, 1);
         pending = true;
       }
@@ -270,13 +274,16 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
     }
   }  // t_cur < T_items
 
-  // The last CTA to finish returns the work counter to zero.
-  __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    if (atomicAdd(p.queue + 1, 1) == (int)gridDim.x - 1) {
-      p.queue[0] = 0;
-      p.queue[1] = 0;
+  // The last CTA to finish returns the work counter to zero (when any warp
+  // claimed from it).
+  if (claims) {
+    __syncthreads();
+    if (tid == 0) {
+      __threadfence();
+      if (atomicAdd(p.queue + 1, 1) == (int)gridDim.x - 1) {
+        p.queue[0] = 0;
+        p.queue[1] = 0;
+      }
     }
   }
 }

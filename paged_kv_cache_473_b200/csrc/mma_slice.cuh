@@ -99,8 +99,11 @@ __device__ __forceinline__ void load_q_frags(uint32_t (&qf)[D / 16][2], const __
 // with 2-D TMA tile loads, one 64-column panel per instruction.  The warp
 // calls this together: lane 0 arms the stage's barrier with the byte count and
 // lanes 0 .. 2*D/64-1 each issue one panel (issuing from several lanes at once
-// costs about as much as one TMA instruction from one lane).  y < 0 (a bad
-// block id) arms the barrier with no bytes and raises PA_DEVERR_BLOCK.
+// costs about as much as one TMA instruction from one lane).  The loads carry
+// an evict-first L2 hint: a decode reads each slice once (measured on B200:
+// Llama-3-8B step 0.974 -> 1.00 and Gemma-2-2B 0.82 -> 0.87 of the HBM copy
+// rate, the partials and tables staying in L2).  y < 0 (a bad block id) arms
+// the barrier with no bytes and raises PA_DEVERR_BLOCK.
 template <int D>
 __device__ __forceinline__ void issue_slice(uint32_t dst, uint32_t bar, const CUtensorMap* kmap,
                                             const CUtensorMap* vmap, int y, int lane) {
@@ -117,7 +120,8 @@ __device__ __forceinline__ void issue_slice(uint32_t dst, uint32_t bar, const CU
   if (lane < 2 * kPanels) {
     const int pn = lane % kPanels;
     const bool is_v = lane >= kPanels;
-    tma_load_2d(dst + (is_v ? SliceBytes<D>::kSlice : 0) + pn * kPanelBytes, is_v ? vmap : kmap, bar, pn * 64, y);
+    tma_load_2d_hint(dst + (is_v ? SliceBytes<D>::kSlice : 0) + pn * kPanelBytes, is_v ? vmap : kmap, bar, pn * 64,
+                     y, l2_policy_evict_first());
   }
 }
 

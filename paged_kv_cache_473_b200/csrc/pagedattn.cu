@@ -386,7 +386,7 @@ cudaError_t launch_dynamic_t(DecodeParams& p, cudaStream_t st, bool pdl, bool al
   if (occ < 1) return cudaErrorInvalidConfiguration;
   const int grid = occ * sm_count();
   const long long unit_bound = (long long)p.batch * p.hkv * p.max_parts;
-  p.merge_in_kernel = (allow_merge && p.max_parts <= 8 && unit_bound <= 2LL * grid * NW) ? 1 : 0;
+  p.merge_in_kernel = (allow_merge && p.max_parts <= pa::kMaxMergeParts && unit_bound <= 2LL * grid * NW) ? 1 : 0;
   p.static_items = 2;
   return launch_ex(kern, dim3(grid), dim3(Cfg::kThreads), smem, st, pdl, kmap, vmap, p);
 }

@@ -455,6 +455,33 @@ def test_dynamic_schedule_counters_return_to_zero():
     assert pa.device_errors() == 0
 
 
+COUNTER_BYTES = 256 * 1024  # the workspace's fixed counter region
+
+
+@pytest.mark.parametrize("name,kw", [("tinyllama_1b", dict(batch=24)),  # fixed items cover the work: no claims
+                                     ("llama3_8b", dict(batch=64))])    # more items than 2 per warp: claims
+def test_dynamic_schedule_counter_region_reads_zero_after_each_call(name, kw):
+    """Whether or not warps claim items from the work counter, the workspace's
+    counter region is all zero when the call ends (the next call relies on it),
+    with the fused append and without."""
+    w = wl.WORKLOADS[name]
+    bc = wl.make_batch(w, prefilled=False, **kw)
+    b = to_dev(bc)
+    need = pa.decode_splitk_workspace_size(bc.q.shape[0], w.num_q_heads, w.head_dim, b.max_context_len, 0,
+                                           w.num_kv_heads)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    kc, vc = b.k_cache.clone(), b.v_cache.clone()
+    for _ in range(2):
+        out = pa.decode_step(b.q, b.k_new, b.v_new, kc, vc, b.block_tables, b.context_lens, w.scale, w.softcap,
+                             w.window, split=True, max_context_len=b.max_context_len, partition_tokens=0,
+                             workspace=ws)
+        torch.cuda.synchronize()
+        assert int(ws[:COUNTER_BYTES].view(torch.int32).abs().sum()) == 0
+    ref, _, _ = oracle_step(bc)
+    assert_close(out, ref, torch.bfloat16, f"{name} step")
+    assert pa.device_errors() == 0
+
+
 @pytest.mark.parametrize("window", [1, 100, 1000])
 def test_dynamic_schedule_window(window):
     w, b_cpu, b = _reduced("tinyllama_1b", prefilled=True)
