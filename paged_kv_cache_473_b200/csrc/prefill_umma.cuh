@@ -4,19 +4,26 @@
 // One CTA takes 128 query rows of one sequence and kv head: TQ = 128 / G query
 // tokens x G heads, row r = (token j0 + r / G, head r % G), the token at
 // position p = L - T + j attending the positions [s0(p + 1), p] of its
-// sequence (causal, sliding window).  The K/V of the union of those ranges
-// stream through a 2-stage ring of 64-token tiles (2-D TMA boxes of 16 rows
-// per physical block, SWIZZLE_128B, which is the canonical K-major layout for
-// K and the MN-major layout for V).  Per tile:
+// sequence (causal, sliding window).  The K and V of the union of those ranges
+// stream through two rings of 64-token tiles (2-D TMA boxes of 16 rows per
+// physical block, SWIZZLE_128B, which is the canonical K-major layout for K
+// and the MN-major layout for V).  The rings are separate so that a K stage is
+// refilled as soon as its S = Q K^T is done and a V stage as soon as its P V
+// is: K runs two tiles ahead of S without waiting for the P V of the tile
+// before.  Per tile:
 //   S = Q K^T        UMMA M=128, N=64, K=D     into one of two TMEM S buffers
 //   softmax          warps 0-3: each thread owns one query row (its TMEM lane):
 //                    tcgen05.ld of its 64 scores, scale / softcap / masks,
 //                    online max and sum, O rescale in TMEM when the max moved,
 //                    P (bf16) to shared memory in the canonical K-major layout
 //   O += P V         UMMA M=128, N=D, K=64                into TMEM
-// Warp 4 issues the TMA loads (one box per lane) and, from lane 0, the MMAs;
-// it issues S for the next tile before waiting for this tile's P, so the
-// tensor core computes S(i+1) while the softmax warps work on S(i).  Completion
+// Warp 5 issues the TMA loads (one box per lane), refilling each stage as soon
+// as the MMA that reads it is done.  Warp 4 issues the MMAs from lane 0: S for
+// the next tile before waiting for this tile's P, so the tensor core computes
+// S(i+1) while the softmax warps work on S(i).  (A per-tile timeline of the
+// version with one K+V ring and one warp for loads and MMAs, on B200: the
+// softmax warps waited 1-1.6 us per tile for S, whose K tile was loaded only
+// after the previous P V had freed the stage.)  Completion
 // travels through mbarriers (TMA bytes, tcgen05.commit); every wait is
 // bounded.  V rows of a tile outside the union range are zeroed in shared
 // memory before P V (P is 0 there, and a NaN canary would still poison it).
@@ -37,25 +44,24 @@ struct PrefillCfg {
   static constexpr int kQPanelBytes = kRows * 128;
   static constexpr int kKVPanelBytes = kTile * 128;
   static constexpr int kKBytes = kPanels * kKVPanelBytes;
-  static constexpr int kStageBytes = 2 * kKBytes;  // K then V
+  static constexpr int kStageBytes = 2 * kKBytes;  // a K stage then a V stage (separate rings)
   static constexpr int kPBytes = kRows * 128;      // 128 rows x 64 bf16
   static constexpr int kQOff = 0;
   static constexpr int kStageOff = kPanels * kQPanelBytes;
   static constexpr int kPOff = kStageOff + kStages * kStageBytes;
   static constexpr int kBarOff = kPOff + kPBytes;
+  static constexpr int kBarBytes = 256;
   // Exactly the layout plus the barrier area (the dynamic shared-memory base is
   // 1024-byte aligned; the kernel checks it), and at least 80 KB so that no more
   // CTAs share an SM than its 512 tensor-memory columns hold (kTmemCols each):
   // two CTAs per SM for head_dim 64 and 128, one for 256.
-  static constexpr int kSmemBytes = (kBarOff + 128) > 80 * 1024 ? (kBarOff + 128) : 80 * 1024;
-  static_assert(16 * kStages + 40 <= 128, "barrier area");
+  static constexpr int kSmemBytes = (kBarOff + kBarBytes) > 80 * 1024 ? (kBarOff + kBarBytes) : 80 * 1024;
+  static_assert(32 * kStages + 48 <= kBarBytes, "barrier area");
   static constexpr int kSCol = 0;                // two S buffers: columns [0, 64) and [64, 128)
   static constexpr int kOCol = 2 * kTile;        // O: columns [128, 128 + D)
   static constexpr int kTmemCols = (2 * kTile + D) <= 256 ? 256 : 512;
-  static constexpr int kThreads = 160;           // 4 softmax warps + the TMA / MMA warp
-  // Register budget: two resident CTAs per SM for head_dim <= 128.  The bound
-  // is stated for 192 threads because registers are allotted to a CTA's warps
-  // in pairs (five warps take six warps' registers).
+  static constexpr int kThreads = 192;           // 4 softmax warps, the MMA warp, the TMA warp
+  // Register budget: two resident CTAs per SM for head_dim <= 128.
   static constexpr int kBoundThreads = 192;
   static constexpr int kMinBlocks = D <= 128 ? 2 : 1;
 };
@@ -103,22 +109,27 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kBoundThreads, PrefillCfg<D>::k
   const uint32_t s_base = smem_addr(smem);
   const uint32_t q_s = s_base + C::kQOff, st_s = s_base + C::kStageOff, p_s = s_base + C::kPOff;
   const uint32_t bar = s_base + C::kBarOff;
-  // Barrier area: full[kStages], empty[kStages], sfull[2], pready, odone, the
-  // TMEM address slot and the abort flag (at most 16*4 + 40 bytes of the 128).
-  const uint32_t full_b = bar, empty_b = bar + 8 * C::kStages, sfull_b = bar + 16 * C::kStages;
-  const uint32_t pready_b = sfull_b + 16, odone_b = sfull_b + 24;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + 16 * C::kStages + 32);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kBarOff + 16 * C::kStages + 36);
+  // Barrier area: kfull/kempty/vfull/vempty[kStages] (the two rings), sfull[2],
+  // pready, odone, the TMEM address slot and the abort flag.
+  const uint32_t kfull_b = bar, kempty_b = bar + 8 * C::kStages;
+  const uint32_t vfull_b = bar + 16 * C::kStages, vempty_b = bar + 24 * C::kStages;
+  const uint32_t sfull_b = bar + 32 * C::kStages;
+  const uint32_t pready_b = sfull_b + 16, odone_b = sfull_b + 24, drain_b = sfull_b + 32;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + 32 * C::kStages + 40);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kBarOff + 32 * C::kStages + 44);
 
   if (tid == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(full_b + 8 * s, 1);
-      mbar_init(empty_b + 8 * s, 1);
+      mbar_init(kfull_b + 8 * s, 1);
+      mbar_init(kempty_b + 8 * s, 1);
+      mbar_init(vfull_b + 8 * s, 1);
+      mbar_init(vempty_b + 8 * s, 1);
     }
     mbar_init(sfull_b, 1);
     mbar_init(sfull_b + 8, 1);
     mbar_init(pready_b, 4);
     mbar_init(odone_b, 1);
+    mbar_init(drain_b, 1);
     *abort_flag = 0;
     mbar_init_fence();
     prefetch_tensormap(&kmap);
@@ -148,18 +159,23 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kBoundThreads, PrefillCfg<D>::k
   const float qk_scale = p.use_softcap ? p.scale : p.scale * kLog2e;
   const int32_t* table = p.block_tables + (size_t)b * p.max_blocks;
 
-  if (warp == 4) {
-    // ================= TMA producer and MMA issuer =================
-    // Tile i: one 2-D box per lane (slice s = lane / (2*panels), K or V, panel).
-    auto issue_tile = [&](int i) {
+  // Wait for completion number `use` of a barrier (completions alternate parity).
+  auto wait_use = [&](uint32_t b, int use) { return __all_sync(FULL, mbar_wait_bounded(b, use & 1, kWaitLimitNs)); };
+  if (warp == 5) {
+    // ================= TMA producer =================
+    // K (kv = 0) or V (kv = 1) of tile i into its ring's stage i % kStages:
+    // one 2-D box per lane (slice s = lane / panels, panel).
+    int issued[2] = {0, 0};
+    auto issue_kv = [&](int i, int kv) {
       const int stage = i % C::kStages;
+      const uint32_t full = (kv ? vfull_b : kfull_b) + 8 * stage;
       const int kt = kt0 + i * C::kTile;
       const int box = lane;
-      const int s = box / (2 * C::kPanels), kv = (box / C::kPanels) & 1, pn = box % C::kPanels;
+      const int s = box / C::kPanels, pn = box % C::kPanels;
       const int t = kt + s * kSliceTokens;
       bool valid = false;
       int y = -1;
-      if (box < 8 * C::kPanels && t + kSliceTokens > ulo && t < uhi) {
+      if (box < 4 * C::kPanels && t + kSliceTokens > ulo && t < uhi) {
         const int phys = table[t >> p.log2_bs];
         if (phys >= 0 && phys < p.num_blocks) {
           valid = true;
@@ -170,18 +186,51 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kBoundThreads, PrefillCfg<D>::k
       }
       const uint32_t nvalid = __popc(__ballot_sync(FULL, valid));
       if (lane == 0) {
-        if (nvalid) mbar_arrive_expect_tx(full_b + 8 * stage, nvalid * kSliceTokens * 128);
-        else mbar_arrive(full_b + 8 * stage);
+        if (nvalid) mbar_arrive_expect_tx(full, nvalid * kSliceTokens * 128);
+        else mbar_arrive(full);
       }
       __syncwarp();
       if (valid) {
         const uint32_t dst = st_s + stage * C::kStageBytes + kv * C::kKBytes + pn * C::kKVPanelBytes + s * kSliceTokens * 128;
-        tma_load_2d(dst, kv ? &vmap : &kmap, full_b + 8 * stage, pn * 64, y);
+        tma_load_2d(dst, kv ? &vmap : &kmap, full, pn * 64, y);
       }
+      issued[kv] = i + 1;
     };
+    // Refill order K(j + 1), V(j): a K stage frees when its S is done, a V
+    // stage when its P V is, and S(j + 1 - kStages) is issued before
+    // P V(j - kStages), so the waits come in completion order.
+    auto refill = [&](int j, int kv) {  // tile j >= kStages into the stage tile j - kStages used
+      const int u = j - C::kStages;
+      if (!wait_use((kv ? vempty_b : kempty_b) + 8 * (u % C::kStages), u / C::kStages)) return false;
+      issue_kv(j, kv);
+      return true;
+    };
+    bool ok = true;
+    for (int i = 0; i < C::kStages && i < n_kv; ++i) issue_kv(i, 0);
+    for (int i = 0; i < C::kStages && i < n_kv; ++i) issue_kv(i, 1);
+    if (C::kStages < n_kv) ok = refill(C::kStages, 0);
+    for (int j = C::kStages; ok && j < n_kv; ++j) {
+      if (*abort_flag) break;
+      if (j + 1 < n_kv) ok = refill(j + 1, 0);
+      if (ok) ok = refill(j, 1);
+    }
+    if (!ok) {
+      if (lane == 0) raise_error(PA_DEVERR_TIMEOUT);
+      *abort_flag = 1;
+    }
+    if (!ok || *abort_flag) {
+      // Before the CTA releases its shared memory: give the last loads of each
+      // ring a bounded time to land (earlier ones have, their stages were reused).
+      for (int kv = 0; kv < 2; ++kv)
+        for (int j = max(issued[kv] - C::kStages, 0); j < issued[kv]; ++j)
+          (void)mbar_wait_bounded((kv ? vfull_b : kfull_b) + 8 * (j % C::kStages), (j / C::kStages) & 1,
+                                  kDrainLimitNs);
+    }
+  } else if (warp == 4) {
+    // ================= MMA issuer (lane 0) =================
     const uint32_t idesc_s = umma::idesc_bf16(128, C::kTile, 0, 0);
     const uint32_t idesc_o = umma::idesc_bf16(128, D, 0, 1);
-    auto issue_s = [&](int i) {  // lane 0: S(i) = Q K(i)^T into buffer i % 2
+    auto issue_s = [&](int i) {  // S(i) = Q K(i)^T into buffer i % 2
       const uint32_t kst = st_s + (i % C::kStages) * C::kStageBytes;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
@@ -190,8 +239,9 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kBoundThreads, PrefillCfg<D>::k
         umma::mma_f16(tmem + C::kSCol + (i & 1) * C::kTile, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
       }
       umma::commit(sfull_b + 8 * (i & 1));
+      umma::commit(kempty_b + 8 * (i % C::kStages));
     };
-    auto issue_o = [&](int i) {  // lane 0: O += P V(i)
+    auto issue_o = [&](int i) {  // O += P V(i)
       const uint32_t vst = st_s + (i % C::kStages) * C::kStageBytes + C::kKBytes;
 #pragma unroll
       for (int k = 0; k < C::kTile / 16; ++k) {
@@ -200,44 +250,35 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kBoundThreads, PrefillCfg<D>::k
         umma::mma_f16(tmem + C::kOCol, ad, bd, idesc_o, (i > 0 || k > 0) ? 1u : 0u);
       }
       umma::commit(odone_b);
-      umma::commit(empty_b + 8 * (i % C::kStages));
+      umma::commit(vempty_b + 8 * (i % C::kStages));
     };
-    bool ok = true;
-    for (int i = 0; i < C::kStages && i < n_kv; ++i) issue_tile(i);
-    ok = __all_sync(FULL, mbar_wait_bounded(full_b, 0, kWaitLimitNs));
-    if (ok && lane == 0) issue_s(0);
+    auto s_when_ready = [&](int j) {
+      if (!wait_use(kfull_b + 8 * (j % C::kStages), j / C::kStages)) return false;
+      umma::fence_after();
+      if (lane == 0) issue_s(j);
+      __syncwarp();
+      return true;
+    };
+    bool ok = s_when_ready(0);
     for (int i = 0; ok && i < n_kv; ++i) {
-      if (i + 1 < n_kv) {
-        const int st = (i + 1) % C::kStages;
-        ok = __all_sync(FULL, mbar_wait_bounded(full_b + 8 * st, ((i + 1) / C::kStages) & 1, kWaitLimitNs));
-        if (!ok) break;
-        umma::fence_after();
-        if (lane == 0) issue_s(i + 1);
-      }
-      ok = __all_sync(FULL, mbar_wait_bounded(pready_b, i & 1, kWaitLimitNs));
+      if (i + 1 < n_kv && !(ok = s_when_ready(i + 1))) break;
+      ok = wait_use(pready_b, i);
       if (!ok || *abort_flag) break;
+      if (!(ok = wait_use(vfull_b + 8 * (i % C::kStages), i / C::kStages))) break;
       umma::fence_after();
       if (lane == 0) issue_o(i);
       __syncwarp();
-      // Refill a released stage with tile jr + kStages.  With more than two
-      // stages it is the one P V(i-1) released (it has had a tile's time to
-      // complete), which keeps the loads kStages - 1 tiles ahead of S; with two
-      // stages S(i+1) needs tile i+2 next, so it is the stage P V(i) releases.
-      constexpr int kLag = C::kStages > 2 ? 1 : 0;
-      const int jr = i - kLag;
-      if (jr >= 0 && jr + C::kStages < n_kv) {
-        ok = __all_sync(FULL, mbar_wait_bounded(empty_b + 8 * (jr % C::kStages), (jr / C::kStages) & 1,
-                                                kWaitLimitNs));
-        if (!ok) break;
-        issue_tile(jr + C::kStages);
-      }
     }
     if (!ok) {
       if (lane == 0) raise_error(PA_DEVERR_TIMEOUT);
       *abort_flag = 1;
     }
+    if (!ok || *abort_flag) {  // the MMAs issued get a bounded time to finish before TMEM is freed
+      if (lane == 0) umma::commit(drain_b);
+      (void)mbar_wait_bounded(drain_b, 0, kDrainLimitNs);
+    }
   } else {
-    // ================= softmax warps: one query row per thread =================
+    // ================= softmax warps 0-3: one query row per thread =================
     const int r = tid;  // TMEM lane = row
     const bool real = r / G < ntok;
     const int end_r = L - T + j0 + r / G + 1;  // p + 1
@@ -329,8 +370,11 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kBoundThreads, PrefillCfg<D>::k
                      "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
                      : "memory");
       }
-      // V rows of this tile outside [ulo, uhi): zero (stale or canary data, P = 0 there).
+      // V rows of this tile outside [ulo, uhi): zero (stale or canary data, P = 0 there),
+      // once V(i) has landed.
       if (kt < ulo || kt + C::kTile > uhi) {
+        ok = __all_sync(FULL, mbar_wait_bounded(vfull_b + 8 * (i % C::kStages), (i / C::kStages) & 1, kWaitLimitNs));
+        if (!ok) break;
         const uint32_t vst = st_s + (i % C::kStages) * C::kStageBytes + C::kKBytes;
         for (int idx = tid; idx < C::kTile * C::kPanels * 8; idx += C::kRows) {
           const int row = idx / (C::kPanels * 8), rem = idx % (C::kPanels * 8);
