@@ -15,8 +15,9 @@
 //   softmax          warps 0-3: each thread owns one query row (its TMEM lane):
 //                    tcgen05.ld of its 64 scores, scale / softcap / masks,
 //                    online max and sum, O rescale in TMEM when the max moved,
-//                    P (bf16) to shared memory in the canonical K-major layout
-//   O += P V         UMMA M=128, N=D, K=64                into TMEM
+//                    P (bf16) back into the TMEM columns its S came from
+//   O += P V         UMMA M=128, N=D, K=64, A (P) from TMEM     into TMEM
+// P never goes through shared memory, which leaves room for a third K stage.
 // Warp 5 issues the TMA loads (one box per lane), refilling each stage as soon
 // as the MMA that reads it is done.  Warp 4 issues the MMAs from lane 0: S for
 // the next tile before waiting for this tile's P, so the tensor core computes
@@ -39,24 +40,23 @@ template <int D>
 struct PrefillCfg {
   static constexpr int kPanels = D / 64;         // 64-element (128-byte) column panels
   static constexpr int kTile = 64;               // K/V tokens per stage
-  static constexpr int kStages = D <= 64 ? 4 : 2;
+  static constexpr int kKStages = D <= 64 ? 4 : 3;  // K ring
+  static constexpr int kVStages = D <= 64 ? 4 : 2;  // V ring
   static constexpr int kRows = 128;              // query rows per CTA (UMMA M)
   static constexpr int kQPanelBytes = kRows * 128;
   static constexpr int kKVPanelBytes = kTile * 128;
   static constexpr int kKBytes = kPanels * kKVPanelBytes;
-  static constexpr int kStageBytes = 2 * kKBytes;  // a K stage then a V stage (separate rings)
-  static constexpr int kPBytes = kRows * 128;      // 128 rows x 64 bf16
   static constexpr int kQOff = 0;
-  static constexpr int kStageOff = kPanels * kQPanelBytes;
-  static constexpr int kPOff = kStageOff + kStages * kStageBytes;
-  static constexpr int kBarOff = kPOff + kPBytes;
+  static constexpr int kKOff = kPanels * kQPanelBytes;
+  static constexpr int kVOff = kKOff + kKStages * kKBytes;
+  static constexpr int kBarOff = kVOff + kVStages * kKBytes;
   static constexpr int kBarBytes = 256;
   // Exactly the layout plus the barrier area (the dynamic shared-memory base is
   // 1024-byte aligned; the kernel checks it), and at least 80 KB so that no more
   // CTAs share an SM than its 512 tensor-memory columns hold (kTmemCols each):
   // two CTAs per SM for head_dim 64 and 128, one for 256.
   static constexpr int kSmemBytes = (kBarOff + kBarBytes) > 80 * 1024 ? (kBarOff + kBarBytes) : 80 * 1024;
-  static_assert(32 * kStages + 48 <= kBarBytes, "barrier area");
+  static_assert(16 * (kKStages + kVStages) + 48 <= kBarBytes, "barrier area");
   static constexpr int kSCol = 0;                // two S buffers: columns [0, 64) and [64, 128)
   static constexpr int kOCol = 2 * kTile;        // O: columns [128, 128 + D)
   static constexpr int kTmemCols = (2 * kTile + D) <= 256 ? 256 : 512;
@@ -107,21 +107,24 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kBoundThreads, PrefillCfg<D>::k
   const int n_kv = (uhi - kt0 + C::kTile - 1) / C::kTile;
 
   const uint32_t s_base = smem_addr(smem);
-  const uint32_t q_s = s_base + C::kQOff, st_s = s_base + C::kStageOff, p_s = s_base + C::kPOff;
+  const uint32_t q_s = s_base + C::kQOff, k_s = s_base + C::kKOff, v_s = s_base + C::kVOff;
   const uint32_t bar = s_base + C::kBarOff;
-  // Barrier area: kfull/kempty/vfull/vempty[kStages] (the two rings), sfull[2],
+  // Barrier area: kfull/kempty[kKStages], vfull/vempty[kVStages], sfull[2],
   // pready, odone, the TMEM address slot and the abort flag.
-  const uint32_t kfull_b = bar, kempty_b = bar + 8 * C::kStages;
-  const uint32_t vfull_b = bar + 16 * C::kStages, vempty_b = bar + 24 * C::kStages;
-  const uint32_t sfull_b = bar + 32 * C::kStages;
+  constexpr int NK = C::kKStages, NV = C::kVStages;
+  const uint32_t kfull_b = bar, kempty_b = bar + 8 * NK;
+  const uint32_t vfull_b = bar + 16 * NK, vempty_b = bar + 16 * NK + 8 * NV;
+  const uint32_t sfull_b = bar + 16 * (NK + NV);
   const uint32_t pready_b = sfull_b + 16, odone_b = sfull_b + 24, drain_b = sfull_b + 32;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + 32 * C::kStages + 40);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kBarOff + 32 * C::kStages + 44);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + 16 * (NK + NV) + 40);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kBarOff + 16 * (NK + NV) + 44);
 
   if (tid == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
+    for (int s = 0; s < NK; ++s) {
       mbar_init(kfull_b + 8 * s, 1);
       mbar_init(kempty_b + 8 * s, 1);
+    }
+    for (int s = 0; s < NV; ++s) {
       mbar_init(vfull_b + 8 * s, 1);
       mbar_init(vempty_b + 8 * s, 1);
     }
@@ -163,11 +166,11 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kBoundThreads, PrefillCfg<D>::k
   auto wait_use = [&](uint32_t b, int use) { return __all_sync(FULL, mbar_wait_bounded(b, use & 1, kWaitLimitNs)); };
   if (warp == 5) {
     // ================= TMA producer =================
-    // K (kv = 0) or V (kv = 1) of tile i into its ring's stage i % kStages:
-    // one 2-D box per lane (slice s = lane / panels, panel).
+    // K (kv = 0) or V (kv = 1) of tile i into its ring's stage: one 2-D box per
+    // lane (slice s = lane / panels, panel).
     int issued[2] = {0, 0};
     auto issue_kv = [&](int i, int kv) {
-      const int stage = i % C::kStages;
+      const int stage = i % (kv ? NV : NK);
       const uint32_t full = (kv ? vfull_b : kfull_b) + 8 * stage;
       const int kt = kt0 + i * C::kTile;
       const int box = lane;
@@ -191,28 +194,29 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kBoundThreads, PrefillCfg<D>::k
       }
       __syncwarp();
       if (valid) {
-        const uint32_t dst = st_s + stage * C::kStageBytes + kv * C::kKBytes + pn * C::kKVPanelBytes + s * kSliceTokens * 128;
+        const uint32_t dst = (kv ? v_s : k_s) + stage * C::kKBytes + pn * C::kKVPanelBytes + s * kSliceTokens * 128;
         tma_load_2d(dst, kv ? &vmap : &kmap, full, pn * 64, y);
       }
       issued[kv] = i + 1;
     };
-    // Refill order K(j + 1), V(j): a K stage frees when its S is done, a V
-    // stage when its P V is, and S(j + 1 - kStages) is issued before
-    // P V(j - kStages), so the waits come in completion order.
-    auto refill = [&](int j, int kv) {  // tile j >= kStages into the stage tile j - kStages used
-      const int u = j - C::kStages;
-      if (!wait_use((kv ? vempty_b : kempty_b) + 8 * (u % C::kStages), u / C::kStages)) return false;
+    // A K stage frees when the S that read it is done, a V stage when its P V
+    // is.  The MMAs complete in issue order, S(m + 1) before P V(m), so the
+    // refills go in that order: K(m + 1 + NK) after S(m + 1), V(m + NV) after
+    // P V(m).
+    auto refill = [&](int j, int kv) {  // tile j into the stage tile j - N (N = the ring's stages) used
+      const int n = kv ? NV : NK, u = j - n;
+      if (!wait_use((kv ? vempty_b : kempty_b) + 8 * (u % n), u / n)) return false;
       issue_kv(j, kv);
       return true;
     };
     bool ok = true;
-    for (int i = 0; i < C::kStages && i < n_kv; ++i) issue_kv(i, 0);
-    for (int i = 0; i < C::kStages && i < n_kv; ++i) issue_kv(i, 1);
-    if (C::kStages < n_kv) ok = refill(C::kStages, 0);
-    for (int j = C::kStages; ok && j < n_kv; ++j) {
+    for (int i = 0; i < NK && i < n_kv; ++i) issue_kv(i, 0);
+    for (int i = 0; i < NV && i < n_kv; ++i) issue_kv(i, 1);
+    if (NK < n_kv) ok = refill(NK, 0);
+    for (int m = 0; ok && (m + 1 + NK < n_kv || m + NV < n_kv); ++m) {
       if (*abort_flag) break;
-      if (j + 1 < n_kv) ok = refill(j + 1, 0);
-      if (ok) ok = refill(j, 1);
+      if (m + 1 + NK < n_kv) ok = refill(m + 1 + NK, 0);
+      if (ok && m + NV < n_kv) ok = refill(m + NV, 1);
     }
     if (!ok) {
       if (lane == 0) raise_error(PA_DEVERR_TIMEOUT);
@@ -221,17 +225,18 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kBoundThreads, PrefillCfg<D>::k
     if (!ok || *abort_flag) {
       // Before the CTA releases its shared memory: give the last loads of each
       // ring a bounded time to land (earlier ones have, their stages were reused).
-      for (int kv = 0; kv < 2; ++kv)
-        for (int j = max(issued[kv] - C::kStages, 0); j < issued[kv]; ++j)
-          (void)mbar_wait_bounded((kv ? vfull_b : kfull_b) + 8 * (j % C::kStages), (j / C::kStages) & 1,
-                                  kDrainLimitNs);
+      for (int kv = 0; kv < 2; ++kv) {
+        const int n = kv ? NV : NK;
+        for (int j = max(issued[kv] - n, 0); j < issued[kv]; ++j)
+          (void)mbar_wait_bounded((kv ? vfull_b : kfull_b) + 8 * (j % n), (j / n) & 1, kDrainLimitNs);
+      }
     }
   } else if (warp == 4) {
     // ================= MMA issuer (lane 0) =================
     const uint32_t idesc_s = umma::idesc_bf16(128, C::kTile, 0, 0);
     const uint32_t idesc_o = umma::idesc_bf16(128, D, 0, 1);
     auto issue_s = [&](int i) {  // S(i) = Q K(i)^T into buffer i % 2
-      const uint32_t kst = st_s + (i % C::kStages) * C::kStageBytes;
+      const uint32_t kst = k_s + (i % NK) * C::kKBytes;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint64_t ad = umma::desc_sw128(q_s + (kk >> 2) * C::kQPanelBytes + (kk & 3) * 32, 16, 1024);
@@ -239,21 +244,21 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kBoundThreads, PrefillCfg<D>::k
         umma::mma_f16(tmem + C::kSCol + (i & 1) * C::kTile, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
       }
       umma::commit(sfull_b + 8 * (i & 1));
-      umma::commit(kempty_b + 8 * (i % C::kStages));
+      umma::commit(kempty_b + 8 * (i % NK));
     };
-    auto issue_o = [&](int i) {  // O += P V(i)
-      const uint32_t vst = st_s + (i % C::kStages) * C::kStageBytes + C::kKBytes;
+    auto issue_o = [&](int i) {  // O += P V(i), P (bf16 pairs) in the columns of S buffer i % 2
+      const uint32_t vst = v_s + (i % NV) * C::kKBytes;
+      const uint32_t pcol = tmem + C::kSCol + (i & 1) * C::kTile;
 #pragma unroll
       for (int k = 0; k < C::kTile / 16; ++k) {
-        const uint64_t ad = umma::desc_sw128(p_s + k * 32, 16, 1024);
         const uint64_t bd = umma::desc_sw128(vst + k * 16 * 128, C::kKVPanelBytes, 1024);
-        umma::mma_f16(tmem + C::kOCol, ad, bd, idesc_o, (i > 0 || k > 0) ? 1u : 0u);
+        umma::mma_f16_tmem_a(tmem + C::kOCol, pcol + k * 8, bd, idesc_o, (i > 0 || k > 0) ? 1u : 0u);
       }
       umma::commit(odone_b);
-      umma::commit(vempty_b + 8 * (i % C::kStages));
+      umma::commit(vempty_b + 8 * (i % NV));
     };
     auto s_when_ready = [&](int j) {
-      if (!wait_use(kfull_b + 8 * (j % C::kStages), j / C::kStages)) return false;
+      if (!wait_use(kfull_b + 8 * (j % NK), j / NK)) return false;
       umma::fence_after();
       if (lane == 0) issue_s(j);
       __syncwarp();
@@ -264,7 +269,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kBoundThreads, PrefillCfg<D>::k
       if (i + 1 < n_kv && !(ok = s_when_ready(i + 1))) break;
       ok = wait_use(pready_b, i);
       if (!ok || *abort_flag) break;
-      if (!(ok = wait_use(vfull_b + 8 * (i % C::kStages), i / C::kStages))) break;
+      if (!(ok = wait_use(vfull_b + 8 * (i % NV), i / NV))) break;
       umma::fence_after();
       if (lane == 0) issue_o(i);
       __syncwarp();
@@ -347,7 +352,16 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kBoundThreads, PrefillCfg<D>::k
         pk[k] = pack_bf16x2(e0, e1);
       }
       l = l * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
-      if (i > 0) {  // P V(i-1) must be done: it reads the P buffer, and O is rescaled below
+      // P row r into this lane's first 32 columns of S buffer i % 2 (its S
+      // values are in registers; P V(i-1) reads the other buffer).
+      {
+        const uint32_t pcol = lane_base + C::kSCol + (i & 1) * C::kTile;
+        uint32_t (&pk0)[16] = *reinterpret_cast<uint32_t(*)[16]>(&pk[0]);
+        uint32_t (&pk1)[16] = *reinterpret_cast<uint32_t(*)[16]>(&pk[16]);
+        umma::st16_nowait(pcol, pk0);
+        umma::st16_nowait(pcol + 16, pk1);
+      }
+      if (i > 0) {  // P V(i-1) must be done before O is rescaled
         ok = __all_sync(FULL, mbar_wait_bounded(odone_b, (i - 1) & 1, kWaitLimitNs));
         if (!ok) break;
         umma::fence_after();
@@ -362,20 +376,13 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kBoundThreads, PrefillCfg<D>::k
           }
         }
       }
-      // P row r (64 bf16 = 8 chunks) in the canonical K-major SWIZZLE_128B layout.
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint32_t dst = p_s + r * 128 + ((c ^ (r & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pk[4 * c]), "r"(pk[4 * c + 1]),
-                     "r"(pk[4 * c + 2]), "r"(pk[4 * c + 3])
-                     : "memory");
-      }
+      umma::wait_st();
       // V rows of this tile outside [ulo, uhi): zero (stale or canary data, P = 0 there),
       // once V(i) has landed.
       if (kt < ulo || kt + C::kTile > uhi) {
-        ok = __all_sync(FULL, mbar_wait_bounded(vfull_b + 8 * (i % C::kStages), (i / C::kStages) & 1, kWaitLimitNs));
+        ok = __all_sync(FULL, mbar_wait_bounded(vfull_b + 8 * (i % NV), (i / NV) & 1, kWaitLimitNs));
         if (!ok) break;
-        const uint32_t vst = st_s + (i % C::kStages) * C::kStageBytes + C::kKBytes;
+        const uint32_t vst = v_s + (i % NV) * C::kKBytes;
         for (int idx = tid; idx < C::kTile * C::kPanels * 8; idx += C::kRows) {
           const int row = idx / (C::kPanels * 8), rem = idx % (C::kPanels * 8);
           const int t = kt + row;
@@ -384,8 +391,8 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kBoundThreads, PrefillCfg<D>::k
             asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
           }
         }
+        fence_proxy_async_smem();  // the zeros are visible to the tensor core's reads
       }
-      fence_proxy_async_smem();
       umma::fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(pready_b);
