@@ -169,17 +169,34 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kBoundThreads, PrefillCfg<D>::k
     // K (kv = 0) or V (kv = 1) of tile i into its ring's stage: one 2-D box per
     // lane (slice s = lane / panels, panel).
     int issued[2] = {0, 0};
+    // Physical blocks of the 16-token slices, per ring: lane l holds slice
+    // wb + l (cur) and wb + 32 + l (nxt), and the window after is loaded as soon
+    // as a ring moves on, so no load waits on a block-table read (with the read
+    // in line, the producer took one L2 round trip per tile and set the pace).
+    auto page_of = [&](int q) {  // slice q of the K/V range; -1 past the attended range
+      const int t = kt0 + q * kSliceTokens;
+      return t < uhi ? table[t >> p.log2_bs] : -1;
+    };
+    int wb[2] = {0, 0}, wcur[2], wnxt[2];
+    wcur[0] = wcur[1] = page_of(lane);
+    wnxt[0] = wnxt[1] = page_of(32 + lane);
     auto issue_kv = [&](int i, int kv) {
       const int stage = i % (kv ? NV : NK);
       const uint32_t full = (kv ? vfull_b : kfull_b) + 8 * stage;
       const int kt = kt0 + i * C::kTile;
+      if (4 * i >= wb[kv] + 32) {  // tiles advance one at a time: the window moves by 32 slices
+        wb[kv] += 32;
+        wcur[kv] = wnxt[kv];
+        wnxt[kv] = page_of(wb[kv] + 32 + lane);
+      }
       const int box = lane;
       const int s = box / C::kPanels, pn = box % C::kPanels;
       const int t = kt + s * kSliceTokens;
+      const int page = __shfl_sync(FULL, wcur[kv], (4 * i + (s & 3) - wb[kv]) & 31);
       bool valid = false;
       int y = -1;
       if (box < 4 * C::kPanels && t + kSliceTokens > ulo && t < uhi) {
-        const int phys = table[t >> p.log2_bs];
+        const int phys = page;
         if (phys >= 0 && phys < p.num_blocks) {
           valid = true;
           y = cache_row(p, phys, g, t);
@@ -328,8 +345,14 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kBoundThreads, PrefillCfg<D>::k
           x[k] = (t >= lo_r && t < hi_r) ? x[k] : -CUDART_INF_F;
         }
       }
+      {  // eight independent chains, then a tree: the 64-long dependent chain took 0.2 us a tile
+        float mx[8];
 #pragma unroll
-      for (int k = 0; k < C::kTile; ++k) mt = fmaxf(mt, x[k]);
+        for (int c = 0; c < 8; ++c) mx[c] = x[c];
+#pragma unroll
+        for (int k = 8; k < C::kTile; ++k) mx[k & 7] = fmaxf(mx[k & 7], x[k]);
+        mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      }
       mt *= xs;  // xs > 0: the maximum of the scaled scores
       // Lazy rescaling: keep the reference m while the tile's maximum exceeds
       // it by at most 8 (log2 units): the weights stay <= 256 and the sum and
