@@ -1,13 +1,15 @@
-// Multi-query rows on the warp-per-item dynamic schedule, for R = T*G <= 16
-// query rows per kv head (speculative-decoding verify with a few draft tokens)
-// and head_dim <= 128 (the 16 x D output tile lives in registers).
+// Multi-query rows on the warp-per-item dynamic schedule, for R = T*G query
+// rows per kv head (speculative-decoding verify with a few draft tokens):
+// MT 16-row tiles per warp, R <= 16 MT, the MT x 16 x D output tiles in
+// registers (MT = 2 at head_dim 64, 1 at 128).
 //
 // The work items, the persistent grid, the index-fixed first items and the
 // claims, and each warp's TMA ring are those of the decode kernel
 // (decode_dynamic.cuh); what differs is the attention: the R query rows of
 // (sequence b, kv head g) -- token j = r / G, head h = r % G, at position
 // p_j = L - T + j -- are the 16-row M dimension of the MMA
-// (attend_slice_rows), each row with its own causal / window range.  The
+// (attend_slice_rows, once per 16-row tile on the same K/V stage), each row
+// with its own causal / window range.  The
 // sequence's union range is [s0 of token 0, L); an item covers one partition
 // of it, and writes either the normalised rows (the sequence's only
 // partition) or partials for the combine kernel, which merges [B][T][Hq] rows.
@@ -20,7 +22,9 @@
 
 namespace pa {
 
-constexpr int kMaxRowsPerWarp = 16;
+// Query rows one warp carries per item: its 16-row MMA tiles times 16.
+template <int D>
+__host__ __device__ constexpr int rows_tiles() { return D <= 64 ? 2 : 1; }
 
 template <int D, int NW, int ST>
 __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
@@ -31,7 +35,8 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int G = p.group, Hkv = p.hkv, P = p.partition, B = p.batch, T = p.q_len;
-  const int R = T * G;  // query rows per (sequence, kv head), <= 16
+  constexpr int MT = rows_tiles<D>();
+  const int R = T * G;  // query rows per (sequence, kv head), <= 16 MT
   int* scratch = reinterpret_cast<int*>(smem + Cfg::kScratchOffset);
   int* pre = reinterpret_cast<int*>(smem + Cfg::kPrefixOffset);  // [B+1] items before sequence b
   int* lens = pre + B + 1;                                        // [B] clamped context lengths
@@ -107,9 +112,10 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
     return it;
   };
 
-  // This lane's rows r0 = lane / 4 and r1 = r0 + 8 of an item: output row
-  // index ((b*T + j)*Hq + g*G + h) and token range inside the item.
-  const int r0 = lane >> 2, r1 = r0 + 8;
+  // This lane's rows 16 m + lane / 4 and 16 m + lane / 4 + 8 of tile m of an
+  // item: output row index ((b*T + j)*Hq + g*G + h) and token range inside
+  // the item.
+  const int r0 = lane >> 2;
   auto out_row = [&](const Item& it, int r) {
     return ((size_t)it.b * T + r / G) * p.hq + (size_t)it.g * G + r % G;
   };
@@ -124,9 +130,13 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
     hi = min(end, it.hi);
   };
   const __nv_bfloat16* q0 = static_cast<const __nv_bfloat16*>(p.q);
-  auto load_q = [&](uint32_t (&qa)[D / 16][4], const Item& it) {
-    load_q_rows<D>(qa, q0 + out_row(it, r0 < R ? r0 : 0) * D, r0 < R, q0 + out_row(it, r1 < R ? r1 : 0) * D,
-                   r1 < R, lane);
+  auto load_q = [&](uint32_t (&qa)[MT][D / 16][4], const Item& it) {
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      const int ra = 16 * m + r0, rb = ra + 8;
+      load_q_rows<D>(qa[m], q0 + out_row(it, ra < R ? ra : 0) * D, ra < R, q0 + out_row(it, rb < R ? rb : 0) * D,
+                     rb < R, lane);
+    }
   };
 
   const int n_static = p.static_items;
@@ -172,7 +182,7 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
       }
     };
     load_rows(ii, 0);
-    uint32_t qa[D / 16][4];  // the next item's rows are loaded when it starts (its K/V are in flight by then)
+    uint32_t qa[MT][D / 16][4];  // the next item's rows are loaded when it starts (its K/V are in flight by then)
     load_q(qa, ci);
 
     auto fill = [&]() {
@@ -195,16 +205,20 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
       }
     };
 
-    WarpRows<D> st;
-    st.reset();
+    WarpRows<D> st[MT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) st[m].reset();
     const float qk_scale = p.use_softcap ? p.scale : p.scale * kLog2e;
     const int tq = lane & 3;
     bool aborted = false;
 
     while (true) {
-      ColRange cr;
-      row_range(ci, r0, cr.lo0, cr.hi0);
-      row_range(ci, r1, cr.lo1, cr.hi1);
+      ColRange cr[MT];
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        row_range(ci, 16 * m + r0, cr[m].lo0, cr[m].hi0);
+        row_range(ci, 16 * m + r0 + 8, cr[m].lo1, cr[m].hi1);
+      }
       for (int ck = 0; ck < ci.n; ++ck) {
         fill();
         bool ok = mbar_wait_bounded(bars + 8 * (gc % ST), (gc / ST) & 1, kWaitLimitNs);
@@ -214,8 +228,11 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
           break;
         }
         const uint32_t kbase = ring + (gc % ST) * Cfg::kStageBytes;
-        attend_slice_rows<D>(st, qa, kbase, kbase + Cfg::kSliceBytes, (ci.j0 + ck) * kSliceTokens, ci.lo, ci.hi, cr,
-                             qk_scale, p, lane);
+#pragma unroll
+        for (int m = 0; m < MT; ++m)
+          if (m == 0 || 16 * m < R)
+            attend_slice_rows<D>(st[m], qa[m], kbase, kbase + Cfg::kSliceBytes, (ci.j0 + ck) * kSliceTokens, ci.lo,
+                                 ci.hi, cr[m], qk_scale, p, lane);
         __syncwarp();
         ++gc;
       }
@@ -223,32 +240,36 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
       fill();  // keep loading the next item while this one is stored
 
       // ---- store this item's rows from registers ----------------------------------------
-      st.reduce_sums();
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int r = e ? r1 : r0;
-        if (r >= R) continue;
-        const size_t row = out_row(ci, r);
-        const float m = e ? st.m1 : st.m0, l = e ? st.l1 : st.l0;
-        if (ci.whole) {
-          const float inv = l > 0.f ? 1.f / l : 0.f;  // a row with no position is zero
-          __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + row * D + 2 * tq;
+      for (int mt = 0; mt < MT; ++mt) {
+        WarpRows<D>& sm = st[mt];
+        sm.reduce_sums();
 #pragma unroll
-          for (int nt = 0; nt < D / 8; ++nt)
-            *reinterpret_cast<uint32_t*>(o + nt * 8) = pack_bf16x2(st.o[nt][2 * e] * inv, st.o[nt][2 * e + 1] * inv);
-        } else {
-          float* po = p.ws_o + (row * p.max_parts + ci.part) * D + 2 * tq;
+        for (int e = 0; e < 2; ++e) {
+          const int r = 16 * mt + r0 + 8 * e;
+          if (r >= R) continue;
+          const size_t row = out_row(ci, r);
+          const float m = e ? sm.m1 : sm.m0, l = e ? sm.l1 : sm.l0;
+          if (ci.whole) {
+            const float inv = l > 0.f ? 1.f / l : 0.f;  // a row with no position is zero
+            __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + row * D + 2 * tq;
 #pragma unroll
-          for (int nt = 0; nt < D / 8; ++nt)
-            *reinterpret_cast<float2*>(po + nt * 8) = make_float2(st.o[nt][2 * e], st.o[nt][2 * e + 1]);
-          if (tq == 0) {
-            float* pml = p.ws_ml + (row * p.max_parts + ci.part) * 2;
-            pml[0] = m;
-            pml[1] = l;
+            for (int nt = 0; nt < D / 8; ++nt)
+              *reinterpret_cast<uint32_t*>(o + nt * 8) = pack_bf16x2(sm.o[nt][2 * e] * inv, sm.o[nt][2 * e + 1] * inv);
+          } else {
+            float* po = p.ws_o + (row * p.max_parts + ci.part) * D + 2 * tq;
+#pragma unroll
+            for (int nt = 0; nt < D / 8; ++nt)
+              *reinterpret_cast<float2*>(po + nt * 8) = make_float2(sm.o[nt][2 * e], sm.o[nt][2 * e + 1]);
+            if (tq == 0) {
+              float* pml = p.ws_ml + (row * p.max_parts + ci.part) * 2;
+              pml[0] = m;
+              pml[1] = l;
+            }
           }
         }
+        sm.reset();
       }
-      st.reset();
 
       // ---- next item ------------------------------------------------------------------
       resolve_next();

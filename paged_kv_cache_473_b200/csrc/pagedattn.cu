@@ -718,10 +718,11 @@ pa_status_t pa_decode_step(const void* q, const void* k_new, const void* v_new, 
 }
 
 // Whether multi-query rows run on the dynamic warp-per-item schedule: at most
-// 16 query rows (T * G) per kv head, head_dim <= 128, and a batch the schedule
+// 32 query rows (T * G) per kv head at head_dim 64, 16 at 128, and a batch the schedule
 // takes.
 bool multi_rows_path(int32_t batch, int32_t q_len, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim) {
-  return head_dim <= 128 && (long long)q_len * (num_q_heads / num_kv_heads) <= pa::kMaxRowsPerWarp &&
+  const int rows = head_dim <= 64 ? 16 * pa::rows_tiles<64>() : 16 * pa::rows_tiles<128>();
+  return head_dim <= 128 && (long long)q_len * (num_q_heads / num_kv_heads) <= rows &&
          batch <= pa::kMaxDynamicBatch && (long long)batch * num_kv_heads <= pa::kMaxDynamicUnits;
 }
 

@@ -58,7 +58,7 @@ def _ref(w, b_cpu, q, window=None, softcap=None, rows=None):
                                cap, win, rows=rows)
 
 
-@pytest.mark.parametrize("name,T", [("tinyllama_1b", 1), ("tinyllama_1b", 2), ("tinyllama_1b", 4),
+@pytest.mark.parametrize("name,T", [("tinyllama_1b", 1), ("tinyllama_1b", 2), ("tinyllama_1b", 3), ("tinyllama_1b", 4),
                                     ("tinyllama_1b", 8), ("gemma2_2b", 5), ("gemma2_2b", 32), ("llama3_8b", 3),
                                     ("llama3_8b", 4), ("llama3_8b", 16), ("long_splitk", 4), ("long_splitk", 6)])
 @pytest.mark.parametrize("split,partition", [(False, 0), (True, 0), (True, 64)])
@@ -82,8 +82,19 @@ def test_multi_window_per_query_token(window, split, T):
     assert_close(out, ref, torch.bfloat16, f"multi window={window} split={split}")
 
 
+@pytest.mark.parametrize("window", [1, 5, 40])
+@pytest.mark.parametrize("T", [3, 4])
+def test_multi_window_two_row_tiles(window, T):
+    """head_dim 64 with 24 and 32 query rows per kv head: two 16-row tiles per
+    warp on the warp-per-item path, the second partly padding at T = 3."""
+    w, b_cpu, b, mq = _case("tinyllama_1b", T)
+    out = _run(w, b, mq["q"], True, 0, window=window)
+    ref = _ref(w, b_cpu, mq["q"], window=window)
+    assert_close(out, ref, torch.bfloat16, f"multi two tiles window={window} T={T}")
+
+
 @pytest.mark.parametrize("split", [False, True])
-@pytest.mark.parametrize("name,T", [("tinyllama_1b", 5), ("tinyllama_1b", 2), ("llama3_8b", 4)])
+@pytest.mark.parametrize("name,T", [("tinyllama_1b", 5), ("tinyllama_1b", 2), ("tinyllama_1b", 4), ("llama3_8b", 4)])
 def test_multi_short_and_empty_sequences(split, name, T):
     """L = 0 rows, L < T (early query tokens see nothing: zero rows), L = T,
     ranges inside one slice and across block edges."""
