@@ -69,6 +69,35 @@ def test_prefill_window_and_softcap(window):
     assert_close(out, ref, torch.bfloat16, f"prefill window={window} softcap 50")
 
 
+@pytest.mark.parametrize("name", ["tinyllama_1b", "llama3_8b"])
+@pytest.mark.parametrize("window", [1, 33, 200])
+def test_prefill_window_small_heads(name, window):
+    """Sliding windows at head_dim 64 and 128: windows that start inside a
+    64-token K/V tile and ones spanning several."""
+    lengths = [300, 129, 17]
+    w, out, ref, _, _ = _run(name, lengths, [260, 129, 17], window=window)
+    assert_close(out, ref, torch.bfloat16, f"prefill {name} window={window}")
+
+
+@pytest.mark.parametrize("name", ["tinyllama_1b", "llama3_8b"])
+def test_prefill_softcap_small_heads(name):
+    lengths = [200, 77]
+    w, out, ref, _, _ = _run(name, lengths, lengths, softcap=30.0)
+    assert_close(out, ref, torch.bfloat16, f"prefill {name} softcap 30")
+
+
+@pytest.mark.parametrize("name", ["tinyllama_1b", "llama3_8b"])
+def test_prefill_query_tile_edges(name):
+    """Prompt lengths at the edges of a CTA's query tile (16 or 32 tokens with
+    8 or 4 query heads per kv head) and of 64- and 128-token K/V spans: the
+    last tile partly filled, and K/V ranges ending inside or at the end of a
+    tile."""
+    lengths = [15, 16, 17, 31, 32, 33, 63, 64, 65, 127, 128, 129]
+    w, out, ref, (kc, vc), (kc_ref, vc_ref) = _run(name, lengths, lengths)
+    assert torch.equal(bits(kc), bits(kc_ref)) and torch.equal(bits(vc), bits(vc_ref))
+    assert_close(out, ref, torch.bfloat16, f"prefill edges {name}")
+
+
 def test_prefill_attend_only():
     """k_new = v_new = NULL: the rows are already in the cache."""
     lengths = [120, 33]
