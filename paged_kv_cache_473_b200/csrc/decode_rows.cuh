@@ -1,7 +1,7 @@
 // Multi-query rows on the warp-per-item dynamic schedule, for R = T*G query
 // rows per kv head (speculative-decoding verify with a few draft tokens):
 // MT 16-row tiles per warp, R <= 16 MT, the MT x 16 x D output tiles in
-// registers (MT = 2 at head_dim 64, 1 at 128).
+// registers (MT = 2 at head_dim 64, 1 at 128 and 256).
 //
 // The work items, the persistent grid, the index-fixed first items and the
 // claims, and each warp's TMA ring are those of the decode kernel

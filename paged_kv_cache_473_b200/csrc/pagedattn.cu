@@ -434,7 +434,14 @@ cudaError_t launch_rows_t(DecodeParams& p, cudaStream_t st) {
 }
 
 cudaError_t launch_rows(DecodeParams& p, cudaStream_t st) {
-  return p.head_dim == 64 ? launch_rows_t<64, 4, 6>(p, st) : launch_rows_t<128, 4, 2>(p, st);
+  switch (p.head_dim) {
+    case 64:
+      return launch_rows_t<64, 4, 6>(p, st);
+    case 128:
+      return launch_rows_t<128, 4, 2>(p, st);
+    default:
+      return launch_rows_t<256, 2, 2>(p, st);
+  }
 }
 
 
@@ -718,11 +725,11 @@ pa_status_t pa_decode_step(const void* q, const void* k_new, const void* v_new, 
 }
 
 // Whether multi-query rows run on the dynamic warp-per-item schedule: at most
-// 32 query rows (T * G) per kv head at head_dim 64, 16 at 128, and a batch the schedule
+// 32 query rows (T * G) per kv head at head_dim 64, 16 at 128 and 256, and a batch the schedule
 // takes.
 bool multi_rows_path(int32_t batch, int32_t q_len, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim) {
   const int rows = head_dim <= 64 ? 16 * pa::rows_tiles<64>() : 16 * pa::rows_tiles<128>();
-  return head_dim <= 128 && (long long)q_len * (num_q_heads / num_kv_heads) <= rows &&
+  return (long long)q_len * (num_q_heads / num_kv_heads) <= rows &&
          batch <= pa::kMaxDynamicBatch && (long long)batch * num_kv_heads <= pa::kMaxDynamicUnits;
 }
 
@@ -735,12 +742,13 @@ int32_t multi_partition(int32_t batch, int32_t q_len, int32_t num_q_heads, int32
     return auto_partition(batch, num_kv_heads, max_context_len, 0);
   // The rows path writes T*G partial rows per item, twice the decode's at
   // T*G = 16: at head_dim 128 512-token partitions keep the partials and the
-  // combine small (a sweep on B200: Llama-3 T=4, 0.76 -> 0.89 of HBM peak);
-  // halved, as for decode, while there are fewer items than resident warps.
+  // combine small (a sweep on B200: Llama-3 T=4, 0.76 -> 0.89 of HBM peak; at
+  // head_dim 256, Gemma-2 T=8: 128 / 256 / 512 tokens gave 155 / 139 / 161
+  // us); halved, as for decode, while there are fewer items than resident warps.
   const long long work = (long long)(batch > 0 ? batch : 1) * (num_kv_heads > 0 ? num_kv_heads : 1) *
                          (max_context_len > 0 ? max_context_len : 1);
-  int P = head_dim <= 64 ? 256 : 512;
-  const int warps_per_sm = head_dim <= 64 ? 8 : 12;
+  int P = head_dim <= 64 ? 256 : head_dim <= 128 ? 512 : 256;
+  const int warps_per_sm = head_dim <= 64 ? 8 : head_dim <= 128 ? 12 : 6;
   while (P > 64 && work / P < (long long)warps_per_sm * 148) P >>= 1;
   return P;
 }

@@ -93,8 +93,20 @@ def test_multi_window_two_row_tiles(window, T):
     assert_close(out, ref, torch.bfloat16, f"multi two tiles window={window} T={T}")
 
 
+@pytest.mark.parametrize("window", [1, 20, 300])
+@pytest.mark.parametrize("T", [5, 8])
+def test_multi_window_head_dim_256(window, T):
+    """head_dim 256 (softcap 50) with 10 and 16 query rows per kv head: the
+    rows kernel's one 16-row tile per warp, per-row windows."""
+    w, b_cpu, b, mq = _case("gemma2_2b", T)
+    out = _run(w, b, mq["q"], True, 0, window=window)
+    ref = _ref(w, b_cpu, mq["q"], window=window)
+    assert_close(out, ref, torch.bfloat16, f"multi head_dim 256 window={window} T={T}")
+
+
 @pytest.mark.parametrize("split", [False, True])
-@pytest.mark.parametrize("name,T", [("tinyllama_1b", 5), ("tinyllama_1b", 2), ("tinyllama_1b", 4), ("llama3_8b", 4)])
+@pytest.mark.parametrize("name,T", [("tinyllama_1b", 5), ("tinyllama_1b", 2), ("tinyllama_1b", 4), ("llama3_8b", 4),
+                                    ("gemma2_2b", 8)])
 def test_multi_short_and_empty_sequences(split, name, T):
     """L = 0 rows, L < T (early query tokens see nothing: zero rows), L = T,
     ranges inside one slice and across block edges."""
