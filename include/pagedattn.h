@@ -211,10 +211,14 @@ pa_status_t pa_decode_step(const void* q, const void* k_new, const void* v_new, 
  *   num_kv_heads) <= 64 (PA_ERR_UNSUPPORTED above).
  *   partition_tokens < 0: one CTA per (sequence, kv head), no workspace
  *   (workspace may be NULL; max_context_len is ignored).  partition_tokens >= 0:
- *   split-K as pa_decode_splitk's grid schedule (0 = library's choice), with a
- *   workspace of pa_decode_multi_workspace_size() bytes under the same
- *   contract as pa_decode_splitk's, and a combine kernel for sequences whose
- *   range spans several partitions.
+ *   split-K (0 = library's choice) with a workspace of
+ *   pa_decode_multi_workspace_size() bytes under the same contract as
+ *   pa_decode_splitk's, and a combine kernel for sequences whose range spans
+ *   several partitions.  With at most 16 query rows per kv head (q_len *
+ *   num_q_heads / num_kv_heads; 32 at head_dim 64) the rows run on
+ *   pa_decode_splitk's warp-per-item schedule, one warp per (sequence, kv
+ *   head, partition); above that, on one CTA per (partition, kv head,
+ *   sequence).
  *   Passages: nano-vllm (ovshake) README, "Features" (chunked prefill,
  *   speculative decoding) and the speculative-decoding command line
  *   (--num-speculative-tokens); causal attention over the cache as in "Key
