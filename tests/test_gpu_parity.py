@@ -458,12 +458,19 @@ def test_dynamic_schedule_counters_return_to_zero():
 COUNTER_BYTES = 256 * 1024  # the workspace's fixed counter region
 
 
-@pytest.mark.parametrize("name,kw", [("tinyllama_1b", dict(batch=24)),  # fixed items cover the work: no claims
-                                     ("llama3_8b", dict(batch=64))])    # more items than 2 per warp: claims
+@pytest.mark.parametrize("name,kw", [
+    ("tinyllama_1b", dict(batch=24)),  # fixed items cover the work, the last partial merges
+    ("llama3_8b", dict(batch=64)),     # more items than 2 per warp (claims), combine kernel
+    # at most 8 partitions but more than 2 items per warp: claims and the combine kernel
+    ("gemma2_2b", dict(batch=256)),
+    ("llama3_8b", dict(batch=128, max_len=2048)),
+    ("tinyllama_1b", dict(batch=256)),
+])
 def test_dynamic_schedule_counter_region_reads_zero_after_each_call(name, kw):
-    """Whether or not warps claim items from the work counter, the workspace's
-    counter region is all zero when the call ends (the next call relies on it),
-    with the fused append and without."""
+    """Whichever way the partitions are merged, and whether or not warps claim
+    items from the work counter, the step matches the oracle and the
+    workspace's counter region is all zero when the call ends (the next call
+    relies on it)."""
     w = wl.WORKLOADS[name]
     bc = wl.make_batch(w, prefilled=False, **kw)
     b = to_dev(bc)
