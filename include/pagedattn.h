@@ -338,6 +338,18 @@ pa_status_t pa_decode_splitk_noalloc(const void* q, const void* k_cache, const v
  */
 pa_status_t pa_device_errors(uint32_t* bits, int32_t clear);
 
+/*
+ * pa_check_bounded_wait -- diagnostic: launch one CTA that waits on an
+ * mbarrier nothing ever arrives on, with the bounded wait every kernel of this
+ * library uses for its TMA and MMA completions.  The wait gives up after
+ * limit_ns nanoseconds of %globaltimer (0 < limit_ns <= 1e9, else
+ * PA_ERR_INVALID) and raises PA_DEVERR_TIMEOUT in the device error word; the
+ * kernel then returns and the context stays usable.  It shows on a GPU that
+ * a wait that never completes ends in an error status instead of a hang.
+ * Asynchronous on stream; read the result with pa_device_errors().
+ */
+pa_status_t pa_check_bounded_wait(uint64_t limit_ns, pa_stream_t stream);
+
 /* Static description of a status code. */
 const char* pa_error_string(pa_status_t status);
 

@@ -25,6 +25,7 @@ from ._binding import (  # noqa: F401
     decode_step,
     decode_splitk_partition,
     decode_splitk_workspace_size,
+    check_bounded_wait,
     device_errors,
     error_string,
     last_launch_count,
@@ -47,6 +48,7 @@ __all__ = [
     "decode_step",
     "decode_splitk_partition",
     "decode_splitk_workspace_size",
+    "check_bounded_wait",
     "device_errors",
     "error_string",
     "last_launch_count",

@@ -100,6 +100,8 @@ def _load_library() -> ctypes.CDLL:
     lib.pa_decode_cascade.restype = _c_i32
     lib.pa_decode_cascade_workspace_size.argtypes = [_c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32, _c_i32]
     lib.pa_decode_cascade_workspace_size.restype = _c_sz
+    lib.pa_check_bounded_wait.argtypes = [ctypes.c_uint64, _c_vp]
+    lib.pa_check_bounded_wait.restype = _c_i32
     lib.pa_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint32), _c_i32]
     lib.pa_device_errors.restype = _c_i32
     lib.pa_error_string.argtypes = [_c_i32]
@@ -445,6 +447,12 @@ def device_errors(clear: bool = True) -> int:
     bits = ctypes.c_uint32(0)
     _check(lib.pa_device_errors(ctypes.byref(bits), 1 if clear else 0), "pa_device_errors")
     return bits.value
+
+
+def check_bounded_wait(limit_ns: int = 1_000_000, stream=None) -> None:
+    """Launch the bounded-wait check (a wait nothing completes, given up after
+    ``limit_ns``); read the resulting PA_DEVERR_TIMEOUT with device_errors()."""
+    _check(lib.pa_check_bounded_wait(int(limit_ns), _stream(stream)), "pa_check_bounded_wait")
 
 
 def last_launch_count() -> int:

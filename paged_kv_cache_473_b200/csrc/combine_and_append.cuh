@@ -101,6 +101,23 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const Decod
   for (int v = 0; v < VEC; ++v) store_out<OutT>(out + v, acc[v] * inv);
 }
 
+// ---- bounded-wait check ---------------------------------------------------------
+//
+// One warp waits on an mbarrier that nothing arrives on, with the bounded wait
+// of every TMA / MMA completion in this library; when it gives up it raises
+// PA_DEVERR_TIMEOUT, as the kernels do, and returns.
+__global__ void bounded_wait_check_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = smem_addr(&bar);
+  if (threadIdx.x == 0) {
+    mbar_init(b, 1);
+    mbar_init_fence();
+  }
+  __syncwarp();
+  const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(b, 0, limit_ns));
+  if (!ok && threadIdx.x == 0) raise_error(PA_DEVERR_TIMEOUT);
+}
+
 // ---- KV append ------------------------------------------------------------------
 //
 // One thread per 16-byte chunk of one (token, kv head) row of K and of V:

@@ -1036,6 +1036,15 @@ pa_status_t pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, i
   return PA_OK;
 }
 
+pa_status_t pa_check_bounded_wait(uint64_t limit_ns, pa_stream_t stream) {
+  t_last_launches = 0;
+  if (limit_ns == 0 || limit_ns > pa::kWaitLimitNs) return PA_ERR_INVALID;
+  pa::bounded_wait_check_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+  if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  t_last_launches = 1;
+  return PA_OK;
+}
+
 pa_status_t pa_device_errors(uint32_t* bits, int32_t clear) {
   if (!bits) return PA_ERR_INVALID;
   unsigned int v = 0;

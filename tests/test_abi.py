@@ -264,3 +264,9 @@ def test_cascade_workspace_covers_its_partition():
     n = pa.decode_cascade_workspace_size(128, 32, 128, 8192, 1024, 0, 8)
     assert n >= pa.decode_splitk_workspace_size(128, 32, 128, 8192, 0, 8)
     assert pa.decode_cascade_workspace_size(128, 32, 128, 8192, 1024, 384, 8) == 0
+
+
+def test_bounded_wait_check_rejects_bad_limits():
+    """pa_check_bounded_wait checks its bound before any launch (no GPU needed)."""
+    assert bnd.lib.pa_check_bounded_wait(0, None) == bnd.PA_ERR_INVALID
+    assert bnd.lib.pa_check_bounded_wait(2_000_000_000, None) == bnd.PA_ERR_INVALID
