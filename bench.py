@@ -430,6 +430,35 @@ class CascadeRunner(Runner):
         self.launches_per_step = n
 
 
+class DecodeOnlyRunner(Runner):
+    """The decode without the append (pa_decode_splitk, library's schedule):
+    the cache already holds position L-1 of every sequence, written once up
+    front, so a step is only the attention."""
+
+    def __init__(self, w: wl.Workload, rank: int):
+        # fused=True: every launch of a step belongs to the timed op, as in the step
+        super().__init__(w, rank, "auto", True, 0, fused=True)
+        b = self.batch
+        for kc, vc in self.pools:
+            self.pa.write_kv(b.k_new, b.v_new, b.slot_mapping, kc, vc)
+        torch.cuda.synchronize()
+
+    def decode(self, r, x):
+        w, b = self.w, self.batch
+        kc, vc = self.pools[r]
+        self.pa.decode_splitk(b.q, kc, vc, b.block_tables, b.context_lens, w.scale, w.softcap, w.window,
+                              max_context_len=self.max_ctx, partition_tokens=0, out=self.out, workspace=self.ws)
+        return self.pa.last_launch_count()
+
+    def step(self, r, x=None, ev=None):
+        if ev is not None:
+            ev[0].record()
+        n = self.decode(r, None)
+        if ev is not None:
+            ev[1].record()
+        self.launches_per_step = n
+
+
 def run_timed(runner: Runner, K: int, W: int, world: int, device_index: int):
     """Warm up W steps, then time exactly K graph-replayed steps."""
     for i in range(W):
@@ -740,6 +769,19 @@ def main_ours(args, world, rank, local):
         "gpu_launches": K * launches_per_step,
         "clocks": clocks,
     }
+    if world == 1 and rank == 0 and runner.fused and split:
+        # The attention alone (the append already done), timed the same way.
+        dr = DecodeOnlyRunner(w, rank)
+        d_total, d_dec, _ = run_timed(dr, K, W, 1, local)
+        d_ms, _ = op_duration(dr, d_total, K, d_dec)
+        line["decode_alone"] = {
+            "ms_per_step": round(d_ms, 5),
+            "tokens_per_s": round(dr.B / (d_ms * 1e-3), 1),
+            "kv_gbs": round(dr.kv_bytes / (d_ms * 1e-3) / 1e9, 1),
+            "frac": round(dr.kv_bytes / (d_ms * 1e-3) / 1e9 / peak, 4),
+            "launches_per_step": dr.launches_per_step,
+        }
+        del dr
     if world == 1 and rank == 0 and args.shapes != "none":
         names = [n for n in wl.WORKLOADS if n not in (w.name, "tiny_fp32")] if args.shapes == "auto" else [
             s for s in args.shapes.split(",") if s]
