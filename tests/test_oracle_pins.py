@@ -426,3 +426,60 @@ def test_chunked_prefill_equals_one_shot_prefill():
     second = oracle.prefill(q[c1:], ks[0][c1:], vs[0][c1:], slots[c1:], torch.tensor([0, L - c1], dtype=torch.int32),
                             kc2, vc2, tables, cl, 0.3)
     assert np.array_equal(np.concatenate([first, second]), one)
+
+
+def _partial_log2(q, k, v, scale, softcap):
+    """One partition's (m, l, o) in the log2 domain, fp64: s = scaled (and
+    capped) scores times log2(e); m = max s, l = sum 2^(s-m), o = sum 2^(s-m) v."""
+    s = (k @ q) * scale
+    if softcap > 0 and math.isfinite(softcap):
+        s = softcap * np.tanh(s / softcap)
+    s = s * math.log2(math.e)
+    if s.size == 0:
+        return -math.inf, 0.0, np.zeros(v.shape[1])
+    m = s.max()
+    w = np.exp2(s - m)
+    return m, w.sum(), w @ v
+
+
+def _merge(parts):
+    """Log-sum-exp merge: M = max m_p, out = sum 2^(m_p - M) o_p / sum 2^(m_p - M) l_p
+    (empty partitions, m = -inf, weigh nothing)."""
+    M = max(m for m, _, _ in parts)
+    num = sum((0.0 if m == -math.inf else 2.0 ** (m - M)) * o for m, _, o in parts)
+    den = sum((0.0 if m == -math.inf else 2.0 ** (m - M)) * l for m, l, _ in parts)
+    return num / den
+
+
+@pytest.mark.parametrize("P", [16, 64, 256])
+@pytest.mark.parametrize("softcap,window", [(0.0, 0), (30.0, 0), (0.0, 50)])
+def test_split_k_merge_rule_reproduces_the_unsplit_definition(P, softcap, window):
+    """The split-K partials and their log-sum-exp merge (what the combine kernel
+    and the in-kernel merges compute) equal the oracle's unsplit attention,
+    for partitions that split the window start and the end, empty
+    partitions included.  The cascade's prefix / own-range split is the same
+    identity with two partitions."""
+    gen = torch.Generator().manual_seed(41)
+    lens = [1, 37, 300]
+    hq, hkv, d = 4, 2, 16
+    ks, vs = _rand_seqs(gen, lens, hkv, d)
+    q = torch.randn((len(lens), hq, d), generator=gen)
+    kc, vc, tables, cl = scatter_to_pool(ks, vs, 16, gen)
+    scale = 1 / math.sqrt(d)
+    ref = oracle.decode(q, kc, vc, tables, cl, scale, softcap=softcap, window=window)
+    for b, L in enumerate(lens):
+        s0 = L - window if window and L > window else 0
+        for h in range(hq):
+            g = h // (hq // hkv)
+            k = ks[b][:, g].double().numpy()
+            v = vs[b][:, g].double().numpy()
+            qv = q[b, h].double().numpy()
+            bounds = [s0] + list(range((s0 // P + 1) * P, L, P)) + [L]
+            parts = [_partial_log2(qv, k[lo:hi], v[lo:hi], scale, softcap) for lo, hi in zip(bounds, bounds[1:])]
+            parts.append(_partial_log2(qv, k[:0], v[:0], scale, softcap))  # an empty partition
+            assert np.max(np.abs(_merge(parts) - ref[b, h])) <= 1e-12
+            if L > 1:  # cascade: prefix [s0, c) and own range [c, L)
+                c = s0 + (L - s0) // 2
+                two = [_partial_log2(qv, k[s0:c], v[s0:c], scale, softcap),
+                       _partial_log2(qv, k[c:L], v[c:L], scale, softcap)]
+                assert np.max(np.abs(_merge(two) - ref[b, h])) <= 1e-12
