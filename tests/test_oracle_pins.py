@@ -465,7 +465,7 @@ def test_split_k_merge_rule_reproduces_the_unsplit_definition(P, softcap, window
     ks, vs = _rand_seqs(gen, lens, hkv, d)
     q = torch.randn((len(lens), hq, d), generator=gen)
     kc, vc, tables, cl = scatter_to_pool(ks, vs, 16, gen)
-    scale = 1 / math.sqrt(d)
+    scale = float(np.float32(1 / math.sqrt(d)))  # the oracle takes the fp32 scale, widened
     ref = oracle.decode(q, kc, vc, tables, cl, scale, softcap=softcap, window=window)
     for b, L in enumerate(lens):
         s0 = L - window if window and L > window else 0
@@ -483,3 +483,39 @@ def test_split_k_merge_rule_reproduces_the_unsplit_definition(P, softcap, window
                 two = [_partial_log2(qv, k[s0:c], v[s0:c], scale, softcap),
                        _partial_log2(qv, k[c:L], v[c:L], scale, softcap)]
                 assert np.max(np.abs(_merge(two) - ref[b, h])) <= 1e-12
+
+
+@pytest.mark.parametrize("tile", [64, 128])
+def test_lazy_rescaled_online_softmax_is_exact(tile):
+    """The prefill softmax's lazy rescaling: the reference maximum moves only
+    when a tile's maximum exceeds it by more than 8 (log2 units), so every
+    weight stays <= 2^8, and since the sum and the output share the
+    reference the result is the exact softmax (fp64 simulation of the tile
+    loop against the oracle's two-pass definition)."""
+    gen = torch.Generator().manual_seed(77)
+    L, hq, hkv, d = 700, 4, 1, 32
+    ks, vs = _rand_seqs(gen, [L], hkv, d)
+    # growing scores along the sequence, so the reference has to move several times
+    ks[0] = ks[0] * torch.linspace(0.2, 3.0, L).view(L, 1, 1)
+    q = torch.randn((1, hq, d), generator=gen) * 2
+    kc, vc, tables, cl = scatter_to_pool(ks, vs, 16, gen)
+    scale = float(np.float32(1 / math.sqrt(d)))  # the oracle takes the fp32 scale, widened
+    ref = oracle.decode(q, kc, vc, tables, cl, scale)
+    k = ks[0][:, 0].double().numpy()
+    v = vs[0][:, 0].double().numpy()
+    for h in range(hq):
+        s = (k @ q[0, h].double().numpy()) * scale * math.log2(math.e)
+        m, l, o, moves = -math.inf, 0.0, np.zeros(d), 0
+        for t0 in range(0, L, tile):
+            st = s[t0 : t0 + tile]
+            mt = st.max()
+            mn = mt if (m == -math.inf or mt > m + 8) else m
+            moves += mn != m
+            alpha = 2.0 ** (m - mn) if m != -math.inf else 0.0
+            w = np.exp2(st - mn)
+            assert w.max() <= 2.0 ** 8
+            l = l * alpha + w.sum()
+            o = o * alpha + w @ v[t0 : t0 + tile]
+            m = mn
+        assert moves >= 2
+        assert np.max(np.abs(o / l - ref[0, h])) <= 1e-12
