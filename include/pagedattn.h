@@ -314,12 +314,19 @@ size_t pa_decode_cascade_workspace_size(int32_t batch, int32_t num_q_heads, int3
  *   (pa_decode_splitk_workspace_size() > PA_NOALLOC_SCRATCH_BYTES); such calls
  *   must use pa_decode_splitk with a workspace of their own.
  *   The first call on a device looks up the array's device address (no
- *   allocation); make that first call before any stream capture.  Every call
- *   uses the same array, and it keeps what the last call left in it: the call
- *   clears the part that must start at zero itself (the dynamic schedule's
- *   counters) with an asynchronous memset on `stream`.  Calls whose executions
- *   overlap on the GPU (different streams, or different host threads without
- *   ordering) race on the array and give wrong results; order them.
+ *   allocation; it may load the library's module on that device): make that
+ *   first call before any stream capture.  The address is looked up again
+ *   whenever the device's context has changed since (after a
+ *   cudaDeviceReset), so the call stays valid across a reset; the first call
+ *   after a reset is again a first call.  Any device ordinal is served.
+ *   Every call uses the same array, and it keeps what the last call left in
+ *   it: when the dynamic schedule runs (partition_tokens == 0 on the
+ *   tensor-core path), the call first clears the part of the array that must
+ *   start at zero (the schedule's counters, at its start) with an
+ *   asynchronous memset on `stream`; a call rejected by a host check touches
+ *   neither the device nor the array.  Calls whose executions overlap on the
+ *   GPU (different streams, or different host threads without ordering) race
+ *   on the array and give wrong results; order them.
  *   It allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
  */
 #define PA_NOALLOC_SCRATCH_BYTES (16u << 20) /* 16 MiB */

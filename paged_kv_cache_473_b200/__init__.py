@@ -2,7 +2,9 @@
 
 The compute lives in ``libpagedattn.so`` (C ABI, include/pagedattn.h); this
 package is its Python binding plus seeded synthetic batch generators
-(``workloads``) and the in-tree build step (``build``).
+(``workloads``) and the in-tree build step (``build``).  The library is opened
+on the first call into it (or the first read of ``lib``), so importing the
+package, or only its input generators, maps no GPU code.
 """
 
 from ._binding import (  # noqa: F401
@@ -29,10 +31,18 @@ from ._binding import (  # noqa: F401
     device_errors,
     error_string,
     last_launch_count,
-    lib,
     prefill,
     write_kv,
 )
+
+
+def __getattr__(name):  # ``lib``: the opened library, resolved on first use
+    if name == "lib":
+        from . import _binding
+
+        return _binding.lib
+    raise AttributeError(f"module {__name__!r} has no attribute {name!r}")
+
 
 __all__ = [
     "BlockManager",

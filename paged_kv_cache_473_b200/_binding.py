@@ -5,6 +5,10 @@ stream go to the C ABI; every step of the computation runs in the library's
 kernels.  torch provides device memory (the optional ``out`` tensors and the
 split-K workspace) and streams.  The binding refuses to run if the library is
 missing or cannot be built; there is no fallback path.
+
+The library is opened on first use (the first call, or the first read of
+``lib``), not at import, so that importing the package for its input
+generators (``workloads``) maps no GPU code.
 """
 
 from __future__ import annotations
@@ -111,11 +115,25 @@ def _load_library() -> ctypes.CDLL:
     return lib
 
 
-lib = _load_library()
+_lib_handle: Optional[ctypes.CDLL] = None
+
+
+def _lib() -> ctypes.CDLL:
+    """The opened library (opened, and built if stale, on first use)."""
+    global _lib_handle
+    if _lib_handle is None:
+        _lib_handle = _load_library()
+    return _lib_handle
+
+
+def __getattr__(name):  # module attribute ``lib``, resolved on first use
+    if name == "lib":
+        return _lib()
+    raise AttributeError(f"module {__name__!r} has no attribute {name!r}")
 
 
 def error_string(status: int) -> str:
-    return lib.pa_error_string(int(status)).decode()
+    return _lib().pa_error_string(int(status)).decode()
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -149,7 +167,7 @@ def write_kv(k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor, k_cac
              v_cache: torch.Tensor, stream=None) -> None:
     """Append ``k``/``v`` rows ``[N, Hkv, D]`` into the caches at ``slot_mapping`` (int64)."""
     nb, hkv, bs, d = k_cache.shape
-    st = lib.pa_write_kv(_ptr(k), _ptr(v), _ptr(slot_mapping), slot_mapping.numel(), _ptr(k_cache), _ptr(v_cache),
+    st = _lib().pa_write_kv(_ptr(k), _ptr(v), _ptr(slot_mapping), slot_mapping.numel(), _ptr(k_cache), _ptr(v_cache),
                          nb, bs, hkv, d, _dtype_code(k_cache), _stream(stream))
     _check(st, "pa_write_kv")
 
@@ -167,7 +185,7 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_
            out: Optional[torch.Tensor] = None, kernel: str = "auto", stream=None) -> torch.Tensor:
     """Paged decode attention, one CTA per (sequence, kv head).  Returns ``out``."""
     B, hq, d, nb, hkv, bs, out = _decode_common(q, k_cache, block_tables, out)
-    st = lib.pa_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens), B, hq, hkv, d,
+    st = _lib().pa_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens), B, hq, hkv, d,
                        bs, block_tables.shape[1], nb, float(scale), float(softcap), int(window), _ptr(out),
                        _dtype_code(q), KERNELS[kernel], _stream(stream))
     _check(st, "pa_decode")
@@ -175,12 +193,12 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, block_
 
 
 def decode_splitk_partition(batch: int, num_kv_heads: int, max_context_len: int, partition_tokens: int = 0) -> int:
-    return lib.pa_decode_splitk_partition(batch, num_kv_heads, max_context_len, partition_tokens)
+    return _lib().pa_decode_splitk_partition(batch, num_kv_heads, max_context_len, partition_tokens)
 
 
 def decode_splitk_workspace_size(batch: int, num_q_heads: int, head_dim: int, max_context_len: int,
                                  partition_tokens: int = 0, num_kv_heads: int = 1) -> int:
-    return lib.pa_decode_splitk_workspace_size(batch, num_q_heads, head_dim, max_context_len, partition_tokens,
+    return _lib().pa_decode_splitk_workspace_size(batch, num_q_heads, head_dim, max_context_len, partition_tokens,
                                                num_kv_heads)
 
 
@@ -197,11 +215,11 @@ def decode_splitk(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
     given.
     """
     B, hq, d, nb, hkv, bs, out = _decode_common(q, k_cache, block_tables, out)
-    need = decode_splitk_workspace_size(B, hq, d, max_context_len, partition_tokens, hkv)
-    if workspace is None:
+    if workspace is None:  # (a given workspace's size is checked by the library)
+        need = decode_splitk_workspace_size(B, hq, d, max_context_len, partition_tokens, hkv)
         workspace = torch.zeros(max(need, 16), dtype=torch.uint8, device=q.device)
     wbytes = workspace.numel() * workspace.element_size()
-    st = lib.pa_decode_splitk(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens), B, hq,
+    st = _lib().pa_decode_splitk(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens), B, hq,
                               hkv, d, bs, block_tables.shape[1], nb, float(scale), float(softcap), int(window),
                               _ptr(out), _dtype_code(q), int(partition_tokens), int(max_context_len),
                               _ptr(workspace), wbytes, KERNELS[kernel], _stream(stream))
@@ -211,7 +229,7 @@ def decode_splitk(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
 
 def decode_cascade_workspace_size(batch: int, num_q_heads: int, head_dim: int, max_context_len: int,
                                   prefix_len: int, partition_tokens: int = 0, num_kv_heads: int = 1) -> int:
-    return lib.pa_decode_cascade_workspace_size(batch, num_q_heads, head_dim, max_context_len, prefix_len,
+    return _lib().pa_decode_cascade_workspace_size(batch, num_q_heads, head_dim, max_context_len, prefix_len,
                                                 partition_tokens, num_kv_heads)
 
 
@@ -228,7 +246,7 @@ def decode_cascade(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
     if workspace is None:
         workspace = torch.zeros(max(need, 16), dtype=torch.uint8, device=q.device)
     wbytes = workspace.numel() * workspace.element_size()
-    st = lib.pa_decode_cascade(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens), B, hq,
+    st = _lib().pa_decode_cascade(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens), B, hq,
                                hkv, d, bs, block_tables.shape[1], nb, float(scale), float(softcap), int(window),
                                _ptr(out), _dtype_code(q), int(n_sharers), int(prefix_len), int(partition_tokens),
                                int(max_context_len), _ptr(workspace), wbytes, _stream(stream))
@@ -254,11 +272,11 @@ def decode_step(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, k_cac
     if split:
         if max_context_len <= 0:
             raise ValueError("decode_step(split=True) needs max_context_len")
-        need = decode_splitk_workspace_size(B, hq, d, max_context_len, partition_tokens, hkv)
-        if workspace is None:
+        if workspace is None:  # (a given workspace's size is checked by the library)
+            need = decode_splitk_workspace_size(B, hq, d, max_context_len, partition_tokens, hkv)
             workspace = torch.zeros(max(need, 16), dtype=torch.uint8, device=q.device)
         wptr, wbytes = _ptr(workspace), workspace.numel() * workspace.element_size()
-    st = lib.pa_decode_step(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+    st = _lib().pa_decode_step(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
                             _ptr(context_lens), B, hq, hkv, d, bs, block_tables.shape[1], nb, float(scale),
                             float(softcap), int(window), _ptr(out), _dtype_code(q), ptoks, int(max_context_len), wptr,
                             wbytes, KERNELS[kernel], _stream(stream))
@@ -268,7 +286,7 @@ def decode_step(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, k_cac
 
 def decode_multi_workspace_size(batch: int, q_len: int, num_q_heads: int, head_dim: int, max_context_len: int,
                                 partition_tokens: int = 0, num_kv_heads: int = 1) -> int:
-    return lib.pa_decode_multi_workspace_size(batch, q_len, num_q_heads, head_dim, max_context_len, partition_tokens,
+    return _lib().pa_decode_multi_workspace_size(batch, q_len, num_q_heads, head_dim, max_context_len, partition_tokens,
                                               num_kv_heads)
 
 
@@ -297,7 +315,7 @@ def decode_multi(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, 
         if workspace is None:
             workspace = torch.zeros(max(need, 16), dtype=torch.uint8, device=q.device)
         wptr, wbytes = _ptr(workspace), workspace.numel() * workspace.element_size()
-    st = lib.pa_decode_multi(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens), B, T, hq,
+    st = _lib().pa_decode_multi(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens), B, T, hq,
                              hkv, d, bs, block_tables.shape[1], nb, float(scale), float(softcap), int(window),
                              _ptr(out), _dtype_code(q), ptoks, int(max_context_len), wptr, wbytes, _stream(stream))
     _check(st, "pa_decode_multi")
@@ -317,7 +335,7 @@ def prefill(q: torch.Tensor, k_new: Optional[torch.Tensor], v_new: Optional[torc
     nb, hkv, bs, _ = k_cache.shape
     if out is None:
         out = torch.empty_like(q)
-    st = lib.pa_prefill(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(slot_mapping), _ptr(cu_q_lens), total,
+    st = _lib().pa_prefill(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(slot_mapping), _ptr(cu_q_lens), total,
                         int(max_q_len), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
                         cu_q_lens.numel() - 1, hq, hkv, d, bs, block_tables.shape[1], nb, float(scale),
                         float(softcap), int(window), _ptr(out), _dtype_code(q), _stream(stream))
@@ -330,7 +348,7 @@ def copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, pairs: torch.Tenso
     ``[n, 2]`` tensor of (src, dst) block ids (copy-on-write)."""
     nb, hkv, bs, d = k_cache.shape
     pairs = pairs.to(torch.int32).contiguous()
-    st = lib.pa_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(pairs), pairs.shape[0], nb, bs, hkv, d,
+    st = _lib().pa_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(pairs), pairs.shape[0], nb, bs, hkv, d,
                             _dtype_code(k_cache), _stream(stream))
     _check(st, "pa_copy_blocks")
 
@@ -347,14 +365,14 @@ class BlockManager:
     carried out on the GPU with :func:`copy_blocks`."""
 
     def __init__(self, num_blocks: int, block_size: int):
-        self._h = lib.pa_bm_create(int(num_blocks), int(block_size))
+        self._h = _lib().pa_bm_create(int(num_blocks), int(block_size))
         if not self._h:
             raise PagedAttnError(PA_ERR_INVALID, "pa_bm_create")
         self.num_blocks, self.block_size = int(num_blocks), int(block_size)
 
     def close(self) -> None:
         if self._h:
-            lib.pa_bm_destroy(self._h)
+            _lib().pa_bm_destroy(self._h)
             self._h = None
 
     def __del__(self):
@@ -365,11 +383,11 @@ class BlockManager:
 
     @property
     def num_free(self) -> int:
-        return lib.pa_bm_num_free(self._h)
+        return _lib().pa_bm_num_free(self._h)
 
     def blocks_needed(self, num_tokens: int, token_ids=None) -> int:
         arr = _i64_array(token_ids)[0] if token_ids is not None else None
-        return lib.pa_bm_blocks_needed(self._h, arr, int(num_tokens))
+        return _lib().pa_bm_blocks_needed(self._h, arr, int(num_tokens))
 
     def add_sequence(self, seq_id: int, num_tokens: int, token_ids=None) -> int:
         """Register a prompt; returns how many leading positions came from the prefix cache."""
@@ -379,7 +397,7 @@ class BlockManager:
             if n != num_tokens:
                 raise ValueError("token_ids must hold num_tokens ids")
         cached = ctypes.c_int32(0)
-        _check(lib.pa_bm_add_sequence(self._h, int(seq_id), arr, int(num_tokens), ctypes.byref(cached)),
+        _check(_lib().pa_bm_add_sequence(self._h, int(seq_id), arr, int(num_tokens), ctypes.byref(cached)),
                "pa_bm_add_sequence")
         return cached.value
 
@@ -390,39 +408,40 @@ class BlockManager:
         slots = (ctypes.c_int64 * max(1, n))()
         cow = (ctypes.c_int32 * max(2, 2 * n))()
         ncow = ctypes.c_int32(0)
-        _check(lib.pa_bm_append_slots(self._h, ids, toks, n, slots, cow, ctypes.byref(ncow)), "pa_bm_append_slots")
+        _check(_lib().pa_bm_append_slots(self._h, ids, toks, n, slots, cow, ctypes.byref(ncow)), "pa_bm_append_slots")
         k = ncow.value
         return (torch.tensor(list(slots)[:n], dtype=torch.int64),
                 torch.tensor(list(cow)[: 2 * k], dtype=torch.int32).reshape(k, 2))
 
     def fork(self, parent_id: int, child_id: int) -> None:
-        _check(lib.pa_bm_fork(self._h, int(parent_id), int(child_id)), "pa_bm_fork")
+        _check(_lib().pa_bm_fork(self._h, int(parent_id), int(child_id)), "pa_bm_fork")
 
     def free(self, seq_id: int) -> None:
-        _check(lib.pa_bm_free_sequence(self._h, int(seq_id)), "pa_bm_free_sequence")
+        _check(_lib().pa_bm_free_sequence(self._h, int(seq_id)), "pa_bm_free_sequence")
 
     def length(self, seq_id: int) -> int:
-        return lib.pa_bm_length(self._h, int(seq_id))
+        return _lib().pa_bm_length(self._h, int(seq_id))
 
     def block_tables(self, seq_ids, max_blocks: int):
         """(tables int32 [n, max_blocks], -1 padded; context_lens int32 [n]) on the host."""
         ids, n = _i64_array(seq_ids)
         tables = torch.empty((n, int(max_blocks)), dtype=torch.int32)
         lens = torch.empty((n,), dtype=torch.int32)
-        _check(lib.pa_bm_block_tables(self._h, ids, n, int(max_blocks), tables.data_ptr(), lens.data_ptr()),
+        _check(_lib().pa_bm_block_tables(self._h, ids, n, int(max_blocks), tables.data_ptr(), lens.data_ptr()),
                "pa_bm_block_tables")
         return tables, lens
 
     def slots(self, seq_id: int, start: int, count: int) -> torch.Tensor:
         out = torch.empty((int(count),), dtype=torch.int64)
-        _check(lib.pa_bm_slots(self._h, int(seq_id), int(start), int(count), out.data_ptr() if count else None),
+        _check(_lib().pa_bm_slots(self._h, int(seq_id), int(start), int(count), out.data_ptr() if count else None),
                "pa_bm_slots")
         return out
 
     def ref_count(self, block: int) -> int:
-        return lib.pa_bm_ref_count(self._h, int(block))
+        return _lib().pa_bm_ref_count(self._h, int(block))
 
 
+# PA_NOALLOC_SCRATCH_BYTES of include/pagedattn.h (a CPU test checks that the two agree).
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -434,7 +453,7 @@ def decode_splitk_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch
     split-K scratch is the library's own fixed array, and ``out`` must be given.
     Calls must not overlap on the GPU (they share that array)."""
     B, hq, d, nb, hkv, bs, out = _decode_common(q, k_cache, block_tables, out)
-    st = lib.pa_decode_splitk_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
+    st = _lib().pa_decode_splitk_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
                                       B, hq, hkv, d, bs, block_tables.shape[1], nb, float(scale), float(softcap),
                                       int(window), _ptr(out), _dtype_code(q), int(partition_tokens),
                                       int(max_context_len), KERNELS[kernel], _stream(stream))
@@ -445,15 +464,15 @@ def decode_splitk_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch
 def device_errors(clear: bool = True) -> int:
     """OR of the PA_DEVERR_* bits raised on the current device (synchronises)."""
     bits = ctypes.c_uint32(0)
-    _check(lib.pa_device_errors(ctypes.byref(bits), 1 if clear else 0), "pa_device_errors")
+    _check(_lib().pa_device_errors(ctypes.byref(bits), 1 if clear else 0), "pa_device_errors")
     return bits.value
 
 
 def check_bounded_wait(limit_ns: int = 1_000_000, stream=None) -> None:
     """Launch the bounded-wait check (a wait nothing completes, given up after
     ``limit_ns``); read the resulting PA_DEVERR_TIMEOUT with device_errors()."""
-    _check(lib.pa_check_bounded_wait(int(limit_ns), _stream(stream)), "pa_check_bounded_wait")
+    _check(_lib().pa_check_bounded_wait(int(limit_ns), _stream(stream)), "pa_check_bounded_wait")
 
 
 def last_launch_count() -> int:
-    return lib.pa_last_launch_count()
+    return _lib().pa_last_launch_count()

@@ -11,6 +11,7 @@
 #include <mutex>
 #include <algorithm>
 #include <utility>
+#include <vector>
 
 #include "../../include/pagedattn.h"
 #include "../../include/block_manager.h"
@@ -74,6 +75,42 @@ bool encode_cache_map(CUtensorMap* map, const void* base, int head_dim, long lon
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// Tensor maps of the K and V caches, encoded once per (base addresses, rows,
+// head_dim) and reused: a map holds only the address, the shape and the fixed
+// box / swizzle, so a cached one is exactly what a fresh encode would give.
+// A small per-thread table (no lock); the oldest entry is replaced.
+bool cache_maps(const void* kbase, const void* vbase, int head_dim, long long rows, CUtensorMap* kmap,
+                CUtensorMap* vmap) {
+  struct Entry {
+    const void* k;
+    const void* v;
+    long long rows;
+    int d;
+    CUtensorMap kmap, vmap;
+  };
+  constexpr int kEntries = 8;
+  thread_local Entry table[kEntries] = {};
+  thread_local int next = 0;
+  for (const Entry& e : table) {
+    if (e.k == kbase && e.v == vbase && e.rows == rows && e.d == head_dim && kbase) {
+      *kmap = e.kmap;
+      *vmap = e.vmap;
+      return true;
+    }
+  }
+  if (!tensor_map_encoder()) return false;
+  if (!encode_cache_map(kmap, kbase, head_dim, rows) || !encode_cache_map(vmap, vbase, head_dim, rows)) return false;
+  Entry& e = table[next];
+  next = (next + 1) % kEntries;
+  e.k = kbase;
+  e.v = vbase;
+  e.rows = rows;
+  e.d = head_dim;
+  e.kmap = *kmap;
+  e.vmap = *vmap;
+  return true;
 }
 
 // ---- argument checks -------------------------------------------------------------
@@ -179,9 +216,7 @@ cudaError_t launch_mma_t(const DecodeParams& p, dim3 grid, cudaStream_t st) {
   using Cfg = pa::MmaCfg<D, NW, ST>;
   CUtensorMap kmap, vmap;
   const long long rows = (long long)p.num_blocks * p.hkv * p.block_size;
-  if (!tensor_map_encoder()) return cudaErrorNotSupported;
-  if (!encode_cache_map(&kmap, p.k_cache, D, rows) || !encode_cache_map(&vmap, p.v_cache, D, rows))
-    return cudaErrorInvalidValue;
+  if (!cache_maps(p.k_cache, p.v_cache, D, rows, &kmap, &vmap)) return cudaErrorInvalidValue;
   auto kern = pa::decode_mma_kernel<D, NW, ST, SPLIT, APPEND>;
   static std::atomic<uint64_t> smem_done{0};
   cudaError_t e = set_smem(kern, Cfg::kSmemBytes, smem_done);
@@ -208,9 +243,7 @@ cudaError_t launch_prefill_t(const DecodeParams& p, dim3 grid, cudaStream_t st) 
   using Cfg = pa::PrefillCfg<D>;
   CUtensorMap kmap, vmap;
   const long long rows = (long long)p.num_blocks * p.hkv * p.block_size;
-  if (!tensor_map_encoder()) return cudaErrorNotSupported;
-  if (!encode_cache_map(&kmap, p.k_cache, D, rows) || !encode_cache_map(&vmap, p.v_cache, D, rows))
-    return cudaErrorInvalidValue;
+  if (!cache_maps(p.k_cache, p.v_cache, D, rows, &kmap, &vmap)) return cudaErrorInvalidValue;
   auto kern = pa::prefill_umma_kernel<D>;
   static std::atomic<uint64_t> smem_done{0};
   cudaError_t e = set_smem(kern, Cfg::kSmemBytes, smem_done);
@@ -239,9 +272,7 @@ cudaError_t launch_multi_t(const DecodeParams& p, dim3 grid, int warps, cudaStre
   using Cfg = pa::MultiCfg<D, ST>;
   CUtensorMap kmap, vmap;
   const long long rows = (long long)p.num_blocks * p.hkv * p.block_size;
-  if (!tensor_map_encoder()) return cudaErrorNotSupported;
-  if (!encode_cache_map(&kmap, p.k_cache, D, rows) || !encode_cache_map(&vmap, p.v_cache, D, rows))
-    return cudaErrorInvalidValue;
+  if (!cache_maps(p.k_cache, p.v_cache, D, rows, &kmap, &vmap)) return cudaErrorInvalidValue;
   auto kern = pa::decode_multi_kernel<D, ST, SPLIT>;
   static std::atomic<uint64_t> smem_done{0};
   cudaError_t e = set_smem(kern, Cfg::kSmemBytes, smem_done);
@@ -359,6 +390,27 @@ cudaError_t set_smem_at_least(Kernel k, int bytes, std::atomic<int>* done /* [64
   return e;
 }
 
+// Resident CTAs per SM of `kern` at `threads` x `smem`, on the current device:
+// queried once per (kernel, shared-memory size, device) and remembered (one
+// entry per device for each kernel instantiation; `cache` is that kernel's).
+template <typename Kernel>
+cudaError_t occupancy(Kernel kern, int threads, int smem, std::atomic<long long>* cache /* [64] */, int* occ) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 64) {
+    const long long v = cache[dev].load(std::memory_order_acquire);
+    if (v > 0 && (v >> 16) == smem) {
+      *occ = (int)(v & 0xffff);
+      return cudaSuccess;
+    }
+  }
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(occ, kern, threads, smem);
+  if (e == cudaSuccess && dev < 64 && *occ > 0 && *occ < 0x10000)
+    cache[dev].store(((long long)smem << 16) | *occ, std::memory_order_release);
+  return e;
+}
+
 // Launch the dynamic schedule with the persistent grid (as many CTAs as are
 // resident at once).  Sets p.merge_in_kernel: the partitions of each unit are
 // merged in-kernel when the step is small next to the resident warps (at most
@@ -372,16 +424,15 @@ cudaError_t launch_dynamic_t(DecodeParams& p, cudaStream_t st, bool pdl, bool al
   using Cfg = pa::DynCfg<D, NW, ST>;
   CUtensorMap kmap, vmap;
   const long long rows = (long long)p.num_blocks * p.hkv * p.block_size;
-  if (!tensor_map_encoder()) return cudaErrorNotSupported;
-  if (!encode_cache_map(&kmap, p.k_cache, D, rows) || !encode_cache_map(&vmap, p.v_cache, D, rows))
-    return cudaErrorInvalidValue;
+  if (!cache_maps(p.k_cache, p.v_cache, D, rows, &kmap, &vmap)) return cudaErrorInvalidValue;
   auto kern = pa::decode_dynamic_kernel<D, NW, ST, APPEND, CASCADE>;
   const int smem = Cfg::smem_bytes(p.batch);
   static std::atomic<int> smem_done[64];
   cudaError_t e = set_smem_at_least(kern, smem, smem_done);
   if (e != cudaSuccess) return e;
   int occ = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, Cfg::kThreads, smem);
+  static std::atomic<long long> occ_cache[64];
+  e = occupancy(kern, Cfg::kThreads, smem, occ_cache, &occ);
   if (e != cudaSuccess) return e;
   if (occ < 1) return cudaErrorInvalidConfiguration;
   const int grid = occ * sm_count();
@@ -416,16 +467,15 @@ cudaError_t launch_rows_t(DecodeParams& p, cudaStream_t st) {
   using Cfg = pa::DynCfg<D, NW, ST>;
   CUtensorMap kmap, vmap;
   const long long rows = (long long)p.num_blocks * p.hkv * p.block_size;
-  if (!tensor_map_encoder()) return cudaErrorNotSupported;
-  if (!encode_cache_map(&kmap, p.k_cache, D, rows) || !encode_cache_map(&vmap, p.v_cache, D, rows))
-    return cudaErrorInvalidValue;
+  if (!cache_maps(p.k_cache, p.v_cache, D, rows, &kmap, &vmap)) return cudaErrorInvalidValue;
   auto kern = pa::decode_rows_kernel<D, NW, ST>;
   const int smem = Cfg::smem_bytes(p.batch);
   static std::atomic<int> smem_done[64];
   cudaError_t e = set_smem_at_least(kern, smem, smem_done);
   if (e != cudaSuccess) return e;
   int occ = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, Cfg::kThreads, smem);
+  static std::atomic<long long> occ_cache[64];
+  e = occupancy(kern, Cfg::kThreads, smem, occ_cache, &occ);
   if (e != cudaSuccess) return e;
   if (occ < 1) return cudaErrorInvalidConfiguration;
   p.merge_in_kernel = 0;
@@ -491,6 +541,74 @@ size_t dynamic_counter_bytes(int32_t batch, int32_t num_kv_heads) {
   return (2 + (size_t)batch * num_kv_heads) * sizeof(int);
 }
 
+// ---- the allocation-free call's scratch ---------------------------------------------
+
+// Split-K scratch of pa_decode_splitk_noalloc: reserved in device memory by the
+// module itself on every device that loads the library, so that call allocates
+// nothing.  In host code the name is a host-side stand-in, not a device
+// address; noalloc_scratch() asks the runtime for the device address.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PA_NOALLOC_SCRATCH_BYTES];
+
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
+PFN_cuCtxGetId_v12000 g_ctx_get_id = nullptr;
+std::once_flag g_ctx_once;
+
+// Unique id of the calling thread's current context, or 0 when no context is
+// current (or the driver cannot tell).
+unsigned long long current_context_id() {
+  std::call_once(g_ctx_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &fn, 4000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+    fn = nullptr;
+    q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &fn, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(fn);
+  });
+  if (!g_ctx_current || !g_ctx_get_id) return 0;
+  CUcontext ctx = nullptr;
+  if (g_ctx_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+  unsigned long long id = 0;
+  return g_ctx_get_id(ctx, &id) == CUDA_SUCCESS ? id : 0;
+}
+
+// Device address of g_noalloc_scratch in the current device's context, or null
+// when the runtime cannot give it.  The lookup allocates nothing; it runs on
+// the first call on a device and again whenever that device's context has
+// changed since (a cudaDeviceReset unloads the module, and the array is placed
+// anew when the library is next used), so no stale address is ever handed to
+// a kernel.  Any device ordinal is served.
+void* noalloc_scratch() {
+  struct Entry {
+    int dev;
+    unsigned long long ctx;  // 0: unknown, look the address up again
+    void* addr;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  Entry* e = nullptr;
+  for (auto& x : cache)
+    if (x.dev == dev) e = &x;
+  const unsigned long long ctx = current_context_id();
+  if (e && ctx != 0 && e->ctx == ctx) return e->addr;
+  void* a = nullptr;
+  if (cudaGetSymbolAddress(&a, g_noalloc_scratch) != cudaSuccess || !a) return nullptr;
+  const unsigned long long now = current_context_id();  // the lookup may have made the context current
+  if (e) {
+    e->ctx = now;
+    e->addr = a;
+  } else {
+    cache.push_back(Entry{dev, now, a});
+  }
+  return a;
+}
+
 // Everything the decode entry points share.  split: partitioned launch plus
 // the combine; append: the fused decode step (k_new / v_new appended at L-1).
 struct DecodeCall {
@@ -510,6 +628,7 @@ struct DecodeCall {
   int32_t partition_tokens, max_context_len;
   void* workspace;
   size_t workspace_bytes;
+  bool noalloc;  // split-K scratch is the library's own array (workspace ignored)
   pa_kernel_t kernel;
   cudaStream_t stream;
 };
@@ -536,10 +655,18 @@ pa_status_t run_decode(const DecodeCall& c) {
     parts = splitk_parts(c.max_context_len, P);
     if (parts > kMaxPartsPerSeq) return PA_ERR_UNSUPPORTED;
     const size_t need = workspace_size(s.batch, s.hq, s.d, c.max_context_len, P);
-    if (s.batch > 0 && (!c.workspace || !aligned(c.workspace, 16) || c.workspace_bytes < need))
+    if (c.noalloc) {
+      if (need > PA_NOALLOC_SCRATCH_BYTES) return PA_ERR_WORKSPACE;
+    } else if (s.batch > 0 && (!c.workspace || !aligned(c.workspace, 16) || c.workspace_bytes < need)) {
       return PA_ERR_WORKSPACE;
+    }
   }
   if (s.batch == 0) return PA_OK;
+  void* workspace = c.workspace;
+  if (c.split && c.noalloc) {  // every host check has passed: only now touch the device
+    workspace = noalloc_scratch();
+    if (!workspace) return PA_ERR_CUDA;
+  }
 
   DecodeParams p = make_params(c.q, c.k_cache, c.v_cache, c.block_tables, c.context_lens, s, c.scale, c.softcap,
                                c.window, c.out);
@@ -551,10 +678,17 @@ pa_status_t run_decode(const DecodeCall& c) {
     p.max_parts = (int)parts;
     p.max_context = c.max_context_len < p.max_context ? c.max_context_len : p.max_context;
     const size_t rows = (size_t)s.batch * s.hq * parts;
-    char* ws = static_cast<char*>(c.workspace);
+    char* ws = static_cast<char*>(workspace);
     p.ws_o = reinterpret_cast<float*>(ws + pa::kCounterBytes);
     p.ws_ml = reinterpret_cast<float*>(ws + pa::kCounterBytes + align256(rows * s.d * 4));
     if (dynamic) {  // resets its counters itself; merges in-kernel or through the combine
+      if (c.noalloc) {
+        // The shared array keeps what the last call left in it.  A call that
+        // completed left the counters (the start of the array) at zero, one
+        // that timed out may not have: clear the ones this call uses.
+        const size_t len = std::min(dynamic_counter_bytes(s.batch, s.hkv), pa::kCounterBytes);
+        if (cudaMemsetAsync(ws, 0, len, c.stream) != cudaSuccess) return PA_ERR_CUDA;
+      }
       p.queue = reinterpret_cast<int*>(ws);
       p.unit_count = p.queue + 2;
       e = c.append ? launch_dynamic<true>(p, c.stream) : launch_dynamic<false>(p, c.stream);
@@ -959,36 +1093,6 @@ size_t pa_decode_multi_workspace_size(int32_t batch, int32_t q_len, int32_t num_
   return workspace_size(batch, num_q_heads, head_dim, max_context_len, P, q_len);
 }
 
-}  // extern "C"
-
-namespace {
-
-// Split-K scratch of pa_decode_splitk_noalloc: reserved in device memory by the
-// module itself, so that call allocates nothing.  Host code must not use the
-// symbol as an address; it asks the runtime for the device address once per
-// device (noalloc_scratch).
-static __device__ __align__(256) unsigned char g_noalloc_scratch[PA_NOALLOC_SCRATCH_BYTES];
-
-// Device address of g_noalloc_scratch on the current device (looked up on the
-// first call per device), or null when the lookup fails.
-void* noalloc_scratch() {
-  static std::mutex mu;
-  static void* addr[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
-    void* a = nullptr;
-    if (cudaGetSymbolAddress(&a, g_noalloc_scratch) != cudaSuccess) return nullptr;
-    addr[dev] = a;
-  }
-  return addr[dev];
-}
-
-}  // namespace
-
-extern "C" {
-
 pa_status_t pa_decode_splitk_noalloc(const void* q, const void* k_cache, const void* v_cache,
                                      const int32_t* block_tables, const int32_t* context_lens, int32_t batch,
                                      int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
@@ -997,23 +1101,31 @@ pa_status_t pa_decode_splitk_noalloc(const void* q, const void* k_cache, const v
                                      int32_t partition_tokens, int32_t max_context_len, pa_kernel_t kernel,
                                      pa_stream_t stream) {
   t_last_launches = 0;
+  // The documented limit: what pa_decode_splitk would ask of a caller's workspace.
   if (batch > 0 && num_q_heads > 0 && head_dim > 0 && max_context_len > 0 && partition_tokens >= 0) {
     const size_t need = pa_decode_splitk_workspace_size(batch, num_q_heads, head_dim, max_context_len,
                                                         partition_tokens, num_kv_heads);
     if (need > PA_NOALLOC_SCRATCH_BYTES) return PA_ERR_WORKSPACE;
   }
-  void* ws = noalloc_scratch();
-  if (!ws) return PA_ERR_CUDA;
-  // The array keeps the previous call's contents; the dynamic schedule's
-  // counters (after its partials) must start at zero.  A call that completes
-  // leaves them at zero, one that timed out may not: clear them every call.
-  if (partition_tokens == 0 && batch > 0 && num_kv_heads > 0) {
-    const size_t len = std::min(dynamic_counter_bytes(batch, num_kv_heads), pa::kCounterBytes);
-    if (cudaMemsetAsync(ws, 0, len, stream) != cudaSuccess) return PA_ERR_CUDA;
-  }
-  return pa_decode_splitk(q, k_cache, v_cache, block_tables, context_lens, batch, num_q_heads, num_kv_heads,
-                          head_dim, block_size, max_blocks_per_seq, num_blocks, scale, softcap, window, out, dtype,
-                          partition_tokens, max_context_len, ws, PA_NOALLOC_SCRATCH_BYTES, kernel, stream);
+  DecodeCall c{};
+  c.q = q;
+  c.k_cache = k_cache;
+  c.v_cache = v_cache;
+  c.block_tables = block_tables;
+  c.context_lens = context_lens;
+  c.shape = Shape{batch, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks};
+  c.scale = scale;
+  c.softcap = softcap;
+  c.window = window;
+  c.out = out;
+  c.dtype = dtype;
+  c.split = true;
+  c.partition_tokens = partition_tokens;
+  c.max_context_len = max_context_len;
+  c.noalloc = true;  // the scratch is looked up, and its counters cleared, only once every check has passed
+  c.kernel = kernel;
+  c.stream = stream;
+  return run_decode(c);
 }
 
 pa_status_t pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs, int32_t n, int32_t num_blocks,

@@ -270,3 +270,62 @@ def test_bounded_wait_check_rejects_bad_limits():
     """pa_check_bounded_wait checks its bound before any launch (no GPU needed)."""
     assert bnd.lib.pa_check_bounded_wait(0, None) == bnd.PA_ERR_INVALID
     assert bnd.lib.pa_check_bounded_wait(2_000_000_000, None) == bnd.PA_ERR_INVALID
+
+
+def _noalloc(**kw):
+    a = dict(q=A, k=A, v=A, bt=A, cl=A, B=4, hq=32, hkv=8, d=128, bs=16, mb=4096, nb=1 << 14, out=A,
+             dt=bnd.PA_BF16, P=0, maxL=2048, kern=0)
+    a.update(kw)
+    return bnd.lib.pa_decode_splitk_noalloc(a["q"], a["k"], a["v"], a["bt"], a["cl"], a["B"], a["hq"], a["hkv"],
+                                            a["d"], a["bs"], a["mb"], a["nb"], 0.1, 0.0, 0, a["out"], a["dt"], a["P"],
+                                            a["maxL"], a["kern"], None)
+
+
+def test_noalloc_scratch_size_matches_the_header():
+    src = open(HEADER).read()
+    m = re.search(r"#define\s+PA_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", src)
+    assert m, "PA_NOALLOC_SCRATCH_BYTES not found in the header"
+    assert int(m.group(1)) << int(m.group(2)) == bnd.NOALLOC_SCRATCH_BYTES
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="fake pointers: CPU-only check")
+def test_noalloc_refuses_exactly_above_its_scratch_and_checks_before_touching_the_device():
+    """The refusal threshold is the header's size: the first context bound whose
+    split-K workspace exceeds it is refused (PA_ERR_WORKSPACE) before anything
+    else; the one below passes every host check and only then asks the runtime
+    for the scratch, which on a machine without a GPU fails (PA_ERR_CUDA).  A
+    call that fails a host check returns that check's status, so it touched
+    neither the device nor the scratch."""
+    B, hq, d, hkv = 4, 32, 128, 8
+    L = 64
+    while pa.decode_splitk_workspace_size(B, hq, d, L * 2, 0, hkv) <= bnd.NOALLOC_SCRATCH_BYTES:
+        L *= 2
+    lo, hi = L, L * 2  # need(lo) <= limit < need(hi): bisect to the first refused bound
+    while hi - lo > 1:
+        mid = (lo + hi) // 2
+        if pa.decode_splitk_workspace_size(B, hq, d, mid, 0, hkv) <= bnd.NOALLOC_SCRATCH_BYTES:
+            lo = mid
+        else:
+            hi = mid
+    mb = (hi + 15) // 16
+    assert _noalloc(maxL=hi, mb=mb) == bnd.PA_ERR_WORKSPACE
+    assert _noalloc(maxL=lo, mb=mb) == bnd.PA_ERR_CUDA
+    assert _noalloc(maxL=lo, mb=mb, q=None) == bnd.PA_ERR_INVALID
+    assert _noalloc(maxL=lo, mb=mb, d=96) == bnd.PA_ERR_UNSUPPORTED
+    assert _noalloc(maxL=2048, mb=128, P=100) == bnd.PA_ERR_INVALID  # not a multiple of 64
+
+
+def test_importing_the_package_maps_no_gpu_code():
+    """The package opens libpagedattn.so on first use, so a process that only
+    draws inputs (the benchmark's CPU-oracle arm) maps none of it."""
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = ("import sys; sys.path.insert(0, %r)\n"
+            "import paged_kv_cache_473_b200, paged_kv_cache_473_b200.workloads\n"
+            "maps = open('/proc/self/maps').read()\n"
+            "print('mapped' if 'libpagedattn' in maps else 'clean')\n" % root)
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.strip() == "clean"
