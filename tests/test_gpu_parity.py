@@ -261,6 +261,7 @@ def test_bad_block_id_and_long_context_are_reported_not_faulted():
 # ---- full sizes, bench launch configuration, sampled rows -----------------------
 
 FULL = ["tinyllama_1b", "gemma2_2b", "llama3_8b", "long_splitk"]
+COUNTER_BYTES = 256 * 1024  # the split-K workspace's fixed counter region
 
 
 @pytest.mark.parametrize("name", FULL)
@@ -320,7 +321,11 @@ def test_fused_step_with_window_and_softcap(window):
 
 
 @pytest.mark.parametrize("name", FULL)
-def test_full_size_fused_step_sampled_rows(name):
+def test_full_size_fused_step_grid_schedule_sampled_rows(name):
+    """The fused step on the fixed partition grid (the library's grid partition
+    for the shape, given explicitly), at full size, on sampled rows.  The
+    dynamic schedule that the benchmark times is compared on its whole output
+    below."""
     w = wl.WORKLOADS[name]
     b = wl.make_batch(w, device="cuda")
     cpu = dict(q=b.q.cpu(), k_new=b.k_new.cpu(), v_new=b.v_new.cpu(), slots=b.slot_mapping.cpu(),
@@ -348,6 +353,45 @@ def test_full_size_fused_step_sampled_rows(name):
                         rows=rows)
     got = torch.stack([out[i, h] for i, h in rows])
     assert_close(got, ref, w.torch_dtype, f"{name} full-size fused step")
+
+
+# ---- the benchmark's timed call, full size, whole output -----------------------------
+
+# (workload, partition argument of bench.Runner): -1 is the workload's own
+# schedule, the headline and per-shape lines of bench.py (the dynamic work
+# queue, or the 512-token grid for the long split-K shape); the long shape is
+# also timed on the dynamic schedule.
+BENCH_STEPS = [("tinyllama_1b", -1), ("gemma2_2b", -1), ("llama3_8b", -1), ("long_splitk", -1), ("long_splitk", 0)]
+
+
+@pytest.mark.parametrize("name,partition", BENCH_STEPS)
+def test_full_size_timed_step_whole_output(name, partition):
+    """The step bench.py times (bench.Runner.step: pa_decode_step with the
+    runner's schedule, workspace and max_context_len), at the full workload
+    size: every output element against the oracle (append, then decode),
+    the whole cache after the step bit-exact against the oracle's append, and
+    the workspace's counter region back at zero."""
+    import bench
+
+    w = wl.WORKLOADS[name]
+    runner = bench.Runner(w, 0, "auto", True, partition, fused=True)
+    b = runner.batch
+    cpu = {k: getattr(b, k).cpu() for k in ("q", "k_new", "v_new", "slot_mapping", "k_cache", "v_cache",
+                                            "block_tables", "context_lens")}
+    runner.step(0)
+    torch.cuda.synchronize()
+    assert pa.device_errors() == 0
+    if runner.partition == 0:
+        assert int(runner.ws[:COUNTER_BYTES].view(torch.int32).abs().sum()) == 0
+    oracle.write_kv(cpu["k_new"], cpu["v_new"], cpu["slot_mapping"], cpu["k_cache"], cpu["v_cache"])
+    kc, vc = runner.pools[0]
+    assert torch.equal(bits(kc), bits(cpu["k_cache"])), "key cache after the step"
+    assert torch.equal(bits(vc), bits(cpu["v_cache"])), "value cache after the step"
+    ref = oracle.decode(cpu["q"], cpu["k_cache"], cpu["v_cache"], cpu["block_tables"], cpu["context_lens"], w.scale,
+                        w.softcap, w.window)
+    assert_close(runner.out, ref, w.torch_dtype, f"{name} timed step (partition {runner.partition}), whole output")
+    del runner
+    torch.cuda.empty_cache()
 
 
 # ---- dynamic (work-queue) split-K schedule ------------------------------------------
@@ -453,9 +497,6 @@ def test_dynamic_schedule_counters_return_to_zero():
         outs.append(out)
     assert torch.equal(bits(outs[0]), bits(outs[3]))
     assert pa.device_errors() == 0
-
-
-COUNTER_BYTES = 256 * 1024  # the workspace's fixed counter region
 
 
 @pytest.mark.parametrize("name,kw", [
