@@ -45,6 +45,13 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # next launch, which on the 65 MB TinyLlama step alone costs ~8 us per step.
 EVENT_EVERY = 10
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+# The decode shapes whose line carries its own roofline, end-to-end figure and
+# CPU baselines beside the headline (the shapes the >= 70 % target names, and
+# the largest one).
+DATA = "synthetic (seeded; q/k/v ~ N(0,1), shuffled physical blocks, NaN canaries in dead slots)"
+TARGET_SHAPES = ("gemma2_2b", "llama3_8b", "long_splitk")
+L2_NOTE = ("L2 defeated: the timed steps rotate over copies of the KV pool totalling at least 4x the L2 size "
+           "(one copy when the pool alone is that large)")
 
 
 def parse():
@@ -528,9 +535,10 @@ def run_e2e(runner: Runner, K: int, world: int):
 
 class OracleSample:
     """The CPU oracle as it stands, timed on a bounded sample of one workload
-    (the batch is copied to host memory once, outside any timing)."""
+    (the batch is copied to host memory once, outside any timing), on
+    ``threads`` host threads (default: every core this process may run on)."""
 
-    def __init__(self, w: wl.Workload, batch: wl.Batch):
+    def __init__(self, w: wl.Workload, batch: wl.Batch, threads: int = 0):
         import oracle
 
         self.oracle = oracle
@@ -539,9 +547,17 @@ class OracleSample:
                         slots=batch.slot_mapping.cpu(), kc=batch.k_cache.cpu(), vc=batch.v_cache.cpu(),
                         tables=batch.block_tables.cpu(), lens=batch.context_lens.cpu())
         oracle.build()
-        self.threads = oracle.num_threads()
         c = self.cpu
         self.B, self.hq = c["q"].shape[0], c["q"].shape[1]
+        self.set_threads(threads)
+
+    def set_threads(self, threads: int = 0):
+        """Run on ``threads`` host threads (0: every core this process may run
+        on), and re-estimate one sequence's cost at that count."""
+        self.n_threads = threads if threads > 0 else len(os.sched_getaffinity(0))
+        self.oracle.set_num_threads(self.n_threads)
+        self.threads = self.oracle.num_threads()
+        c = self.cpu
         t0 = time.perf_counter()
         self._decode([(0, h) for h in range(self.hq)])
         el = time.perf_counter() - t0
@@ -556,6 +572,7 @@ class OracleSample:
         """Whole steps (append + decode of every sequence) until ``seconds`` of
         work have run, or one step over the first n sequences when a whole step
         would take longer than that."""
+        self.oracle.set_num_threads(self.n_threads)
         c = self.cpu
         B, hq = self.B, self.hq
         n_seq = B if self.per_seq * B <= seconds else max(1, int(seconds / self.per_seq))
@@ -576,27 +593,47 @@ class OracleSample:
                 "seconds": round(el, 3)}
 
 
-def describe(w: wl.Workload, runner: Runner, args, l2_note: str):
+def cpu_baselines(w: wl.Workload, batch: wl.Batch, seconds: float) -> dict:
+    """The oracle on every host core and on one core, each on a bounded sample."""
+    out = {}
+    sampler = OracleSample(w, batch)
+    for key, threads, secs in (("cpu_baseline", 0, seconds), ("cpu_baseline_1core", 1, seconds / 2)):
+        sampler.set_threads(threads)
+        info = sampler.run(secs)
+        info["value"] = round(info["value"], 2)
+        out[key] = info
+    sampler.set_threads(0)
+    return out
+
+
+def workload_config(w: wl.Workload, batch: wl.Batch) -> dict:
+    """The workload a line measures, as both arms (the library and the CPU
+    oracle) describe it: the same dict on both lines."""
     return {
         "workload": w.name,
-        "batch": runner.B,
+        "batch": int(batch.q.shape[0]),
         "num_q_heads": w.num_q_heads,
         "num_kv_heads": w.num_kv_heads,
         "head_dim": w.head_dim,
         "block_size": w.block_size,
         "lengths": list(w.lengths),
-        "mean_context": round(float(runner.batch.context_lens.double().mean()), 1),
+        "mean_context": round(float(batch.context_lens.double().mean()), 1),
         "softcap": w.softcap,
         "window": w.window,
         "prefix_share": w.prefix_share,
-        "path": ("pa_decode_step" if runner.fused else "pa_write_kv + " + ("pa_decode_splitk" if runner.split else
-                                                                          "pa_decode"))
-        + ((" (split-K, dynamic work queue)" if runner.partition == 0 else
-            f" (split-K, partition {runner.partition})") if runner.split else " (one CTA per sequence, kv head)"),
-        "kernel": args.kernel,
-        "l2": l2_note,
+        "l2": L2_NOTE,
         "seed": "workload seed + 7919 * rank",
     }
+
+
+def describe_path(runner: Runner, kernel: str, l2_detail: str) -> dict:
+    """How the library arm ran the workload (kept out of ``config``, which
+    names only the workload)."""
+    path = ("pa_decode_step" if runner.fused else "pa_write_kv + " + ("pa_decode_splitk" if runner.split else
+                                                                      "pa_decode"))
+    path += ((" (split-K, dynamic work queue)" if runner.partition == 0 else
+              f" (split-K, partition {runner.partition})") if runner.split else " (one CTA per sequence, kv head)")
+    return {"call": path, "kernel": kernel, "l2": l2_detail}
 
 
 def op_duration(runner: "Runner", total_ms: float, K: int, dec_ms: float):
@@ -610,28 +647,99 @@ def op_duration(runner: "Runner", total_ms: float, K: int, dec_ms: float):
     return dec_ms, f"CUDA events around the decode call of every {EVENT_EVERY}th step of the timed graph"
 
 
-def shape_summary(w: wl.Workload, rank: int, kernel: str, K: int, W: int, world: int, dev_idx: int, peak: float,
-                  partition: int = -1):
-    runner = Runner(w, rank, kernel, True, partition)
-    total_ms, dec_ms, _ = run_timed(runner, K, W, world, dev_idx)
-    ms = total_ms / K
-    op_ms, _ = op_duration(runner, total_ms, K, dec_ms)
-    res = {
-        "tokens_per_s": round(runner.B / (ms * 1e-3), 1),
-        "ms_per_step": round(ms, 5),
-        "decode_ms": round(op_ms, 5),
-        "decode_gbs": round(runner.kv_bytes / (op_ms * 1e-3) / 1e9, 1),
-        "decode_frac": round(runner.kv_bytes / (op_ms * 1e-3) / 1e9 / peak, 4),
-        "launches_per_step": runner.launches_per_step,
-        "kv_bytes": runner.kv_bytes,
-        "kv_bytes_unique": runner.kv_bytes_unique,
-        "partition": runner.partition,
+def roofline_block(runner: Runner, op_ms: float, op_timing: str, dec_ms: float, peak: float, peak_kind: str,
+                   traffic_key: str) -> dict:
+    """HBM roofline of the decode op: algorithmic bytes are the UNIQUE KV bytes
+    the step must read (a prefix block shared by several sequences counts
+    once); the logical bytes (every sequence's own view) over the same time are
+    reported beside them as the effective rate."""
+    uniq, logical = runner.kv_bytes_unique, runner.kv_bytes
+    achieved = uniq / (op_ms * 1e-3) / 1e9
+    return {
+        "bound": "hbm",
+        "kernel": ("fused append + " if runner.fused else "") + (
+            "split-K decode + LSE merge" if runner.split else "decode"),
+        "achieved": round(achieved, 1),
+        "peak": peak,
+        "peak_kind": peak_kind,
+        "unit": "GB/s",
+        "frac": round(achieved / peak, 4),
+        "traffic": recorded_traffic(runner.w.name, traffic_key),
+        "traffic_scope": "dram bytes read + written by all launches of one step (ncu), per step",
+        "algorithmic_bytes_per_launch": uniq,
+        "logical_bytes_per_launch": logical,
+        "effective_gbs_logical": round(logical / (op_ms * 1e-3) / 1e9, 1),
+        "launch_ms": round(op_ms, 5),
+        "launch_timing": op_timing,
+        "launch_ms_event_sampled": round(dec_ms, 5),
     }
-    if runner.kv_bytes_unique != runner.kv_bytes:
-        res["decode_gbs_unique"] = round(runner.kv_bytes_unique / (dec_ms * 1e-3) / 1e9, 1)
+
+
+def traffic_key(runner: Runner) -> str:
+    """Key of a step's record in profiles/traffic.json."""
+    key = ("step" if runner.fused else "decode") + ("_splitk" if runner.split else "")
+    return key + ("_dynamic" if runner.split and runner.partition == 0 and runner.w.partition_tokens else "")
+
+
+def decode_line(w: wl.Workload, rank: int, kernel: str, split: bool, partition: int, fused: bool, K: int, W: int,
+                world: int, dev_idx: int, peak: float, peak_kind: str, e2e: bool = True, cpu_seconds: float = 0.0):
+    """Time the decode step on one workload and return the keys of a bench line
+    for it: value (tokens/s over all ranks), ms_per_step, config, path,
+    roofline, e2e (host buffers, copies inside the timed region), the CPU
+    oracle baselines when ``cpu_seconds`` > 0, and the clocks."""
+    runner = Runner(w, rank, kernel, split, partition, fused=fused)
+    l2 = torch.cuda.get_device_properties(dev_idx).L2_cache_size
+    l2_detail = f"rotating {runner.R} KV pool copies ({runner.pool_bytes_total / 1e6:.0f} MB, L2 {l2 / 1e6:.0f} MB)"
+    total_ms, dec_ms, clocks = run_timed(runner, K, W, world, dev_idx)
+    total_ms = max_over_ranks(total_ms, world)
+    dec_ms = max_over_ranks(dec_ms, world)
+    tokens = sum_over_ranks(runner.B * K, world)
+    op_ms, op_timing = op_duration(runner, total_ms, K, dec_ms)
+    line = {
+        "value": round(tokens / (total_ms * 1e-3), 1),
+        "unit": "tokens/s",
+        "ms_per_step": round(total_ms / K, 5),
+        "config": workload_config(w, runner.batch),
+        "path": describe_path(runner, kernel, l2_detail),
+        "roofline": roofline_block(runner, op_ms, op_timing, dec_ms, peak, peak_kind, traffic_key(runner)),
+        "gpu_launches": K * runner.launches_per_step,
+        "launches_per_step": runner.launches_per_step,
+        "clocks": clocks,
+    }
+    if e2e:
+        e2e_ms, h2d, d2h = run_e2e(runner, K, world)
+        e2e_ms = max_over_ranks(e2e_ms, world)
+        line["e2e"] = {"value": round(tokens / (e2e_ms * 1e-3), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                       "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / K, 5)}
+    batch = runner.batch
     del runner
     torch.cuda.empty_cache()
-    return res
+    if cpu_seconds > 0 and world == 1 and rank == 0:
+        line.update(cpu_baselines(w, batch, cpu_seconds))
+    del batch
+    torch.cuda.empty_cache()
+    return line
+
+
+def shape_summary(w: wl.Workload, rank: int, kernel: str, K: int, W: int, world: int, dev_idx: int, peak: float,
+                  partition: int = -1):
+    """A decode shape timed like the headline, without the end-to-end leg and
+    CPU baselines: tokens/s and the HBM fraction on unique bytes."""
+    d = decode_line(w, rank, kernel, True, partition, True, K, W, world, dev_idx, peak, "measured", e2e=False)
+    r = d["roofline"]
+    return {
+        "tokens_per_s": d["value"],
+        "ms_per_step": d["ms_per_step"],
+        "decode_ms": r["launch_ms"],
+        "decode_gbs": r["achieved"],
+        "decode_frac": r["frac"],
+        "effective_gbs_logical": r["effective_gbs_logical"],
+        "launches_per_step": d["launches_per_step"],
+        "kv_bytes_unique": r["algorithmic_bytes_per_launch"],
+        "kv_bytes": r["logical_bytes_per_launch"],
+        "traffic": r["traffic"],
+        "path": d["path"]["call"],
+    }
 
 
 def multi_summary(w: wl.Workload, q_len: int, rank: int, K: int, W: int, world: int, dev_idx: int, peak: float):
@@ -712,64 +820,35 @@ def main_ours(args, world, rank, local):
     if args.op != "decode":
         return main_op(args, world, rank, local)
     split = not args.no_split
-    runner = Runner(w, rank, args.kernel, split, args.partition, fused=not args.unfused)
-    l2 = torch.cuda.get_device_properties(local).L2_cache_size
-    l2_note = (f"rotating {runner.R} KV pool copies ({runner.pool_bytes_total / 1e6:.0f} MB, "
-               f"L2 {l2 / 1e6:.0f} MB)")
     K, W = args.steps, args.warmup
-    total_ms, dec_ms, clocks = run_timed(runner, K, W, world, local)
-    total_ms = max_over_ranks(total_ms, world)
-    dec_ms = max_over_ranks(dec_ms, world)
-    tokens = sum_over_ranks(runner.B * K, world)
-    value = tokens / (total_ms * 1e-3)
-    e2e_ms, h2d, d2h = run_e2e(runner, K, world)
-    e2e_ms = max_over_ranks(e2e_ms, world)
     peak, peak_kind = measured_peaks()
-    op_ms, op_timing = op_duration(runner, total_ms, K, dec_ms)
-    achieved = runner.kv_bytes / (op_ms * 1e-3) / 1e9
-    kernel_key = ("step" if runner.fused else "decode") + ("_splitk" if split else "")
-    traffic = recorded_traffic(w.name, kernel_key)
-    launches_per_step = runner.launches_per_step
+    one = world == 1 and rank == 0
+    head = decode_line(w, rank, args.kernel, split, args.partition, not args.unfused, K, W, world, local, peak,
+                       peak_kind, e2e=True, cpu_seconds=0.0 if args.no_cpu else args.cpu_seconds)
     line = {
         "metric": METRIC,
-        "value": round(value, 1),
+        "value": head["value"],
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": K,
         "warmup": W,
-        "ms_per_step": round(total_ms / K, 5),
+        "ms_per_step": head["ms_per_step"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": w.dtype,
-        "data": "synthetic (seeded; q/k/v ~ N(0,1), shuffled physical blocks, NaN canaries in dead slots)",
-        "config": describe(w, runner, args, l2_note),
-        "roofline": {
-            "bound": "hbm",
-            "kernel": ("fused append + " if runner.fused else "") + (
-                "split-K decode + LSE combine" if split else "decode"),
-            "achieved": round(achieved, 1),
-            "peak": peak,
-            "peak_kind": peak_kind,
-            "unit": "GB/s",
-            "frac": round(achieved / peak, 4),
-            "traffic": traffic,
-            "algorithmic_bytes_per_launch": runner.kv_bytes,
-            "launch_ms": round(op_ms, 5),
-            "launch_timing": op_timing,
-            "launch_ms_event_sampled": round(dec_ms, 5),
-        },
-        "e2e": {
-            "value": round(tokens / (e2e_ms * 1e-3), 1),
-            "unit": "tokens/s",
-            "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h,
-            "ms_per_step": round(e2e_ms / K, 5),
-        },
-        "gpu_launches": K * launches_per_step,
-        "clocks": clocks,
+        "data": DATA,
+        "config": head["config"],
+        "path": head["path"],
+        "roofline": head["roofline"],
+        "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"],
+        "clocks": head["clocks"],
     }
-    if world == 1 and rank == 0 and runner.fused and split:
+    for k in ("cpu_baseline", "cpu_baseline_1core"):
+        if k in head:
+            line[k] = head[k]
+    if one and not args.unfused and split:
         # The attention alone (the append already done), timed the same way.
         dr = DecodeOnlyRunner(w, rank)
         d_total, d_dec, _ = run_timed(dr, K, W, 1, local)
@@ -777,21 +856,26 @@ def main_ours(args, world, rank, local):
         line["decode_alone"] = {
             "ms_per_step": round(d_ms, 5),
             "tokens_per_s": round(dr.B / (d_ms * 1e-3), 1),
-            "kv_gbs": round(dr.kv_bytes / (d_ms * 1e-3) / 1e9, 1),
-            "frac": round(dr.kv_bytes / (d_ms * 1e-3) / 1e9 / peak, 4),
+            "kv_gbs": round(dr.kv_bytes_unique / (d_ms * 1e-3) / 1e9, 1),
+            "frac": round(dr.kv_bytes_unique / (d_ms * 1e-3) / 1e9 / peak, 4),
             "launches_per_step": dr.launches_per_step,
         }
         del dr
-    if world == 1 and rank == 0 and args.shapes != "none":
+        torch.cuda.empty_cache()
+    if one and args.shapes != "none":
         names = [n for n in wl.WORKLOADS if n not in (w.name, "tiny_fp32")] if args.shapes == "auto" else [
             s for s in args.shapes.split(",") if s]
         extra = {}
-        del runner
-        torch.cuda.empty_cache()
         for n in names:
-            extra[n] = shape_summary(wl.WORKLOADS[n], rank, args.kernel, 50, 5, world, local, peak)
-            if wl.WORKLOADS[n].partition_tokens:  # also the dynamic schedule
-                extra[n + "@dynamic"] = shape_summary(wl.WORKLOADS[n], rank, args.kernel, 50, 5, world, local, peak, 0)
+            wn = wl.WORKLOADS[n]
+            if n in TARGET_SHAPES:
+                # A full line: roofline, end-to-end and CPU baselines of its own.
+                extra[n] = decode_line(wn, rank, args.kernel, True, -1, True, 50, 5, world, local, peak, peak_kind,
+                                       e2e=True, cpu_seconds=0.0 if args.no_cpu else args.cpu_seconds / 2)
+            else:
+                extra[n] = shape_summary(wn, rank, args.kernel, 50, 5, world, local, peak)
+            if wn.partition_tokens:  # also the dynamic schedule
+                extra[n + "@dynamic"] = shape_summary(wn, rank, args.kernel, 50, 5, world, local, peak, 0)
         for n, T in MULTI_SHAPES:
             if args.shapes == "auto" or n in names or n == w.name:
                 extra[f"{n}@multi{T}"] = multi_summary(wl.WORKLOADS[n], T, rank, 50, 5, world, local, peak)
@@ -802,12 +886,6 @@ def main_ours(args, world, rank, local):
             if args.shapes == "auto" or n in names or n == w.name:
                 extra[f"{n}@prefill{P_}x{T}"] = prefill_summary(wl.WORKLOADS[n], P_, T, rank, 20, 3, world, local)
         line["per_shape"] = extra
-        runner = None
-    if world == 1 and rank == 0 and not args.no_cpu:
-        b = wl.make_batch(w, seed=rank_seed(w, rank), device="cuda")
-        info = OracleSample(w, b).run(args.cpu_seconds)
-        info["value"] = round(info["value"], 2)
-        line["cpu_baseline"] = info
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -866,6 +944,7 @@ def main_reference(args, rank):
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     b = wl.make_batch(w, seed=rank_seed(w, 0), device=dev)
     sampler = OracleSample(w, b)
+    config = workload_config(w, b)
     del b
     K, W = args.steps, args.warmup
     budget = max(0.05, 120.0 / max(1, K + W))  # keep the whole run within a few minutes
@@ -891,9 +970,10 @@ def main_reference(args, rank):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "f64",
-        "data": "synthetic (seeded)",
+        "data": DATA,
         "impl": "reference",
-        "config": {"workload": w.name, "batch": sampler.B, "path": "fp64 CPU oracle (C, OpenMP)"},
+        "config": config,
+        "path": {"call": "fp64 CPU oracle (C, OpenMP): append + decode", "kernel": "none", "l2": "n/a"},
         "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": info["cores"], "kind": "oracle",
                          "sample": f"each step: {info['sample']}"},
         "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
