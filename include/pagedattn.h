@@ -250,7 +250,9 @@ size_t pa_decode_multi_workspace_size(int32_t batch, int32_t q_len, int32_t num_
  *   (causal, window, softcap).  A chunk of a chunked prefill is the same call
  *   with the earlier chunks already in the cache.
  *   bf16 only.  One launch for the append and one for the attention, whose
- *   CTAs each take 64 / G query tokens of one sequence and one kv head; no
+ *   CTAs each take 128 / G query tokens of one sequence and one kv head
+ *   (max_q_len / (128 / G) <= 65535, else PA_ERR_UNSUPPORTED), each
+ *   sequence's last tokens (the most keys under the causal mask) first; no
  *   workspace.
  *   Passages: nano-vllm (ovshake) README, "Key Concepts Explained: KV Cache"
  *   (prefill processes the prompt and stores its keys and values) and

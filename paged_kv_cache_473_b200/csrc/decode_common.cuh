@@ -53,6 +53,7 @@ struct DecodeParams {
   int block_size, log2_bs, max_blocks, num_blocks;
   int window;
   int partition;    // tokens per partition (a multiple of 64); 1 << 30 without split
+  int log2_partition;  // dynamic schedule: log2(partition) (its partitions are powers of two)
   int max_parts;    // partitions per sequence in the workspace
   int max_context;  // bound on context_lens[b]
   float scale;      // multiplies q.k

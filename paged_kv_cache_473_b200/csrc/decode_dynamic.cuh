@@ -18,17 +18,31 @@
 // into the next item before the current one is finished, so its ring stays
 // full across item boundaries.
 //
-// Merge: each (sequence, kv head) unit has an arrival counter in the
-// workspace.  A warp that stored a partial publishes it (memory fence) and
-// counts it; the warp that brings the count to the unit's number of
-// partitions reads every partial back from L2, writes the normalised output
-// rows (log-sum-exp merge, merge_unit) and returns the counter to zero.  The
-// last CTA to finish returns the work counter to zero, so the workspace is
-// ready for the next call without a second kernel.
+// Merge (small steps): each (sequence, kv head) unit has an arrival counter in
+// the workspace.  A warp that stored a partial publishes it (release fence)
+// and counts it; the warp that brings the count to the unit's number of
+// partitions reads every partial back through L2 in partition order (the same
+// bits whichever warp merges), merges them (log-sum-exp) and writes the
+// normalised output rows; it returns the counter to zero.  (Measured on
+// B200 and not kept: counting arrivals before the stores, so that the last
+// warp merges without storing its own partial; the waits it adds cost more
+// than the store and fence it saves.)  The last CTA to
+// finish returns the work counter to zero, so the workspace is ready for the
+// next call without a second kernel.  Larger steps leave the merge to the
+// combine kernel.
 //
-// Items are numbered sequence-major; each CTA first builds, with block-wide
-// scans over context_lens, the number of items before each sequence and
-// decodes an item number with a binary search in shared memory.
+// Items are numbered sequence-major.  The number of items before each sequence
+// is a scan over context_lens, and an item number is decoded with a binary
+// search over that prefix in shared memory.  For batches of up to
+// kWarpScanBatch sequences every warp scans the lengths itself, into its own
+// slice of shared memory, so that no barrier across the CTA's warps stands
+// between a warp's start and its first TMA issue; larger batches share one
+// CTA-wide scan.
+//
+// The kernel is launched as a programmatic dependent of whatever precedes it
+// on the stream: everything before griddepcontrol.wait (barrier set-up, the
+// tensor-map prefetch) overlaps that kernel's tail, and no global memory is
+// touched before the wait (the cascade's own-range pass waits at its end).
 //
 // APPEND (the fused decode step): the item that ends at the sequence's last
 // token writes the step's new key/value row to the cache slot of position L-1
@@ -42,6 +56,9 @@
 namespace pa {
 
 constexpr int kMaxDynamicBatch = 2048;  // prefix arrays live in shared memory
+// Batches up to this size are scanned by every warp for itself (per-warp prefix
+// arrays, two sequences per lane); larger ones by the CTA together.
+constexpr int kWarpScanBatch = 64;
 // The split-K workspace starts with a fixed counter region: [0] work-item
 // counter, [1] finished CTAs, then one arrival count per (sequence, kv head).
 constexpr int kMaxDynamicUnits = 65534;
@@ -70,6 +87,10 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int& to
 
 // Partitions of sequence b's attended range [s0, L) (0 when it is empty).
 __device__ __forceinline__ int seq_parts(int L, int s0, int P) { return L > s0 ? (L + P - 1) / P - s0 / P : 0; }
+// The same for a partition of 2^lp tokens.
+__device__ __forceinline__ int seq_parts_sh(int L, int s0, int lp) {
+  return L > s0 ? ((L + (1 << lp) - 1) >> lp) - (s0 >> lp) : 0;
+}
 
 // First position this kernel attends for sequence b: the window start, or
 // (CASCADE) the end of the shared prefix for a sharer.
@@ -91,77 +112,114 @@ struct Item {
 // larger splits with the combine kernel).
 constexpr int kMaxMergeParts = 8;
 
-// Log-sum-exp merge of the `n` <= kMaxMergeParts partials [pb, pb + n) of unit
-// (b, g) into the normalised output rows of its G query heads:
-//   M = max_p m_p,  out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p
-// (m in the log2 domain, o unnormalised relative to m).  lph lanes per head (a
-// power of two), each covering D / lph dims in chunks of 16; the partials are
-// read through L2 (other SMs wrote them).  The merge runs after the unit's
-// last partition, on the critical path of the call's tail, so every load of a
-// chunk is issued before any is used: one L2 round trip instead of one per
-// few partials (kBatch partials at a time where registers are tight).
+// In-kernel merge.  A unit's partials are stored in LANE ORDER: the D floats of
+// head h's slot for partition i hold, at [r * D/8 + 2 * mt + e], dimension
+// mt * 16 + r + 8 e, where r = lane / 4 is the row group of the lane that holds
+// that value in the MMA accumulator layout (WarpAttn: lane holds heads 2 (lane
+// % 4) and + 1, dimensions mt * 16 + lane / 4 (+ 8)).  So each lane writes, and
+// the merging warp's same lane reads, its own D/8 values per head as whole
+// 16-byte vectors, and the merge needs no exchange between lanes.  (m, l) sit
+// in the [row][part][2] array as for the combine.
+
+// This warp's partial state of its G heads into partition `part`'s slots.
 template <int D>
-__device__ __forceinline__ void merge_unit(const DecodeParams& p, int b, int g, int pb, int n, int lane) {
-  constexpr int kBatch = D == 128 ? 4 : kMaxMergeParts;  // head_dim 128 runs with a 170-register cap
-  const int G = p.group;
-  const int lph = min(G == 1 ? 32 : G == 2 ? 16 : G <= 4 ? 8 : 4, D / 16);
-  const int h = lane / lph, s = lane & (lph - 1);
-  const bool active = h < G;
-  const size_t row = (size_t)b * p.hq + (size_t)g * G + (active ? h : 0);
-  const float2* ml = reinterpret_cast<const float2*>(p.ws_ml) + row * p.max_parts + pb;
-  float2 mlv[kMaxMergeParts];
+__device__ __forceinline__ void store_partial_lanes(const WarpAttn<D>& st, const DecodeParams& p, size_t row0,
+                                                    int part, int G, int lane) {
+  const int n0 = 2 * (lane & 3), r = lane >> 2;
+  const size_t slot0 = (row0 + n0) * p.max_parts + part;  // head n0; head n0 + 1 is max_parts slots further
+  float4* po0 = reinterpret_cast<float4*>(p.ws_o + slot0 * D + r * (D / 8));
+  float4* po1 = reinterpret_cast<float4*>(p.ws_o + (slot0 + p.max_parts) * D + r * (D / 8));
 #pragma unroll
-  for (int i = 0; i < kMaxMergeParts; ++i) mlv[i] = i < n ? __ldcg(ml + i) : make_float2(-CUDART_INF_F, 0.f);
-  const int E = D / lph;
-  const float* po = p.ws_o + (row * p.max_parts + pb) * D + s * E;
-  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row * D + s * E;
-  for (int c0 = 0; c0 < E; c0 += 16) {
-    float acc[16];
+  for (int k = 0; k < D / 32; ++k) {  // vector k: mt = 2k and 2k + 1
+    if (n0 < G) po0[k] = make_float4(st.o[2 * k][0], st.o[2 * k][2], st.o[2 * k + 1][0], st.o[2 * k + 1][2]);
+    if (n0 + 1 < G) po1[k] = make_float4(st.o[2 * k][1], st.o[2 * k][3], st.o[2 * k + 1][1], st.o[2 * k + 1][3]);
+  }
+  if (lane < 4) {
+    float2* pml = reinterpret_cast<float2*>(p.ws_ml) + slot0;
+    if (n0 < G) pml[0] = make_float2(st.m0, st.l0);
+    if (n0 + 1 < G) pml[p.max_parts] = make_float2(st.m1, st.l1);
+  }
+}
+
+// Log-sum-exp merge of a unit's n <= kMaxMergeParts partitions into `st`:
+//   M = max_i m_i,  o = sum_i 2^(m_i - M) o_i,  l = sum_i 2^(m_i - M) l_i
+// (m in the log2 domain, o unnormalised relative to m), the sums taken in
+// partition order, so the result is the same bits whichever warp merges.  The
+// merging warp's own partition `own` has been stored like the others; its
+// (m, l) come from registers.
+// The loads of kB partials are issued before any is used (one L2 round trip
+// per batch).
+template <int D>
+__device__ __forceinline__ void merge_lanes(WarpAttn<D>& st, const DecodeParams& p, size_t row0, int pb, int n,
+                                            int own, int G, int lane) {
+  constexpr int V = D / 32;                // 16-byte vectors per head per lane
+  // Partials per batch.  At head_dim 64 all of them, so that every load of the
+  // merge, (m, l) included, is in one L2 round trip (the kernel's two CTAs per
+  // SM are set by shared memory, so the registers cost no occupancy); head_dim
+  // 128 runs at a 170-register cap.
+  constexpr int kB = D == 64 ? kMaxMergeParts : 1;
+  const int n0 = 2 * (lane & 3), r = lane >> 2;
+  const bool h0 = n0 < G, h1 = n0 + 1 < G;
+  const size_t slot0 = (row0 + n0) * p.max_parts + pb;
+  const float2* ml = reinterpret_cast<const float2*>(p.ws_ml) + slot0;
+  float2 a[kMaxMergeParts], c[kMaxMergeParts];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) acc[k] = 0.f;
-    float den = 0.f;
+  for (int i = 0; i < kMaxMergeParts; ++i) {
+    const bool other = i < n && i != own;
+    a[i] = i == own ? make_float2(st.m0, st.l0)
+                    : (other && h0 ? __ldcg(ml + i) : make_float2(-CUDART_INF_F, 0.f));
+    c[i] = i == own ? make_float2(st.m1, st.l1)
+                    : (other && h1 ? __ldcg(ml + p.max_parts + i) : make_float2(-CUDART_INF_F, 0.f));
+  }
+  float M0 = -CUDART_INF_F, M1 = -CUDART_INF_F;
 #pragma unroll
-    for (int i0 = 0; i0 < kMaxMergeParts; i0 += kBatch) {
-      if (i0 >= n) break;
-      float4 x[kBatch][4];
+  for (int i = 0; i < kMaxMergeParts; ++i) {
+    M0 = fmaxf(M0, a[i].x);
+    M1 = fmaxf(M1, c[i].x);
+  }
+  st.l0 = st.l1 = 0.f;
 #pragma unroll
-      for (int i = 0; i < kBatch; ++i) {
-        const float4* src = reinterpret_cast<const float4*>(po + (size_t)(i0 + i) * D + c0);
+  for (int mt = 0; mt < D / 16; ++mt) st.o[mt][0] = st.o[mt][1] = st.o[mt][2] = st.o[mt][3] = 0.f;
+  const float* base0 = p.ws_o + slot0 * D + r * (D / 8);
+  const float* base1 = p.ws_o + (slot0 + p.max_parts) * D + r * (D / 8);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) x[i][k] = i0 + i < n ? __ldcg(src + k) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-      float M = -CUDART_INF_F;
+  for (int i0 = 0; i0 < kMaxMergeParts; i0 += kB) {
+    if (i0 >= n) break;
+    float4 x0[kB][V], x1[kB][V];
 #pragma unroll
-      for (int i = 0; i < kMaxMergeParts; ++i) M = fmaxf(M, mlv[i].x);
+    for (int j = 0; j < kB; ++j) {
+      const int i = i0 + j;
+      const float4* s0 = reinterpret_cast<const float4*>(base0 + (size_t)i * D);
+      const float4* s1 = reinterpret_cast<const float4*>(base1 + (size_t)i * D);
 #pragma unroll
-      for (int i = 0; i < kBatch; ++i) {
-        const float2 v = mlv[i0 + i];
-        const float w = v.x == -CUDART_INF_F ? 0.f : exp2f(v.x - M);  // empty or absent partial: weight 0
-        den = fmaf(w, v.y, den);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          acc[4 * k + 0] = fmaf(w, x[i][k].x, acc[4 * k + 0]);
-          acc[4 * k + 1] = fmaf(w, x[i][k].y, acc[4 * k + 1]);
-          acc[4 * k + 2] = fmaf(w, x[i][k].z, acc[4 * k + 2]);
-          acc[4 * k + 3] = fmaf(w, x[i][k].w, acc[4 * k + 3]);
-        }
+      for (int k = 0; k < V; ++k) {
+        x0[j][k] = i < n && h0 ? __ldcg(s0 + k) : make_float4(0.f, 0.f, 0.f, 0.f);
+        x1[j][k] = i < n && h1 ? __ldcg(s1 + k) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
-    if (active) {
-      const float inv = 1.f / den;
-      uint4 lo, hi;
-      lo.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-      lo.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
-      lo.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
-      lo.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
-      hi.x = pack_bf16x2(acc[8] * inv, acc[9] * inv);
-      hi.y = pack_bf16x2(acc[10] * inv, acc[11] * inv);
-      hi.z = pack_bf16x2(acc[12] * inv, acc[13] * inv);
-      hi.w = pack_bf16x2(acc[14] * inv, acc[15] * inv);
-      reinterpret_cast<uint4*>(out + c0)[0] = lo;
-      reinterpret_cast<uint4*>(out + c0)[1] = hi;
+#pragma unroll
+    for (int j = 0; j < kB; ++j) {
+      const int i = i0 + j;
+      if (i >= kMaxMergeParts) break;
+      const float wa = a[i].x == -CUDART_INF_F ? 0.f : exp2f(a[i].x - M0);  // absent partition: weight 0
+      const float wc = c[i].x == -CUDART_INF_F ? 0.f : exp2f(c[i].x - M1);
+      st.l0 = fmaf(wa, a[i].y, st.l0);
+      st.l1 = fmaf(wc, c[i].y, st.l1);
+#pragma unroll
+      for (int k = 0; k < V; ++k) {
+        st.o[2 * k][0] = fmaf(wa, x0[j][k].x, st.o[2 * k][0]);
+        st.o[2 * k][2] = fmaf(wa, x0[j][k].y, st.o[2 * k][2]);
+        st.o[2 * k + 1][0] = fmaf(wa, x0[j][k].z, st.o[2 * k + 1][0]);
+        st.o[2 * k + 1][2] = fmaf(wa, x0[j][k].w, st.o[2 * k + 1][2]);
+        st.o[2 * k][1] = fmaf(wc, x1[j][k].x, st.o[2 * k][1]);
+        st.o[2 * k][3] = fmaf(wc, x1[j][k].y, st.o[2 * k][3]);
+        st.o[2 * k + 1][1] = fmaf(wc, x1[j][k].z, st.o[2 * k + 1][1]);
+        st.o[2 * k + 1][3] = fmaf(wc, x1[j][k].w, st.o[2 * k + 1][3]);
+      }
     }
   }
+  st.m0 = M0;
+  st.m1 = M1;
 }
 
 template <int D, int NW, int ST>
@@ -175,6 +233,11 @@ struct DynCfg {
   static constexpr int kScratchOffset = kBarOffset + NW * ST * 8;
   static constexpr int kPrefixOffset = kScratchOffset + 32 * 4;
   static __host__ __device__ constexpr int smem_bytes(int B) { return kPrefixOffset + (2 * B + 1) * 4 + 1024; }
+  // decode_dynamic_kernel: one prefix / length array per warp up to
+  // kWarpScanBatch sequences, one per CTA above.
+  static __host__ __device__ constexpr int decode_smem_bytes(int B) {
+    return kPrefixOffset + (B <= kWarpScanBatch ? NW : 1) * (2 * B + 1) * 4 + 1024;
+  }
 };
 
 // Resident CTAs per SM the configurations are sized for (shared memory allows
@@ -191,59 +254,117 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int G = p.group, Hkv = p.hkv, P = p.partition, B = p.batch;
-  int* scratch = reinterpret_cast<int*>(smem + Cfg::kScratchOffset);
-  int* pre = reinterpret_cast<int*>(smem + Cfg::kPrefixOffset);  // [B+1] items before sequence b
-  int* lens = pre + B + 1;                                        // [B] clamped context lengths
-
-  // Without the in-kernel merge the combine kernel (a programmatic dependent)
-  // may launch now; it waits for this grid to finish before it reads anything.
-  if (!p.merge_in_kernel) pdl_launch_dependents();
-
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+  const bool warp_scan = B <= kWarpScanBatch;
+  int* scratch = reinterpret_cast<int*>(smem + Cfg::kScratchOffset);
+  // [B+1] items before sequence b, then [B] clamped context lengths: this
+  // warp's own arrays (warp_scan), else the CTA's.
+  int* pre = reinterpret_cast<int*>(smem + Cfg::kPrefixOffset) + (warp_scan ? warp * (2 * B + 1) : 0);
+  int* lens = pre + B + 1;
+
+  // The next kernel on the stream (the combine, or the next step when it is a
+  // programmatic dependent too) may launch now; it waits for this grid to
+  // finish before it touches global memory.
+  pdl_launch_dependents();
+
   const uint32_t ring = smem_addr(smem) + warp * ST * Cfg::kStageBytes;
   const uint32_t bars = smem_addr(smem + Cfg::kBarOffset) + warp * ST * 8;
   // A warp's first two items are fixed by its index (W warps in the grid: items
   // w and W + w); later ones are claimed from the counter, offset by 2W, so the
   // launch does not start with every warp contending for one address.
-  const int W = gridDim.x * NW, wg = blockIdx.x * NW + warp;
   if (lane == 0) {
 #pragma unroll
     for (int s = 0; s < ST; ++s) mbar_init(bars + 8 * s, 1);
     mbar_init_fence();
-    if (warp == 0) {
-      prefetch_tensormap(&kmap);
-      prefetch_tensormap(&vmap);
+    prefetch_tensormap(&kmap);
+    prefetch_tensormap(&vmap);
+  }
+  if (tid == 0) {
+    // The small inputs the prologue reads one after another (lengths, then
+    // block tables and queries), brought into L2 while the preceding kernel
+    // finishes: each CTA a share.  Prefetches only warm L2; they read no value
+    // this grid uses before the wait below.
+    auto share = [&](const void* base, size_t bytes) {
+      const size_t chunk = max((size_t)256, (bytes + gridDim.x - 1) / gridDim.x);
+      const size_t off = (size_t)blockIdx.x * chunk;
+      if (off < bytes) prefetch_l2(static_cast<const char*>(base) + off, min(chunk, bytes - off));
+    };
+    share(p.context_lens, (size_t)B * 4);
+    share(p.block_tables, (size_t)B * p.max_blocks * 4);
+    share(p.q, (size_t)B * p.hq * D * 2);
+    if (APPEND) {
+      share(p.k_new, (size_t)B * Hkv * D * 2);
+      share(p.v_new, (size_t)B * Hkv * D * 2);
     }
   }
+  // Nothing above touched global memory; the preceding kernel's writes (and
+  // its reads of what this grid writes) are complete after this.  (The
+  // cascade's own-range pass reads nothing its preceding prefix pass writes
+  // and waits for it at its end instead, so the two passes overlap.)
+  if (!CASCADE) pdl_wait();
 
   // ---- items before each sequence ---------------------------------------------
-  // All lengths are loaded at once (independent loads), then scanned.
-#pragma unroll 4
-  for (int b = tid; b < B; b += blockDim.x) lens[b] = clamp_context(p, b, blockIdx.x == 0);
-  __syncthreads();
-  int base = 0;
-  for (int b0 = 0; b0 < B; b0 += blockDim.x) {
-    const int b = b0 + tid;
-    int items = 0;
-    if (b < B) {
-      const int L = lens[b];
-      items = Hkv * seq_parts(L, seq_start<CASCADE>(p, b, L), P);
+  const int W = gridDim.x * NW, wg = blockIdx.x * NW + warp;
+  if (warp_scan) {
+    // This warp alone: a warp scan over the items of the lengths it loaded
+    // (sequences 2l and 2l + 1 to lane l).
+    const int b0 = 2 * lane, lp = p.log2_partition;
+    int L0 = 0, L1 = 0, n0 = 0, n1 = 0;
+    if (b0 < B) {
+      L0 = clamp_context(p, b0, wg == 0);
+      n0 = Hkv * seq_parts_sh(L0, seq_start<CASCADE>(p, b0, L0), lp);
     }
-    int total;
-    const int ex = block_exclusive_scan(items, scratch, total);
-    if (b < B) pre[b] = base + ex;
-    base += total;
+    if (b0 + 1 < B) {
+      L1 = clamp_context(p, b0 + 1, wg == 0);
+      n1 = Hkv * seq_parts_sh(L1, seq_start<CASCADE>(p, b0 + 1, L1), lp);
+    }
+    int incl = n0 + n1;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(FULL, incl, off);
+      if (lane >= off) incl += y;
+    }
+    const int base = incl - n0 - n1;
+    if (b0 < B) {
+      lens[b0] = L0;
+      pre[b0] = base;
+    }
+    if (b0 + 1 < B) {
+      lens[b0 + 1] = L1;
+      pre[b0 + 1] = base + n0;
+    }
+    if (lane == 31) pre[B] = incl;
+    __syncwarp();
+  } else {
+    // The CTA together: all lengths loaded at once (independent loads), then scanned.
+#pragma unroll 4
+    for (int b = tid; b < B; b += blockDim.x) lens[b] = clamp_context(p, b, blockIdx.x == 0);
+    __syncthreads();
+    int base = 0;
+    for (int b0 = 0; b0 < B; b0 += blockDim.x) {
+      const int b = b0 + tid;
+      int items = 0;
+      if (b < B) {
+        const int L = lens[b];
+        items = Hkv * seq_parts(L, seq_start<CASCADE>(p, b, L), P);
+      }
+      int total;
+      const int ex = block_exclusive_scan(items, scratch, total);
+      if (b < B) pre[b] = base + ex;
+      base += total;
+    }
+    if (tid == 0) pre[B] = base;
+    __syncthreads();
   }
-  if (tid == 0) pre[B] = base;
-  __syncthreads();
   const int T = pre[B];
   // Sequences with nothing to attend (L == 0) get zero rows; no item covers
   // them.  (A cascade sharer whose range lies inside the shared prefix has no
-  // item either: the prefix pass writes its rows.)
-  for (int b = blockIdx.x; b < B; b += gridDim.x) {
+  // item either: the prefix pass writes its rows.)  Warp wg takes sequences
+  // wg, wg + W, ...
+  for (int b = wg; b < B; b += W) {
     if (pre[b + 1] != pre[b] || (CASCADE && lens[b] != 0)) continue;
     __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + (size_t)b * p.hq * D;
-    for (int i = tid; i < p.hq * D; i += blockDim.x) o[i] = __float2bfloat16_rn(0.f);
+    for (int i = lane; i < p.hq * D; i += 32) o[i] = __float2bfloat16_rn(0.f);
   }
 
   // Item number -> item.
@@ -394,22 +515,8 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
       // ---- store this item's result from registers ------------------------------------
       st.reduce_sums();
       const size_t row0 = (size_t)ci.b * p.hq + (size_t)ci.g * G;
-      if (ci.whole) {
-        const float inv0 = 1.f / st.l0, inv1 = 1.f / st.l1;
-        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row0 * D;
-#pragma unroll
-        for (int mt = 0; mt < D / 16; ++mt) {
-          const int d = mt * 16 + (lane >> 2);
-          if (n0 < G) {
-            out[(size_t)n0 * D + d] = __float2bfloat16_rn(st.o[mt][0] * inv0);
-            out[(size_t)n0 * D + d + 8] = __float2bfloat16_rn(st.o[mt][2] * inv0);
-          }
-          if (n0 + 1 < G) {
-            out[(size_t)(n0 + 1) * D + d] = __float2bfloat16_rn(st.o[mt][1] * inv1);
-            out[(size_t)(n0 + 1) * D + d + 8] = __float2bfloat16_rn(st.o[mt][3] * inv1);
-          }
-        }
-      } else {
+      bool write_rows = ci.whole;
+      if (!ci.whole && !p.merge_in_kernel) {  // the combine kernel merges: [row][part][D] partials
         const size_t slot0 = (row0 + n0) * p.max_parts + ci.part;  // head n0; head n0+1 is max_parts further
         float* po = p.ws_o + slot0 * D;
         const size_t hstride = (size_t)p.max_parts * D;
@@ -436,18 +543,35 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
             pml[(size_t)p.max_parts * 2 + 1] = st.l1;
           }
         }
-        if (p.merge_in_kernel) {
-          // Publish the partial, then count it (release); the unit's last
-          // partial merges them all (acquire).
+      } else if (!ci.whole) {  // merged in this kernel
+        // Publish the partial, then count it (release); the unit's last
+        // partial merges them all (acquire).
+        store_partial_lanes<D>(st, p, row0, ci.part, G, lane);
+        fence_acq_rel_gpu();
+        __syncwarp();
+        int* cnt = p.unit_count + (size_t)ci.b * Hkv + ci.g;
+        int last = 0;
+        if (lane == 0) last = atomicAdd(cnt, 1) == ci.parts - 1;
+        if (__shfl_sync(FULL, last, 0)) {
           fence_acq_rel_gpu();
-          __syncwarp();
-          int* cnt = p.unit_count + (size_t)ci.b * Hkv + ci.g;
-          int last = 0;
-          if (lane == 0) last = atomicAdd(cnt, 1) == ci.parts - 1;
-          if (__shfl_sync(FULL, last, 0)) {
-            fence_acq_rel_gpu();
-            merge_unit<D>(p, ci.b, ci.g, ci.pb, ci.parts, lane);
-            if (lane == 0) *cnt = 0;  // every partial of the unit has arrived: ready for the next call
+          merge_lanes<D>(st, p, row0, ci.pb, ci.parts, ci.part - ci.pb, G, lane);
+          write_rows = true;
+          if (lane == 0) *cnt = 0;  // every partial of the unit has arrived: ready for the next call
+        }
+      }
+      if (write_rows) {  // the normalised rows of the G heads, from registers
+        const float inv0 = 1.f / st.l0, inv1 = 1.f / st.l1;
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row0 * D;
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+          const int d = mt * 16 + (lane >> 2);
+          if (n0 < G) {
+            out[(size_t)n0 * D + d] = __float2bfloat16_rn(st.o[mt][0] * inv0);
+            out[(size_t)n0 * D + d + 8] = __float2bfloat16_rn(st.o[mt][2] * inv0);
+          }
+          if (n0 + 1 < G) {
+            out[(size_t)(n0 + 1) * D + d] = __float2bfloat16_rn(st.o[mt][1] * inv1);
+            out[(size_t)(n0 + 1) * D + d + 8] = __float2bfloat16_rn(st.o[mt][3] * inv1);
           }
         }
       }

@@ -90,7 +90,7 @@ bool cache_maps(const void* kbase, const void* vbase, int head_dim, long long ro
     int d;
     CUtensorMap kmap, vmap;
   };
-  constexpr int kEntries = 8;
+  constexpr int kEntries = 16;
   thread_local Entry table[kEntries] = {};
   thread_local int next = 0;
   for (const Entry& e : table) {
@@ -233,37 +233,6 @@ cudaError_t launch_mma(const DecodeParams& p, dim3 grid, cudaStream_t st) {
       return launch_mma_t<128, 4, 3, SPLIT, APPEND>(p, grid, st);
     default:
       return launch_mma_t<256, 2, 3, SPLIT, APPEND>(p, grid, st);
-  }
-}
-
-// Paged prefill attention on tcgen05: one CTA per 128 query rows (128 / G
-// tokens) of one sequence and kv head.
-template <int D>
-cudaError_t launch_prefill_t(const DecodeParams& p, dim3 grid, cudaStream_t st) {
-  using Cfg = pa::PrefillCfg<D>;
-  CUtensorMap kmap, vmap;
-  const long long rows = (long long)p.num_blocks * p.hkv * p.block_size;
-  if (!cache_maps(p.k_cache, p.v_cache, D, rows, &kmap, &vmap)) return cudaErrorInvalidValue;
-  auto kern = pa::prefill_umma_kernel<D>;
-  static std::atomic<uint64_t> smem_done{0};
-  cudaError_t e = set_smem(kern, Cfg::kSmemBytes, smem_done);
-  if (e != cudaSuccess) return e;
-  // The whole shared-memory carveout, so that kMinBlocks CTAs fit per SM.
-  static std::once_flag carveout_once;
-  std::call_once(carveout_once, [&] {
-    (void)cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-  });
-  return launch_ex(kern, grid, dim3(Cfg::kThreads), Cfg::kSmemBytes, st, false, kmap, vmap, p);
-}
-
-cudaError_t launch_prefill(const DecodeParams& p, dim3 grid, cudaStream_t st) {
-  switch (p.head_dim) {
-    case 64:
-      return launch_prefill_t<64>(p, grid, st);
-    case 128:
-      return launch_prefill_t<128>(p, grid, st);
-    default:
-      return launch_prefill_t<256>(p, grid, st);
   }
 }
 
@@ -411,6 +380,38 @@ cudaError_t occupancy(Kernel kern, int threads, int smem, std::atomic<long long>
   return e;
 }
 
+// Paged prefill attention on tcgen05: one CTA per 128 query rows (128 / G
+// tokens) of one sequence and kv head; grid (kv heads, sequences, query tiles
+// counted back from each sequence's end), so the longest tiles go first.
+template <int D>
+cudaError_t launch_prefill_t(const DecodeParams& p, dim3 grid, cudaStream_t st) {
+  using Cfg = pa::PrefillCfg<D>;
+  CUtensorMap kmap, vmap;
+  const long long rows = (long long)p.num_blocks * p.hkv * p.block_size;
+  if (!cache_maps(p.k_cache, p.v_cache, D, rows, &kmap, &vmap)) return cudaErrorInvalidValue;
+  auto kern = pa::prefill_umma_kernel<D>;
+  static std::atomic<uint64_t> smem_done{0};
+  cudaError_t e = set_smem(kern, Cfg::kSmemBytes, smem_done);
+  if (e != cudaSuccess) return e;
+  // The whole shared-memory carveout, so that kMinBlocks CTAs fit per SM.
+  static std::once_flag carveout_once;
+  std::call_once(carveout_once, [&] {
+    (void)cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  });
+  return launch_ex(kern, grid, dim3(Cfg::kThreads), Cfg::kSmemBytes, st, false, kmap, vmap, p);
+}
+
+cudaError_t launch_prefill(const DecodeParams& p, dim3 grid, cudaStream_t st) {
+  switch (p.head_dim) {
+    case 64:
+      return launch_prefill_t<64>(p, grid, st);
+    case 128:
+      return launch_prefill_t<128>(p, grid, st);
+    default:
+      return launch_prefill_t<256>(p, grid, st);
+  }
+}
+
 // Launch the dynamic schedule with the persistent grid (as many CTAs as are
 // resident at once).  Sets p.merge_in_kernel: the partitions of each unit are
 // merged in-kernel when the step is small next to the resident warps (at most
@@ -426,7 +427,7 @@ cudaError_t launch_dynamic_t(DecodeParams& p, cudaStream_t st, bool pdl, bool al
   const long long rows = (long long)p.num_blocks * p.hkv * p.block_size;
   if (!cache_maps(p.k_cache, p.v_cache, D, rows, &kmap, &vmap)) return cudaErrorInvalidValue;
   auto kern = pa::decode_dynamic_kernel<D, NW, ST, APPEND, CASCADE>;
-  const int smem = Cfg::smem_bytes(p.batch);
+  const int smem = Cfg::decode_smem_bytes(p.batch);
   static std::atomic<int> smem_done[64];
   cudaError_t e = set_smem_at_least(kern, smem, smem_done);
   if (e != cudaSuccess) return e;
@@ -438,16 +439,19 @@ cudaError_t launch_dynamic_t(DecodeParams& p, cudaStream_t st, bool pdl, bool al
   const int grid = occ * sm_count();
   const long long unit_bound = (long long)p.batch * p.hkv * p.max_parts;
   p.merge_in_kernel = (allow_merge && p.max_parts <= pa::kMaxMergeParts && unit_bound <= 2LL * grid * NW) ? 1 : 0;
+  if (!pow2(p.partition)) return cudaErrorInvalidValue;  // the schedule's partitions are powers of two
+  p.log2_partition = ilog2(p.partition);
   p.static_items = 2;
   return launch_ex(kern, dim3(grid), dim3(Cfg::kThreads), smem, st, pdl, kmap, vmap, p);
 }
 
-// CASCADE: the cascade's own-range pass (sharers start at the prefix end),
-// launched as a programmatic dependent of the prefix pass, merged by the
-// combine.
+// Launched as a programmatic dependent of the preceding kernel on the stream
+// (the kernel waits for it before touching global memory).  CASCADE: the
+// cascade's own-range pass (sharers start at the prefix end), which overlaps
+// the prefix pass and is merged by the combine.
 template <bool APPEND, bool CASCADE = false>
 cudaError_t launch_dynamic(DecodeParams& p, cudaStream_t st) {
-  const bool pdl = CASCADE, allow_merge = !CASCADE;
+  const bool pdl = true, allow_merge = !CASCADE;
   switch (p.head_dim) {
     // Warps are independent (one work item each); CTAs of a few warps with a
     // 2-6 stage ring each put ~192 KB of loads in flight per SM.
@@ -971,13 +975,13 @@ pa_status_t pa_prefill(const void* q, const void* k_new, const void* v_new, cons
   const int G = num_q_heads / num_kv_heads;
   const int q_tile = 128 / G;  // one CTA: 128 query rows = q_tile tokens x G heads
   const long long tiles = ((long long)max_q_len + q_tile - 1) / q_tile;
-  if (tiles > INT_MAX) return PA_ERR_UNSUPPORTED;
+  if (tiles > kMaxGridYZ) return PA_ERR_UNSUPPORTED;
   DecodeParams p = make_params(q, k_cache, v_cache, block_tables, context_lens, s, scale, softcap, window, out);
   p.cu_q = cu_q_lens;
   p.q_tile = q_tile;
   p.max_q_len = max_q_len;
   p.total_q = total_q;
-  cudaError_t e = launch_prefill(p, dim3((unsigned)tiles, num_kv_heads, batch), stream);
+  cudaError_t e = launch_prefill(p, dim3(num_kv_heads, batch, (unsigned)tiles), stream);
   if (e != cudaSuccess) return PA_ERR_CUDA;
   t_last_launches = append ? 2 : 1;
   return PA_OK;

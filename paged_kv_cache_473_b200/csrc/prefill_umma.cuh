@@ -74,7 +74,11 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kBoundThreads, PrefillCfg<D>::k
   constexpr uint32_t FULL = 0xffffffffu;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
-  const int g = blockIdx.y, b = blockIdx.z, G = p.group;
+  // Grid (kv heads, sequences, query tiles): blockIdx.z counts a sequence's
+  // query tiles back from its last one, so every sequence's longest tiles (the
+  // most keys under the causal mask) are dispatched first and the short ones
+  // fill the end of the launch.
+  const int g = blockIdx.x, b = blockIdx.y, back = blockIdx.z, G = p.group;
   const int TQ = C::kRows / G;
   if (smem_addr(smem) & 1023) {  // the swizzled tiles need 1024-byte alignment
     if (tid == 0) raise_error(PA_DEVERR_LAYOUT);
@@ -84,14 +88,16 @@ __global__ void __launch_bounds__(PrefillCfg<D>::kBoundThreads, PrefillCfg<D>::k
   // ---- this CTA's query tokens and K/V range ------------------------------------------
   const int a = p.cu_q[b], e = p.cu_q[b + 1];
   if (a < 0 || e < a || e > p.total_q || e - a > p.max_q_len) {  // malformed offsets: report, write nothing
-    if (blockIdx.x == 0 && g == 0 && tid == 0) raise_error(PA_DEVERR_CONTEXT);
+    if (back == 0 && g == 0 && tid == 0) raise_error(PA_DEVERR_CONTEXT);
     return;
   }
   const int T = e - a;
-  const int j0 = blockIdx.x * TQ;
+  const int tile = (T + TQ - 1) / TQ - 1 - back;
+  if (tile < 0) return;
+  const int j0 = tile * TQ;
   const int ntok = min(TQ, T - j0);
   if (ntok <= 0) return;
-  const int L = clamp_context(p, b, blockIdx.x == 0 && g == 0 && tid == 0);
+  const int L = clamp_context(p, b, back == 0 && g == 0 && tid == 0);
   const int ulo = window_start(max(L - T + j0 + 1, 0), p.window);
   const int uhi = min(L, L - T + j0 + ntok);
   const size_t row0 = (size_t)a + j0;  // q / out row of token j0

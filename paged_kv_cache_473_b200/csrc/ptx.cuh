@@ -67,6 +67,19 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
 // fence).
 __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
+// Hint: bring [addr, addr + bytes) into L2.  The range is widened to whole
+// 16-byte chunks (a chunk never straddles a page, so nothing unmapped is
+// touched).  A prefetch changes no memory contents or visibility.
+__device__ __forceinline__ void prefetch_l2(const void* addr, size_t bytes) {
+  if (bytes == 0) return;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(addr);
+  const uintptr_t lo = a & ~uintptr_t(15), hi = (a + bytes + 15) & ~uintptr_t(15);
+  for (uintptr_t x = lo; x < hi; x += (1u << 20)) {
+    const uint32_t n = (uint32_t)((hi - x) < (1u << 20) ? (hi - x) : (1u << 20));
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(x), "r"(n) : "memory");
+  }
+}
+
 // ---- TMA --------------------------------------------------------------------
 
 // 2-D tiled bulk tensor load global -> shared, completion counted in bytes on

@@ -530,6 +530,23 @@ def test_dynamic_schedule_counter_region_reads_zero_after_each_call(name, kw):
     assert pa.device_errors() == 0
 
 
+def test_in_kernel_merge_is_deterministic():
+    """At the headline shape the dynamic schedule merges each unit's partitions
+    in the decode kernel, by whichever warp arrives last; the sums run in
+    partition order, so repeated steps on the same inputs give the same bits."""
+    w = wl.WORKLOADS["tinyllama_1b"]
+    b = wl.make_batch(w, device="cuda", prefilled=True)
+    need = pa.decode_splitk_workspace_size(w.batch, w.num_q_heads, w.head_dim, b.max_context_len, 0, w.num_kv_heads)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    outs = [pa.decode_splitk(b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, w.scale,
+                             max_context_len=b.max_context_len, partition_tokens=0, workspace=ws)
+            for _ in range(12)]
+    torch.cuda.synchronize()
+    for o in outs[1:]:
+        assert torch.equal(bits(o), bits(outs[0]))
+    assert pa.device_errors() == 0
+
+
 @pytest.mark.parametrize("window", [1, 100, 1000])
 def test_dynamic_schedule_window(window):
     w, b_cpu, b = _reduced("tinyllama_1b", prefilled=True)
