@@ -57,8 +57,10 @@ namespace pa {
 
 constexpr int kMaxDynamicBatch = 2048;  // prefix arrays live in shared memory
 // Batches up to this size are scanned by every warp for itself (per-warp prefix
-// arrays, two sequences per lane); larger ones by the CTA together.
-constexpr int kWarpScanBatch = 64;
+// arrays, up to eight sequences per lane); larger ones by the CTA together.
+constexpr int kWarpScanBatch = 256;
+
+
 // The split-K workspace starts with a fixed counter region: [0] work-item
 // counter, [1] finished CTAs, then one arrival count per (sequence, kv head).
 constexpr int kMaxDynamicUnits = 65534;
@@ -90,6 +92,45 @@ __device__ __forceinline__ int seq_parts(int L, int s0, int P) { return L > s0 ?
 // The same for a partition of 2^lp tokens.
 __device__ __forceinline__ int seq_parts_sh(int L, int s0, int lp) {
   return L > s0 ? ((L + (1 << lp) - 1) >> lp) - (s0 >> lp) : 0;
+}
+
+// One warp's scan of the items before each sequence, for B <= kWarpScanBatch:
+// lane l takes sequences [c l, c l + c), c = ceil(B / 32), their lengths in
+// registers; items(b) = Hkv * (partitions of b's range); a warp shuffle scan
+// gives each lane its base.  Writes lens[b], pre[b] for b < B and pre[B].
+template <typename RangeStart>
+__device__ __forceinline__ void warp_items_scan(const DecodeParams& p, int B, int Hkv, int lp, bool report,
+                                                int* pre, int* lens, int lane, RangeStart start) {
+  constexpr uint32_t FULL = 0xffffffffu;
+  const int c = (B + 31) >> 5, b0 = lane * c;
+  int L[8], n[8];
+  int sum = 0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    L[k] = n[k] = 0;
+    if (k < c && b0 + k < B) {
+      L[k] = clamp_context(p, b0 + k, report);
+      n[k] = Hkv * seq_parts_sh(L[k], start(b0 + k, L[k]), lp);
+    }
+    sum += n[k];
+  }
+  int incl = sum;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(FULL, incl, off);
+    if (lane >= off) incl += y;
+  }
+  int base = incl - sum;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    if (k < c && b0 + k < B) {
+      lens[b0 + k] = L[k];
+      pre[b0 + k] = base;
+      base += n[k];
+    }
+  }
+  if (lane == 31) pre[B] = incl;
+  __syncwarp();
 }
 
 // First position this kernel attends for sequence b: the window start, or
@@ -306,35 +347,9 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
   // ---- items before each sequence ---------------------------------------------
   const int W = gridDim.x * NW, wg = blockIdx.x * NW + warp;
   if (warp_scan) {
-    // This warp alone: a warp scan over the items of the lengths it loaded
-    // (sequences 2l and 2l + 1 to lane l).
-    const int b0 = 2 * lane, lp = p.log2_partition;
-    int L0 = 0, L1 = 0, n0 = 0, n1 = 0;
-    if (b0 < B) {
-      L0 = clamp_context(p, b0, wg == 0);
-      n0 = Hkv * seq_parts_sh(L0, seq_start<CASCADE>(p, b0, L0), lp);
-    }
-    if (b0 + 1 < B) {
-      L1 = clamp_context(p, b0 + 1, wg == 0);
-      n1 = Hkv * seq_parts_sh(L1, seq_start<CASCADE>(p, b0 + 1, L1), lp);
-    }
-    int incl = n0 + n1;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int y = __shfl_up_sync(FULL, incl, off);
-      if (lane >= off) incl += y;
-    }
-    const int base = incl - n0 - n1;
-    if (b0 < B) {
-      lens[b0] = L0;
-      pre[b0] = base;
-    }
-    if (b0 + 1 < B) {
-      lens[b0 + 1] = L1;
-      pre[b0 + 1] = base + n0;
-    }
-    if (lane == 31) pre[B] = incl;
-    __syncwarp();
+    // This warp alone.
+    warp_items_scan(p, B, Hkv, p.log2_partition, wg == 0, pre, lens, lane,
+                    [&](int b, int L) { return seq_start<CASCADE>(p, b, L); });
   } else {
     // The CTA together: all lengths loaded at once (independent loads), then scanned.
 #pragma unroll 4

@@ -4,8 +4,9 @@
 // registers (MT = 2 at head_dim 64, 1 at 128 and 256).
 //
 // The work items, the persistent grid, the index-fixed first items and the
-// claims, and each warp's TMA ring are those of the decode kernel
-// (decode_dynamic.cuh); what differs is the attention: the R query rows of
+// claims, each warp's TMA ring, the prologue (inputs prefetched into L2 before
+// the grid-dependency wait, a per-warp length scan for small batches) are
+// those of the decode kernel (decode_dynamic.cuh); what differs is the attention: the R query rows of
 // (sequence b, kv head g) -- token j = r / G, head h = r % G, at position
 // p_j = L - T + j -- are the 16-row M dimension of the MMA
 // (attend_slice_rows, once per 16-row tile on the same K/V stage), each row
@@ -37,13 +38,16 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
   const int G = p.group, Hkv = p.hkv, P = p.partition, B = p.batch, T = p.q_len;
   constexpr int MT = rows_tiles<D>();
   const int R = T * G;  // query rows per (sequence, kv head), <= 16 MT
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
+  const bool warp_scan = B <= kWarpScanBatch;
   int* scratch = reinterpret_cast<int*>(smem + Cfg::kScratchOffset);
-  int* pre = reinterpret_cast<int*>(smem + Cfg::kPrefixOffset);  // [B+1] items before sequence b
-  int* lens = pre + B + 1;                                        // [B] clamped context lengths
+  // [B+1] items before sequence b, then [B] clamped context lengths: this
+  // warp's own arrays (warp_scan), else the CTA's.
+  int* pre = reinterpret_cast<int*>(smem + Cfg::kPrefixOffset) + (warp_scan ? warp * (2 * B + 1) : 0);
+  int* lens = pre + B + 1;
 
   pdl_launch_dependents();  // the combine may launch; it waits for this grid to finish
 
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, tid = threadIdx.x;
   const uint32_t ring = smem_addr(smem) + warp * ST * Cfg::kStageBytes;
   const uint32_t bars = smem_addr(smem + Cfg::kBarOffset) + warp * ST * 8;
   const int W = gridDim.x * NW, wg = blockIdx.x * NW + warp;
@@ -51,40 +55,56 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
 #pragma unroll
     for (int s = 0; s < ST; ++s) mbar_init(bars + 8 * s, 1);
     mbar_init_fence();
-    if (warp == 0) {
-      prefetch_tensormap(&kmap);
-      prefetch_tensormap(&vmap);
-    }
+    prefetch_tensormap(&kmap);
+    prefetch_tensormap(&vmap);
   }
+  if (tid == 0) {  // the prologue's small inputs into L2, as in the decode kernel (hints only)
+    auto share = [&](const void* base, size_t bytes) {
+      const size_t chunk = max((size_t)256, (bytes + gridDim.x - 1) / gridDim.x);
+      const size_t off = (size_t)blockIdx.x * chunk;
+      if (off < bytes) prefetch_l2(static_cast<const char*>(base) + off, min(chunk, bytes - off));
+    };
+    share(p.context_lens, (size_t)B * 4);
+    share(p.block_tables, (size_t)B * p.max_blocks * 4);
+    share(p.q, (size_t)B * T * p.hq * D * 2);
+  }
+  // Launched as a programmatic dependent: nothing above touched global memory.
+  pdl_wait();
 
   // The union of a sequence's rows' ranges starts at token 0's window start.
   auto union_start = [&](int L) { return window_start(max(L - T + 1, 0), p.window); };
 
   // ---- items before each sequence ---------------------------------------------
+  if (warp_scan) {  // this warp alone (as in the decode kernel)
+    warp_items_scan(p, B, Hkv, p.log2_partition, wg == 0, pre, lens, lane,
+                    [&](int, int L) { return union_start(L); });
+  } else {
 #pragma unroll 4
-  for (int b = tid; b < B; b += blockDim.x) lens[b] = clamp_context(p, b, blockIdx.x == 0);
-  __syncthreads();
-  int base = 0;
-  for (int b0 = 0; b0 < B; b0 += blockDim.x) {
-    const int b = b0 + tid;
-    int items = 0;
-    if (b < B) {
-      const int L = lens[b];
-      items = Hkv * seq_parts(L, union_start(L), P);
+    for (int b = tid; b < B; b += blockDim.x) lens[b] = clamp_context(p, b, blockIdx.x == 0);
+    __syncthreads();
+    int base = 0;
+    for (int b0 = 0; b0 < B; b0 += blockDim.x) {
+      const int b = b0 + tid;
+      int items = 0;
+      if (b < B) {
+        const int L = lens[b];
+        items = Hkv * seq_parts(L, union_start(L), P);
+      }
+      int total;
+      const int ex = block_exclusive_scan(items, scratch, total);
+      if (b < B) pre[b] = base + ex;
+      base += total;
     }
-    int total;
-    const int ex = block_exclusive_scan(items, scratch, total);
-    if (b < B) pre[b] = base + ex;
-    base += total;
+    if (tid == 0) pre[B] = base;
+    __syncthreads();
   }
-  if (tid == 0) pre[B] = base;
-  __syncthreads();
   const int T_items = pre[B];
   // Sequences with no position (L == 0) get zero rows; no item covers them.
-  for (int b = blockIdx.x; b < B; b += gridDim.x) {
+  // Warp wg takes sequences wg, wg + W, ...
+  for (int b = wg; b < B; b += W) {
     if (pre[b + 1] != pre[b]) continue;
     __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + (size_t)b * T * p.hq * D;
-    for (int i = tid; i < T * p.hq * D; i += blockDim.x) o[i] = __float2bfloat16_rn(0.f);
+    for (int i = lane; i < T * p.hq * D; i += 32) o[i] = __float2bfloat16_rn(0.f);
   }
 
   auto decode = [&](int t) {

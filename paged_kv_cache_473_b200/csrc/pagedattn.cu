@@ -473,7 +473,7 @@ cudaError_t launch_rows_t(DecodeParams& p, cudaStream_t st) {
   const long long rows = (long long)p.num_blocks * p.hkv * p.block_size;
   if (!cache_maps(p.k_cache, p.v_cache, D, rows, &kmap, &vmap)) return cudaErrorInvalidValue;
   auto kern = pa::decode_rows_kernel<D, NW, ST>;
-  const int smem = Cfg::smem_bytes(p.batch);
+  const int smem = Cfg::decode_smem_bytes(p.batch);
   static std::atomic<int> smem_done[64];
   cudaError_t e = set_smem_at_least(kern, smem, smem_done);
   if (e != cudaSuccess) return e;
@@ -484,7 +484,11 @@ cudaError_t launch_rows_t(DecodeParams& p, cudaStream_t st) {
   if (occ < 1) return cudaErrorInvalidConfiguration;
   p.merge_in_kernel = 0;
   p.static_items = 2;
-  return launch_ex(kern, dim3(occ * sm_count()), dim3(Cfg::kThreads), smem, st, false, kmap, vmap, p);
+  if (!pow2(p.partition)) return cudaErrorInvalidValue;  // the schedule's partitions are powers of two
+  p.log2_partition = ilog2(p.partition);
+  // A programmatic dependent of the preceding kernel: it waits for it before
+  // touching global memory.
+  return launch_ex(kern, dim3(occ * sm_count()), dim3(Cfg::kThreads), smem, st, true, kmap, vmap, p);
 }
 
 cudaError_t launch_rows(DecodeParams& p, cudaStream_t st) {
