@@ -555,3 +555,43 @@ def test_dynamic_schedule_window(window):
     torch.cuda.synchronize()
     ref, _, _ = oracle_step(b_cpu, window=window, append=False)
     assert_close(out, ref, torch.bfloat16, f"dynamic window={window}")
+
+
+# Shapes small enough that the dynamic schedule merges the partitions in the
+# decode kernel (at most 8 partitions per sequence, at most two items per
+# resident warp): the lane-order partials and the merge at every head_dim and at
+# group sizes below the 8 MMA columns (lanes holding padding columns store and
+# read nothing).  One launch per call shows that no combine kernel ran.
+IN_KERNEL_MERGE = [
+    # (num_q_heads, num_kv_heads, head_dim, batch, max context)
+    (32, 8, 128, 32, 2048),   # G = 4
+    (24, 8, 128, 32, 2048),   # G = 3
+    (16, 16, 128, 24, 2048),  # G = 1
+    (8, 4, 256, 32, 1024),    # G = 2, head_dim 256
+    (16, 8, 64, 24, 2048),    # G = 2, head_dim 64
+]
+
+
+@pytest.mark.parametrize("hq,hkv,d,batch,max_len", IN_KERNEL_MERGE)
+def test_in_kernel_merge_at_every_head_dim_and_group(hq, hkv, d, batch, max_len):
+    w = wl.WORKLOADS["llama3_8b"].replace(num_q_heads=hq, num_kv_heads=hkv, head_dim=d, prefix_share=0.0)
+    g = torch.Generator().manual_seed(77)
+    lengths = [max_len] + torch.randint(300, max_len + 1, (batch - 1,), generator=g).tolist()  # one at the bound
+    b_cpu = wl.make_batch(w, lengths=lengths, seed=77)
+    b = to_dev(b_cpu)
+    need = pa.decode_splitk_workspace_size(batch, hq, d, max_len, 0, hkv)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    outs = []
+    for _ in range(2):
+        kc, vc = b.k_cache.clone(), b.v_cache.clone()
+        out = pa.decode_step(b.q, b.k_new, b.v_new, kc, vc, b.block_tables, b.context_lens, w.scale, w.softcap,
+                             w.window, split=True, max_context_len=max_len, partition_tokens=0, workspace=ws)
+        assert pa.last_launch_count() == 1  # merged in the decode kernel
+        torch.cuda.synchronize()
+        assert int(ws[:COUNTER_BYTES].view(torch.int32).abs().sum()) == 0
+        outs.append(out)
+    assert torch.equal(bits(outs[0]), bits(outs[1]))
+    ref, kc_ref, vc_ref = oracle_step(b_cpu)
+    assert torch.equal(bits(kc), bits(kc_ref)) and torch.equal(bits(vc), bits(vc_ref))
+    assert_close(outs[0], ref, torch.bfloat16, f"in-kernel merge G={hq // hkv} D={d}")
+    assert pa.device_errors() == 0
