@@ -282,6 +282,7 @@ class Runner:
         self.kv_bytes = wl.kv_bytes(b)
         self.kv_bytes_unique = wl.kv_bytes(b, unique=True)
         self.launches_per_step = 0
+        self.schedule = "none"  # the library's schedule for the decode (pa_last_decode_schedule)
 
     def inputs(self):
         b = self.batch
@@ -316,6 +317,7 @@ class Runner:
         if ev is not None:
             ev[0].record()
         n += self.decode(r, x)
+        self.schedule = self.pa.last_decode_schedule()
         if ev is not None:
             ev[1].record()
         self.launches_per_step = n
@@ -712,14 +714,23 @@ def workload_config(w: wl.Workload, batch: wl.Batch) -> dict:
     }
 
 
+SCHEDULE_NAMES = {
+    "dynamic_merged": "work queue: warps claim (sequence, kv head, partition) items, merged in the decode kernel",
+    "dynamic": "work queue: warps claim (sequence, kv head, partition) items, then the combine kernel",
+    "grid": "one CTA per (partition, kv head, sequence), then the combine kernel",
+    "single": "one CTA per (sequence, kv head)",
+}
+
+
 def describe_path(runner: Runner, kernel: str, l2_detail: str) -> dict:
     """How the library arm ran the workload (kept out of ``config``, which
     names only the workload)."""
     path = ("pa_decode_step" if runner.fused else "pa_write_kv + " + ("pa_decode_splitk" if runner.split else
                                                                       "pa_decode"))
-    path += ((" (split-K, dynamic work queue)" if runner.partition == 0 else
+    path += ((" (split-K, library schedule)" if runner.partition == 0 else
               f" (split-K, partition {runner.partition})") if runner.split else " (one CTA per sequence, kv head)")
-    return {"call": path, "kernel": kernel, "l2": l2_detail}
+    return {"call": path, "schedule": SCHEDULE_NAMES.get(runner.schedule, runner.schedule), "kernel": kernel,
+            "l2": l2_detail}
 
 
 def op_duration(runner: "Runner", total_ms: float, K: int, dec_ms: float):
@@ -830,6 +841,7 @@ def shape_summary(w: wl.Workload, rank: int, kernel: str, K: int, W: int, world:
         "kv_bytes": r["logical_bytes_per_launch"],
         "traffic": r["traffic"],
         "path": d["path"]["call"],
+        "schedule": d["path"]["schedule"],
     }
 
 

@@ -79,6 +79,15 @@ typedef enum {
  * CUDA-core kernel for fp32.  MMA is bf16 only. */
 typedef enum { PA_KERNEL_AUTO = 0, PA_KERNEL_CUDA_CORE = 1, PA_KERNEL_MMA = 2 } pa_kernel_t;
 
+/* Decode schedules (see pa_decode_splitk), as reported by pa_last_decode_schedule. */
+typedef enum {
+  PA_SCHEDULE_NONE = 0,
+  PA_SCHEDULE_SINGLE = 1,          /* one CTA per (sequence, kv head), no split */
+  PA_SCHEDULE_GRID = 2,            /* one CTA per (partition, kv head, sequence), then the combine */
+  PA_SCHEDULE_DYNAMIC = 3,         /* warp work queue, then the combine */
+  PA_SCHEDULE_DYNAMIC_MERGED = 4   /* warp work queue, partitions merged in the same kernel */
+} pa_schedule_t;
+
 /* Bits of the device error word. */
 enum {
   PA_DEVERR_SLOT = 1u,       /* write_kv: slot >= num_blocks * block_size (row skipped) */
@@ -365,6 +374,12 @@ const char* pa_error_string(pa_status_t status);
 /* Number of kernels the last successful call on this host thread launched
  * (0 after a failed call).  For accounting in benchmarks. */
 int32_t pa_last_launch_count(void);
+
+/* The schedule the last decode call (pa_decode, pa_decode_splitk,
+ * pa_decode_splitk_noalloc, pa_decode_step) on this host thread ran: one of
+ * pa_schedule_t, PA_SCHEDULE_NONE after a failed call or a call that launched
+ * nothing.  For tests and benchmarks that report which path ran. */
+int32_t pa_last_decode_schedule(void);
 
 #ifdef __cplusplus
 }

@@ -30,6 +30,7 @@ from ._binding import (  # noqa: F401
     check_bounded_wait,
     device_errors,
     error_string,
+    last_decode_schedule,
     last_launch_count,
     prefill,
     write_kv,
@@ -61,6 +62,7 @@ __all__ = [
     "check_bounded_wait",
     "device_errors",
     "error_string",
+    "last_decode_schedule",
     "last_launch_count",
     "prefill",
     "PagedAttnError",

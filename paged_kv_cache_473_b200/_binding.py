@@ -23,6 +23,8 @@ from . import build as _build
 
 PA_F32, PA_BF16 = 0, 1
 PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_WORKSPACE, PA_ERR_CUDA = 0, 1, 2, 3, 4
+# pa_schedule_t (include/pagedattn.h)
+SCHEDULES = {0: "none", 1: "single", 2: "grid", 3: "dynamic", 4: "dynamic_merged"}
 KERNELS = {"auto": 0, "cuda_core": 1, "mma": 2}
 DEVERR_SLOT, DEVERR_BLOCK, DEVERR_CONTEXT, DEVERR_TIMEOUT, DEVERR_LAYOUT = 1, 2, 4, 8, 16
 
@@ -112,6 +114,8 @@ def _load_library() -> ctypes.CDLL:
     lib.pa_error_string.restype = ctypes.c_char_p
     lib.pa_last_launch_count.argtypes = []
     lib.pa_last_launch_count.restype = _c_i32
+    lib.pa_last_decode_schedule.argtypes = []
+    lib.pa_last_decode_schedule.restype = _c_i32
     return lib
 
 
@@ -476,3 +480,9 @@ def check_bounded_wait(limit_ns: int = 1_000_000, stream=None) -> None:
 
 def last_launch_count() -> int:
     return _lib().pa_last_launch_count()
+
+
+def last_decode_schedule() -> str:
+    """Name of the schedule the last decode call on this thread ran
+    ("dynamic_merged", "dynamic", "grid", "single", or "none")."""
+    return SCHEDULES.get(_lib().pa_last_decode_schedule(), "unknown")

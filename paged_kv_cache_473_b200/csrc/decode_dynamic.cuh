@@ -10,7 +10,10 @@
 // and the whole GPU finishes together.  A warp runs an
 // item alone: it streams the item's 16-token slices through its own ST-deep
 // ring of TMA-filled shared-memory stages, keeps the online-softmax state in
-// registers (attend_slice), and at the end writes either the normalised output
+// registers (attend_slice; two slices per softmax step, attend_pair, where the
+// ring has at least four stages: a warp's time per slice is its own dependent
+// latency, not the memory's, so halving the softmax steps shortens it), and at
+// the end writes either the normalised output
 // (the item is the sequence's only partition) or its partial state (m, l, o)
 // to the [B][Hq][max_parts] workspace, straight from registers.  No barrier
 // joins the warps of a CTA after the prologue, so an SM holds many independent
@@ -292,6 +295,7 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
                           const DecodeParams p) {
   using Cfg = DynCfg<D, NW, ST>;
   constexpr uint32_t FULL = 0xffffffffu;
+  constexpr bool kPairs = ST >= 4;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int G = p.group, Hkv = p.hkv, P = p.partition, B = p.batch;
@@ -498,9 +502,13 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
         knew = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.k_new) + off);
         vnew = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.v_new) + off);
       }
-      for (int ck = 0; ck < ci.n; ++ck) {
+      for (int ck = 0; ck < ci.n;) {
         fill();
+        // Two slices per step where the ring is deep enough to keep loading
+        // while both are attended.
+        const int step = (kPairs && ck + 1 < ci.n) ? 2 : 1;
         bool ok = mbar_wait_bounded(bars + 8 * (gc % ST), (gc / ST) & 1, kWaitLimitNs);
+        if (step == 2) ok = ok && mbar_wait_bounded(bars + 8 * ((gc + 1) % ST), ((gc + 1) / ST) & 1, kWaitLimitNs);
         ok = __all_sync(FULL, ok);
         if (!ok) {
           aborted = true;
@@ -508,9 +516,12 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
         }
         const uint32_t kbase = ring + (gc % ST) * Cfg::kStageBytes;
         const uint32_t vbase = kbase + Cfg::kSliceBytes;
-        if (append_item && ck == ci.n - 1) {
+        const uint32_t kbase1 = ring + ((gc + 1) % ST) * Cfg::kStageBytes;
+        const uint32_t vbase1 = kbase1 + Cfg::kSliceBytes;
+        if (append_item && ck + step == ci.n) {
           // The item's last slice holds position L-1: append the new rows.
-          overwrite_slice_row<D>(kbase, vbase, (ci.L - 1) & (kSliceTokens - 1), knew, vnew, lane);
+          overwrite_slice_row<D>(step == 2 ? kbase1 : kbase, step == 2 ? vbase1 : vbase,
+                                 (ci.L - 1) & (kSliceTokens - 1), knew, vnew, lane);
           if (lane < D / 8) {
             const int phys = p.block_tables[(size_t)ci.b * p.max_blocks + ((ci.L - 1) >> p.log2_bs)];
             if (phys >= 0 && phys < p.num_blocks) {
@@ -520,9 +531,15 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
             }
           }
         }
-        attend_slice<D>(st, qf, kbase, vbase, (ci.j0 + ck) * kSliceTokens, ci.lo, ci.hi, qk_scale, p, lane);
+        if (step == 2) {
+          attend_pair<D>(st, qf, kbase, vbase, kbase1, vbase1, (ci.j0 + ck) * kSliceTokens, ci.lo, ci.hi, qk_scale,
+                         p, lane);
+        } else {
+          attend_slice<D>(st, qf, kbase, vbase, (ci.j0 + ck) * kSliceTokens, ci.lo, ci.hi, qk_scale, p, lane);
+        }
         __syncwarp();
-        ++gc;
+        gc += step;
+        ck += step;
       }
       if (aborted) break;
       fill();  // keep loading the next item while this one is stored

@@ -249,6 +249,113 @@ __device__ __forceinline__ void attend_slice(WarpAttn<D>& st, const uint32_t (&q
   }
 }
 
+// Attend two consecutive slices, tokens [t0, t0+16) at kbase0/vbase0 and
+// [t0+16, t0+32) at kbase1/vbase1, in one online-softmax step: the same
+// arithmetic as attend_slice over a 32-token block (one running-maximum
+// update, one rescale of o, one shuffle reduction for both slices), with the
+// two S^T products independent of each other.  Only tokens in [lo, hi) count;
+// each slice must hold at least one of them.
+template <int D>
+__device__ __forceinline__ void attend_pair(WarpAttn<D>& st, const uint32_t (&qf)[D / 16][2], uint32_t kbase0,
+                                            uint32_t vbase0, uint32_t kbase1, uint32_t vbase1, int t0, int lo,
+                                            int hi, float qk_scale, const DecodeParams& p, int lane) {
+  constexpr uint32_t FULL = 0xffffffffu;
+  const uint32_t k_lane = ((lane & 7) | (lane & 8)) * 128;
+  const uint32_t v_lane = ((lane & 7) | ((lane >> 4) << 3)) * 128;
+  const uint32_t k_sub = lane >> 4, v_sub = (lane >> 3) & 1, swz = lane & 7;
+
+  // ---- S^T = K Q^T for both slices ---------------------------------------------
+  float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * kPanelBytes + k_lane + (((((kk & 3) << 1) | k_sub) ^ swz) << 4);
+    uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
+    ldsm_x4(kbase0 + off, a0, a1, a2, a3);
+    ldsm_x4(kbase1 + off, b0, b1, b2, b3);
+    mma_bf16_16816(sc[0], a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+    mma_bf16_16816(sc[1], b0, b1, b2, b3, qf[kk][0], qf[kk][1]);
+  }
+  // sc[s][0], sc[s][1]: token t0 + 16 s + lane/4, heads n0, n0+1; [2], [3]: token + 8.
+  float x[2][4];
+#pragma unroll
+  for (int s2 = 0; s2 < 2; ++s2) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float v = sc[s2][e] * qk_scale;
+      if (p.use_softcap) v = p.softcap * tanhf(v * p.inv_softcap) * kLog2e;
+      x[s2][e] = v;
+    }
+  }
+  uint32_t keep_lo[2] = {0xffffffffu, 0xffffffffu}, keep_hi[2] = {0xffffffffu, 0xffffffffu};
+  bool partial[2];
+#pragma unroll
+  for (int s2 = 0; s2 < 2; ++s2) {
+    const int ts = t0 + s2 * kSliceTokens;
+    partial[s2] = (ts < lo) || (ts + kSliceTokens > hi);
+    if (partial[s2]) {
+      const int ta = ts + (lane >> 2), tb = ta + 8;
+      if (!(ta >= lo && ta < hi)) x[s2][0] = x[s2][1] = -CUDART_INF_F;
+      if (!(tb >= lo && tb < hi)) x[s2][2] = x[s2][3] = -CUDART_INF_F;
+      const int tc = ts + 2 * (lane & 3);
+      auto ok = [&](int t) { return t >= lo && t < hi; };
+      keep_lo[s2] = (ok(tc) ? 0x0000ffffu : 0u) | (ok(tc + 1) ? 0xffff0000u : 0u);
+      keep_hi[s2] = (ok(tc + 8) ? 0x0000ffffu : 0u) | (ok(tc + 9) ? 0xffff0000u : 0u);
+    }
+  }
+
+  // ---- online softmax over the 32 tokens ---------------------------------------
+  float mx0 = fmaxf(fmaxf(x[0][0], x[0][2]), fmaxf(x[1][0], x[1][2]));
+  float mx1 = fmaxf(fmaxf(x[0][1], x[0][3]), fmaxf(x[1][1], x[1][3]));
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, off));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, off));
+  }
+  const float mn0 = fmaxf(st.m0, mx0), mn1 = fmaxf(st.m1, mx1);
+  const float al0 = exp2f(st.m0 - mn0), al1 = exp2f(st.m1 - mn1);
+  st.m0 = mn0;
+  st.m1 = mn1;
+  uint32_t plo[2], phi[2];
+#pragma unroll
+  for (int s2 = 0; s2 < 2; ++s2) {
+    plo[s2] = pack_bf16x2(exp2f(x[s2][0] - mn0), exp2f(x[s2][1] - mn1));
+    phi[s2] = pack_bf16x2(exp2f(x[s2][2] - mn0), exp2f(x[s2][3] - mn1));
+  }
+  st.l0 = st.l0 * al0 + ((bf16_lo(plo[0]) + bf16_lo(phi[0])) + (bf16_lo(plo[1]) + bf16_lo(phi[1])));
+  st.l1 = st.l1 * al1 + ((bf16_hi(plo[0]) + bf16_hi(phi[0])) + (bf16_hi(plo[1]) + bf16_hi(phi[1])));
+#pragma unroll
+  for (int mt = 0; mt < D / 16; ++mt) {
+    st.o[mt][0] *= al0;
+    st.o[mt][1] *= al1;
+    st.o[mt][2] *= al0;
+    st.o[mt][3] *= al1;
+  }
+  uint32_t pb[2][2];
+#pragma unroll
+  for (int s2 = 0; s2 < 2; ++s2) {
+    pb[s2][0] = movmatrix_trans(plo[s2]);
+    pb[s2][1] = movmatrix_trans(phi[s2]);
+  }
+
+  // ---- O^T += V^T P^T, one k-step per slice -----------------------------------------
+#pragma unroll
+  for (int mt = 0; mt < D / 16; ++mt) {
+    const uint32_t off = (mt >> 2) * kPanelBytes + v_lane + (((((mt & 3) << 1) | v_sub) ^ swz) << 4);
+#pragma unroll
+    for (int s2 = 0; s2 < 2; ++s2) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4_trans((s2 ? vbase1 : vbase0) + off, a0, a1, a2, a3);
+      if (partial[s2]) {
+        a0 &= keep_lo[s2];
+        a1 &= keep_lo[s2];
+        a2 &= keep_hi[s2];
+        a3 &= keep_hi[s2];
+      }
+      mma_bf16_16816(st.o[mt], a0, a1, a2, a3, pb[s2][0], pb[s2][1]);
+    }
+  }
+}
+
 // ---- query rows as the MMA M dimension -------------------------------------------
 //
 // For several query tokens per sequence (multi-query rows) with R = T*G <= 16

@@ -29,6 +29,7 @@ namespace {
 using pa::DecodeParams;
 
 thread_local int32_t t_last_launches = 0;
+thread_local int32_t t_last_schedule = PA_SCHEDULE_NONE;
 
 constexpr int kNoSplitPartition = 1 << 30;
 constexpr int kMaxPartsPerSeq = 8192;
@@ -642,6 +643,7 @@ struct DecodeCall {
 };
 
 pa_status_t run_decode(const DecodeCall& c) {
+  t_last_schedule = PA_SCHEDULE_NONE;
   const Shape& s = c.shape;
   pa_status_t st = check_decode_args(c.q, c.k_cache, c.v_cache, c.block_tables, c.context_lens, s, c.softcap,
                                      c.out, c.dtype, c.kernel);
@@ -702,6 +704,7 @@ pa_status_t run_decode(const DecodeCall& c) {
       e = c.append ? launch_dynamic<true>(p, c.stream) : launch_dynamic<false>(p, c.stream);
       if (e != cudaSuccess) return PA_ERR_CUDA;
       t_last_launches = 1;
+      t_last_schedule = p.merge_in_kernel ? PA_SCHEDULE_DYNAMIC_MERGED : PA_SCHEDULE_DYNAMIC;
       if (!p.merge_in_kernel && parts > 1) {
         e = launch_combine<__nv_bfloat16>(p, c.stream);
         if (e != cudaSuccess) return PA_ERR_CUDA;
@@ -713,6 +716,7 @@ pa_status_t run_decode(const DecodeCall& c) {
     e = c.append ? launch_decode<true, true>(p, c.dtype, c.kernel, grid, c.stream)
                  : launch_decode<true, false>(p, c.dtype, c.kernel, grid, c.stream);
     if (e != cudaSuccess) return PA_ERR_CUDA;
+    t_last_schedule = PA_SCHEDULE_GRID;
     if (parts > 1) {
       e = c.dtype == PA_BF16 ? launch_combine<__nv_bfloat16>(p, c.stream) : launch_combine<float>(p, c.stream);
       if (e != cudaSuccess) return PA_ERR_CUDA;
@@ -726,6 +730,7 @@ pa_status_t run_decode(const DecodeCall& c) {
                  : launch_decode<false, false>(p, c.dtype, c.kernel, grid, c.stream);
     if (e != cudaSuccess) return PA_ERR_CUDA;
     t_last_launches = 1;
+    t_last_schedule = PA_SCHEDULE_SINGLE;
   }
   return PA_OK;
 }
@@ -1195,5 +1200,7 @@ const char* pa_error_string(pa_status_t status) {
 }
 
 int32_t pa_last_launch_count(void) { return t_last_launches; }
+
+int32_t pa_last_decode_schedule(void) { return t_last_schedule; }
 
 }  // extern "C"

@@ -29,7 +29,7 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ["pa_write_kv", "pa_decode", "pa_decode_splitk", "pa_decode_splitk_workspace_size",
-              "pa_decode_splitk_partition", "pa_device_errors", "pa_error_string", "pa_last_launch_count",
+              "pa_decode_splitk_partition", "pa_device_errors", "pa_error_string", "pa_last_launch_count", "pa_last_decode_schedule",
               "pa_decode_step", "pa_decode_splitk_noalloc", "pa_decode_multi", "pa_decode_multi_workspace_size",
               "pa_prefill", "pa_copy_blocks", "pa_bm_create", "pa_bm_append_slots", "pa_bm_block_tables",
               "pa_decode_cascade", "pa_decode_cascade_workspace_size"]:

@@ -435,12 +435,14 @@ def test_dynamic_schedule_short_and_empty_sequences(lengths):
 
 
 def test_dynamic_schedule_many_units_per_cta():
-    """Many short sequences: thousands of items, prefix arrays of a large batch."""
+    """Many short sequences: thousands of items, prefix arrays of a large batch
+    (the CTA-wide length scan)."""
     w = wl.WORKLOADS["llama3_8b"].replace(prefix_share=0.0, lengths=("uniform", 1, 40))
     b_cpu = wl.make_batch(w, batch=2000, prefilled=True)
     b = to_dev(b_cpu)
     out = pa.decode_splitk(b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, w.scale,
                            max_context_len=b.max_context_len, partition_tokens=0)
+    assert pa.last_decode_schedule() in ("dynamic", "dynamic_merged")
     torch.cuda.synchronize()
     rows = [(i, h) for i in range(0, 2000, 37) for h in (0, 13, 31)]
     ref = oracle.decode(b_cpu.q, b_cpu.k_cache, b_cpu.v_cache, b_cpu.block_tables, b_cpu.context_lens, w.scale,
@@ -499,15 +501,15 @@ def test_dynamic_schedule_counters_return_to_zero():
     assert pa.device_errors() == 0
 
 
-@pytest.mark.parametrize("name,kw", [
-    ("tinyllama_1b", dict(batch=24)),  # fixed items cover the work, the last partial merges
-    ("llama3_8b", dict(batch=64)),     # more items than 2 per warp (claims), combine kernel
+@pytest.mark.parametrize("name,kw,max_ctx,schedule", [
+    ("tinyllama_1b", dict(batch=48), None, "dynamic_merged"),  # fixed items cover the work, the last partial merges
+    ("llama3_8b", dict(batch=64), None, "dynamic"),           # more items than 2 per warp (claims), combine kernel
     # at most 8 partitions but more than 2 items per warp: claims and the combine kernel
-    ("gemma2_2b", dict(batch=256)),
-    ("llama3_8b", dict(batch=128, max_len=2048)),
-    ("tinyllama_1b", dict(batch=256)),
+    ("gemma2_2b", dict(batch=256), None, "dynamic"),
+    ("llama3_8b", dict(batch=128, max_len=2048), None, "dynamic"),
+    ("tinyllama_1b", dict(batch=256), None, "dynamic"),
 ])
-def test_dynamic_schedule_counter_region_reads_zero_after_each_call(name, kw):
+def test_dynamic_schedule_counter_region_reads_zero_after_each_call(name, kw, max_ctx, schedule):
     """Whichever way the partitions are merged, and whether or not warps claim
     items from the work counter, the step matches the oracle and the
     workspace's counter region is all zero when the call ends (the next call
@@ -515,14 +517,14 @@ def test_dynamic_schedule_counter_region_reads_zero_after_each_call(name, kw):
     w = wl.WORKLOADS[name]
     bc = wl.make_batch(w, prefilled=False, **kw)
     b = to_dev(bc)
-    need = pa.decode_splitk_workspace_size(bc.q.shape[0], w.num_q_heads, w.head_dim, b.max_context_len, 0,
-                                           w.num_kv_heads)
+    mx = max_ctx or b.max_context_len
+    need = pa.decode_splitk_workspace_size(bc.q.shape[0], w.num_q_heads, w.head_dim, mx, 0, w.num_kv_heads)
     ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
     kc, vc = b.k_cache.clone(), b.v_cache.clone()
     for _ in range(2):
         out = pa.decode_step(b.q, b.k_new, b.v_new, kc, vc, b.block_tables, b.context_lens, w.scale, w.softcap,
-                             w.window, split=True, max_context_len=b.max_context_len, partition_tokens=0,
-                             workspace=ws)
+                             w.window, split=True, max_context_len=mx, partition_tokens=0, workspace=ws)
+        assert pa.last_decode_schedule() == schedule
         torch.cuda.synchronize()
         assert int(ws[:COUNTER_BYTES].view(torch.int32).abs().sum()) == 0
     ref, _, _ = oracle_step(bc)
@@ -530,17 +532,21 @@ def test_dynamic_schedule_counter_region_reads_zero_after_each_call(name, kw):
     assert pa.device_errors() == 0
 
 
-def test_in_kernel_merge_is_deterministic():
-    """At the headline shape the dynamic schedule merges each unit's partitions
-    in the decode kernel, by whichever warp arrives last; the sums run in
-    partition order, so repeated steps on the same inputs give the same bits."""
+@pytest.mark.parametrize("batch,schedule", [(64, "dynamic_merged"), (48, "dynamic_merged")])
+def test_in_kernel_merge_is_deterministic(batch, schedule):
+    """At the headline shape (64 sequences, and at 48) the dynamic schedule
+    merges each unit's partitions in the decode kernel, by whichever warp
+    arrives last; the sums run in partition order, so repeated steps on the
+    same inputs give the same bits."""
     w = wl.WORKLOADS["tinyllama_1b"]
-    b = wl.make_batch(w, device="cuda", prefilled=True)
-    need = pa.decode_splitk_workspace_size(w.batch, w.num_q_heads, w.head_dim, b.max_context_len, 0, w.num_kv_heads)
+    b = wl.make_batch(w, device="cuda", prefilled=True, batch=batch)
+    need = pa.decode_splitk_workspace_size(batch, w.num_q_heads, w.head_dim, b.max_context_len, 0, w.num_kv_heads)
     ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
-    outs = [pa.decode_splitk(b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, w.scale,
-                             max_context_len=b.max_context_len, partition_tokens=0, workspace=ws)
-            for _ in range(12)]
+    outs = []
+    for _ in range(12):
+        outs.append(pa.decode_splitk(b.q, b.k_cache, b.v_cache, b.block_tables, b.context_lens, w.scale,
+                                     max_context_len=b.max_context_len, partition_tokens=0, workspace=ws))
+        assert pa.last_decode_schedule() == schedule
     torch.cuda.synchronize()
     for o in outs[1:]:
         assert torch.equal(bits(o), bits(outs[0]))
@@ -564,9 +570,9 @@ def test_dynamic_schedule_window(window):
 # read nothing).  One launch per call shows that no combine kernel ran.
 IN_KERNEL_MERGE = [
     # (num_q_heads, num_kv_heads, head_dim, batch, max context)
-    (32, 8, 128, 32, 2048),   # G = 4
-    (24, 8, 128, 32, 2048),   # G = 3
-    (16, 16, 128, 24, 2048),  # G = 1
+    (32, 8, 128, 24, 512),    # G = 4
+    (24, 8, 128, 24, 512),    # G = 3
+    (16, 16, 128, 12, 512),   # G = 1
     (8, 4, 256, 32, 1024),    # G = 2, head_dim 256
     (16, 8, 64, 24, 2048),    # G = 2, head_dim 64
 ]
@@ -576,7 +582,7 @@ IN_KERNEL_MERGE = [
 def test_in_kernel_merge_at_every_head_dim_and_group(hq, hkv, d, batch, max_len):
     w = wl.WORKLOADS["llama3_8b"].replace(num_q_heads=hq, num_kv_heads=hkv, head_dim=d, prefix_share=0.0)
     g = torch.Generator().manual_seed(77)
-    lengths = [max_len] + torch.randint(300, max_len + 1, (batch - 1,), generator=g).tolist()  # one at the bound
+    lengths = [max_len] + torch.randint(max_len // 2, max_len + 1, (batch - 1,), generator=g).tolist()  # one at the bound
     b_cpu = wl.make_batch(w, lengths=lengths, seed=77)
     b = to_dev(b_cpu)
     need = pa.decode_splitk_workspace_size(batch, hq, d, max_len, 0, hkv)
@@ -587,6 +593,7 @@ def test_in_kernel_merge_at_every_head_dim_and_group(hq, hkv, d, batch, max_len)
         out = pa.decode_step(b.q, b.k_new, b.v_new, kc, vc, b.block_tables, b.context_lens, w.scale, w.softcap,
                              w.window, split=True, max_context_len=max_len, partition_tokens=0, workspace=ws)
         assert pa.last_launch_count() == 1  # merged in the decode kernel
+        assert pa.last_decode_schedule() == "dynamic_merged"
         torch.cuda.synchronize()
         assert int(ws[:COUNTER_BYTES].view(torch.int32).abs().sum()) == 0
         outs.append(out)
@@ -594,4 +601,23 @@ def test_in_kernel_merge_at_every_head_dim_and_group(hq, hkv, d, batch, max_len)
     ref, kc_ref, vc_ref = oracle_step(b_cpu)
     assert torch.equal(bits(kc), bits(kc_ref)) and torch.equal(bits(vc), bits(vc_ref))
     assert_close(outs[0], ref, torch.bfloat16, f"in-kernel merge G={hq // hkv} D={d}")
+    assert pa.device_errors() == 0
+
+
+@pytest.mark.parametrize("window", [0, 100, 333, 1000])
+def test_dynamic_queue_merged_by_the_combine_kernel_with_windows(window):
+    """A step too large for the in-kernel merge: the dynamic queue's partials go
+    through the combine kernel.  A window makes a sequence's first item start
+    inside a partition and leaves the partitions before it without tokens."""
+    w = wl.WORKLOADS["llama3_8b"].replace(prefix_share=0.0)
+    b_cpu = wl.make_batch(w, batch=16, max_len=3000, seed=91)
+    b = to_dev(b_cpu)
+    kc, vc = b.k_cache.clone(), b.v_cache.clone()
+    out = pa.decode_step(b.q, b.k_new, b.v_new, kc, vc, b.block_tables, b.context_lens, w.scale, w.softcap, window,
+                         split=True, max_context_len=b.max_context_len, partition_tokens=0)
+    assert pa.last_launch_count() == 2  # decode and combine
+    assert pa.last_decode_schedule() == "dynamic"
+    torch.cuda.synchronize()
+    ref, _, _ = oracle_step(b_cpu, window=window)
+    assert_close(out, ref, torch.bfloat16, f"dynamic queue + combine, window={window}")
     assert pa.device_errors() == 0

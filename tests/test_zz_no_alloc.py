@@ -43,14 +43,14 @@ def _call_noalloc(b, w, out, partition_tokens, max_ctx):
 
 # (workload, batch size / length bound, partition): how the partitions are merged
 CASES = [
-    ("tinyllama_1b", dict(batch=16), 0),                # dynamic schedule, merged inside the decode kernel
-    ("llama3_8b", dict(batch=48, max_len=3000), 0),     # dynamic schedule, merged by the combine kernel
-    ("tinyllama_1b", dict(batch=16), 128),              # fixed partition grid and the combine kernel
+    ("tinyllama_1b", dict(batch=48), 0, "dynamic_merged"),          # work queue, merged inside the decode kernel
+    ("llama3_8b", dict(batch=24, max_len=3000), 0, "dynamic"),      # work queue, merged by the combine kernel
+    ("tinyllama_1b", dict(batch=16), 128, "grid"),                  # fixed partition grid and the combine kernel
 ]
 
 
-@pytest.mark.parametrize("name,kw,partition_tokens", CASES)
-def test_noalloc_equals_the_workspace_entry_point_and_the_oracle_on_two_calls(name, kw, partition_tokens):
+@pytest.mark.parametrize("name,kw,partition_tokens,schedule", CASES)
+def test_noalloc_equals_the_workspace_entry_point_and_the_oracle_on_two_calls(name, kw, partition_tokens, schedule):
     w = wl.WORKLOADS[name].replace(prefix_share=0.0)
     pa.device_errors(clear=True)
     for call, seed in enumerate((w.seed, w.seed + 1)):  # different inputs on the second call
@@ -64,6 +64,7 @@ def test_noalloc_equals_the_workspace_entry_point_and_the_oracle_on_two_calls(na
                                w.window, max_context_len=max_ctx, partition_tokens=partition_tokens)
         out = torch.full_like(b.q, float("nan"))
         assert _call_noalloc(b, w, out, partition_tokens, max_ctx) == bnd.PA_OK
+        assert pa.last_decode_schedule() == schedule
         torch.cuda.synchronize()
         assert torch.equal(bits(out), bits(ref)), f"call {call}: differs from pa_decode_splitk"
         want = oracle.decode(b_cpu.q, b_cpu.k_cache, b_cpu.v_cache, b_cpu.block_tables, b_cpu.context_lens, w.scale,
