@@ -22,8 +22,8 @@
 // full across item boundaries.
 //
 // Merge (small steps): each (sequence, kv head) unit has an arrival counter in
-// the workspace.  A warp that stored a partial publishes it (release fence)
-// and counts it; the warp that brings the count to the unit's number of
+// the workspace.  A warp that stored a partial publishes and counts it with
+// one acquire-release atomic; the warp that brings the count to the unit's number of
 // partitions reads every partial back through L2 in partition order (the same
 // bits whichever warp merges), merges them (log-sum-exp) and writes the
 // normalised output rows; it returns the counter to zero.  (Measured on
@@ -576,16 +576,19 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
           }
         }
       } else if (!ci.whole) {  // merged in this kernel
-        // Publish the partial, then count it (release); the unit's last
-        // partial merges them all (acquire).
+        // Publish the partial and count it with one acquire-release atomic
+        // (lane 0, after the warp barrier that orders every lane's stores
+        // before it); the unit's last partial merges them all, its lanes'
+        // loads ordered after the acquire by a second warp barrier.  (One
+        // atomic with both orderings measured 0.6 us shorter on B200 than a
+        // release fence followed by a relaxed count and an acquire fence.)
         store_partial_lanes<D>(st, p, row0, ci.part, G, lane);
-        fence_acq_rel_gpu();
         __syncwarp();
         int* cnt = p.unit_count + (size_t)ci.b * Hkv + ci.g;
         int last = 0;
-        if (lane == 0) last = atomicAdd(cnt, 1) == ci.parts - 1;
+        if (lane == 0) last = atom_add_acq_rel_gpu(cnt, 1) == ci.parts - 1;
         if (__shfl_sync(FULL, last, 0)) {
-          fence_acq_rel_gpu();
+          __syncwarp();
           merge_lanes<D>(st, p, row0, ci.pb, ci.parts, ci.part - ci.pb, G, lane);
           write_rows = true;
           if (lane == 0) *cnt = 0;  // every partial of the unit has arrived: ready for the next call

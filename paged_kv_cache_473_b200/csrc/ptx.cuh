@@ -61,11 +61,15 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
   }
 }
 
-// Acquire-release fence at GPU scope: before a relaxed atomic it publishes
-// this thread's earlier writes (release); after one it orders the reads that
-// follow (acquire).  Lighter than __threadfence (a sequentially consistent
-// fence).
-__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+// atomicAdd at GPU scope with acquire-release semantics: the writes ordered
+// before it are visible to a thread that reads its result with acquire
+// semantics, and the reads that follow it see the writes released before the
+// values it read.  Returns the old value.
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int* addr, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v) : "memory");
+  return old;
+}
 
 // Hint: bring [addr, addr + bytes) into L2.  The range is widened to whole
 // 16-byte chunks (a chunk never straddles a page, so nothing unmapped is
