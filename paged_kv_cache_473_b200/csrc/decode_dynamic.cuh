@@ -192,7 +192,7 @@ __device__ __forceinline__ void store_partial_lanes(const WarpAttn<D>& st, const
 // merging warp's own partition `own` has been stored like the others; its
 // (m, l) come from registers.
 // The loads of kB partials are issued before any is used (one L2 round trip
-// per batch).
+// per batch), the first batch together with the (m, l) loads.
 template <int D>
 __device__ __forceinline__ void merge_lanes(WarpAttn<D>& st, const DecodeParams& p, size_t row0, int pb, int n,
                                             int own, int G, int lane) {
@@ -215,21 +215,10 @@ __device__ __forceinline__ void merge_lanes(WarpAttn<D>& st, const DecodeParams&
     c[i] = i == own ? make_float2(st.m1, st.l1)
                     : (other && h1 ? __ldcg(ml + p.max_parts + i) : make_float2(-CUDART_INF_F, 0.f));
   }
-  float M0 = -CUDART_INF_F, M1 = -CUDART_INF_F;
-#pragma unroll
-  for (int i = 0; i < kMaxMergeParts; ++i) {
-    M0 = fmaxf(M0, a[i].x);
-    M1 = fmaxf(M1, c[i].x);
-  }
-  st.l0 = st.l1 = 0.f;
-#pragma unroll
-  for (int mt = 0; mt < D / 16; ++mt) st.o[mt][0] = st.o[mt][1] = st.o[mt][2] = st.o[mt][3] = 0.f;
   const float* base0 = p.ws_o + slot0 * D + r * (D / 8);
   const float* base1 = p.ws_o + (slot0 + p.max_parts) * D + r * (D / 8);
-#pragma unroll
-  for (int i0 = 0; i0 < kMaxMergeParts; i0 += kB) {
-    if (i0 >= n) break;
-    float4 x0[kB][V], x1[kB][V];
+  float4 x0[kB][V], x1[kB][V];
+  auto load_batch = [&](int i0) {
 #pragma unroll
     for (int j = 0; j < kB; ++j) {
       const int i = i0 + j;
@@ -241,6 +230,21 @@ __device__ __forceinline__ void merge_lanes(WarpAttn<D>& st, const DecodeParams&
         x1[j][k] = i < n && h1 ? __ldcg(s1 + k) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
+  };
+  load_batch(0);  // in flight with the (m, l) loads: the maximum below needs only the latter
+  float M0 = -CUDART_INF_F, M1 = -CUDART_INF_F;
+#pragma unroll
+  for (int i = 0; i < kMaxMergeParts; ++i) {
+    M0 = fmaxf(M0, a[i].x);
+    M1 = fmaxf(M1, c[i].x);
+  }
+  st.l0 = st.l1 = 0.f;
+#pragma unroll
+  for (int mt = 0; mt < D / 16; ++mt) st.o[mt][0] = st.o[mt][1] = st.o[mt][2] = st.o[mt][3] = 0.f;
+#pragma unroll
+  for (int i0 = 0; i0 < kMaxMergeParts; i0 += kB) {
+    if (i0 >= n) break;
+    if (i0 > 0) load_batch(i0);
 #pragma unroll
     for (int j = 0; j < kB; ++j) {
       const int i = i0 + j;
