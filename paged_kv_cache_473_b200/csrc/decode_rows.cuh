@@ -33,6 +33,7 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
                        const DecodeParams p) {
   using Cfg = DynCfg<D, NW, ST>;
   constexpr uint32_t FULL = 0xffffffffu;
+  constexpr bool kPairs = ST >= 4;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int G = p.group, Hkv = p.hkv, P = p.partition, B = p.batch, T = p.q_len;
@@ -239,22 +240,34 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
         row_range(ci, 16 * m + r0, cr[m].lo0, cr[m].hi0);
         row_range(ci, 16 * m + r0 + 8, cr[m].lo1, cr[m].hi1);
       }
-      for (int ck = 0; ck < ci.n; ++ck) {
+      for (int ck = 0; ck < ci.n;) {
         fill();
+        // Two slices per softmax step where the ring is deep enough to keep
+        // loading while both are attended.
+        const int step = (kPairs && ck + 1 < ci.n) ? 2 : 1;
         bool ok = mbar_wait_bounded(bars + 8 * (gc % ST), (gc / ST) & 1, kWaitLimitNs);
+        if (step == 2) ok = ok && mbar_wait_bounded(bars + 8 * ((gc + 1) % ST), ((gc + 1) / ST) & 1, kWaitLimitNs);
         ok = __all_sync(FULL, ok);
         if (!ok) {
           aborted = true;
           break;
         }
         const uint32_t kbase = ring + (gc % ST) * Cfg::kStageBytes;
+        const uint32_t kbase1 = ring + ((gc + 1) % ST) * Cfg::kStageBytes;
 #pragma unroll
-        for (int m = 0; m < MT; ++m)
-          if (m == 0 || 16 * m < R)
-            attend_slice_rows<D>(st[m], qa[m], kbase, kbase + Cfg::kSliceBytes, (ci.j0 + ck) * kSliceTokens, ci.lo,
-                                 ci.hi, cr[m], qk_scale, p, lane);
+        for (int m = 0; m < MT; ++m) {
+          if (m == 0 || 16 * m < R) {
+            if (step == 2)
+              attend_pair_rows<D>(st[m], qa[m], kbase, kbase + Cfg::kSliceBytes, kbase1, kbase1 + Cfg::kSliceBytes,
+                                  (ci.j0 + ck) * kSliceTokens, ci.lo, ci.hi, cr[m], qk_scale, p, lane);
+            else
+              attend_slice_rows<D>(st[m], qa[m], kbase, kbase + Cfg::kSliceBytes, (ci.j0 + ck) * kSliceTokens,
+                                   ci.lo, ci.hi, cr[m], qk_scale, p, lane);
+          }
+        }
         __syncwarp();
-        ++gc;
+        gc += step;
+        ck += step;
       }
       if (aborted) break;
       fill();  // keep loading the next item while this one is stored

@@ -501,4 +501,124 @@ __device__ __forceinline__ void attend_slice_rows(WarpRows<D>& st, const uint32_
   }
 }
 
+// attend_slice_rows over two consecutive slices, tokens [t0, t0+16) at
+// kbase0/vbase0 and [t0+16, t0+32) at kbase1/vbase1, in one online-softmax
+// step: one row maximum, one rescale of o and one running-sum update per 32
+// tokens, the two S products independent of each other, and O += P V as two
+// k-steps.  Same per-row bounds as attend_slice_rows.
+template <int D>
+__device__ __forceinline__ void attend_pair_rows(WarpRows<D>& st, const uint32_t (&qa)[D / 16][4], uint32_t kbase0,
+                                                 uint32_t vbase0, uint32_t kbase1, uint32_t vbase1, int t0, int lo,
+                                                 int hi, const ColRange& cr, float qk_scale, const DecodeParams& p,
+                                                 int lane) {
+  constexpr uint32_t FULL = 0xffffffffu;
+  const int mi = lane >> 3, mj = lane & 7;
+  const int tq = lane & 3;
+
+  // ---- S = Q K^T for both slices: s[slice][n-tile][4] ----------------------------------
+  float s[2][2][4];
+#pragma unroll
+  for (int a = 0; a < 2; ++a)
+#pragma unroll
+    for (int b = 0; b < 2; ++b) s[a][b][0] = s[a][b][1] = s[a][b][2] = s[a][b][3] = 0.f;
+  {
+    const int tok = ((mi >> 1) << 3) | mj;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const int chunk = 2 * kk + (mi & 1);
+      const uint32_t off = (chunk >> 3) * kPanelBytes + tok * 128 + ((((chunk & 7) ^ (tok & 7))) << 4);
+      uint32_t b00, b01, b10, b11, c00, c01, c10, c11;
+      ldsm_x4(kbase0 + off, b00, b01, b10, b11);
+      ldsm_x4(kbase1 + off, c00, c01, c10, c11);
+      mma_bf16_16816(s[0][0], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b00, b01);
+      mma_bf16_16816(s[0][1], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b10, b11);
+      mma_bf16_16816(s[1][0], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], c00, c01);
+      mma_bf16_16816(s[1][1], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], c10, c11);
+    }
+  }
+#pragma unroll
+  for (int sl = 0; sl < 2; ++sl)
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float v = s[sl][nt][e] * qk_scale;
+        if (p.use_softcap) v = p.softcap * tanhf(v * p.inv_softcap) * kLog2e;
+        const int t = t0 + 16 * sl + 8 * nt + 2 * tq + (e & 1);
+        const bool ok = e < 2 ? (t >= cr.lo0 && t < cr.hi0) : (t >= cr.lo1 && t < cr.hi1);
+        s[sl][nt][e] = ok ? v : -CUDART_INF_F;
+      }
+
+  // ---- online softmax per row over the 32 tokens -------------------------------------
+  float mx0 = -CUDART_INF_F, mx1 = -CUDART_INF_F;
+#pragma unroll
+  for (int sl = 0; sl < 2; ++sl)
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      mx0 = fmaxf(mx0, fmaxf(s[sl][nt][0], s[sl][nt][1]));
+      mx1 = fmaxf(mx1, fmaxf(s[sl][nt][2], s[sl][nt][3]));
+    }
+#pragma unroll
+  for (int off = 1; off < 4; off <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(FULL, mx0, off));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(FULL, mx1, off));
+  }
+  const float mn0 = fmaxf(st.m0, mx0), mn1 = fmaxf(st.m1, mx1);
+  const float r0 = mn0 == -CUDART_INF_F ? 0.f : mn0;
+  const float r1 = mn1 == -CUDART_INF_F ? 0.f : mn1;
+  const float al0 = exp2f(st.m0 - r0), al1 = exp2f(st.m1 - r1);
+  st.m0 = mn0;
+  st.m1 = mn1;
+  uint32_t a[2][4];  // P of each slice as the A operand of P V
+#pragma unroll
+  for (int sl = 0; sl < 2; ++sl) {
+    a[sl][0] = pack_bf16x2(exp2f(s[sl][0][0] - r0), exp2f(s[sl][0][1] - r0));
+    a[sl][1] = pack_bf16x2(exp2f(s[sl][0][2] - r1), exp2f(s[sl][0][3] - r1));
+    a[sl][2] = pack_bf16x2(exp2f(s[sl][1][0] - r0), exp2f(s[sl][1][1] - r0));
+    a[sl][3] = pack_bf16x2(exp2f(s[sl][1][2] - r1), exp2f(s[sl][1][3] - r1));
+  }
+  st.l0 = st.l0 * al0 + ((bf16_lo(a[0][0]) + bf16_hi(a[0][0]) + bf16_lo(a[0][2]) + bf16_hi(a[0][2])) +
+                         (bf16_lo(a[1][0]) + bf16_hi(a[1][0]) + bf16_lo(a[1][2]) + bf16_hi(a[1][2])));
+  st.l1 = st.l1 * al1 + ((bf16_lo(a[0][1]) + bf16_hi(a[0][1]) + bf16_lo(a[0][3]) + bf16_hi(a[0][3])) +
+                         (bf16_lo(a[1][1]) + bf16_hi(a[1][1]) + bf16_lo(a[1][3]) + bf16_hi(a[1][3])));
+#pragma unroll
+  for (int nt = 0; nt < D / 8; ++nt) {
+    st.o[nt][0] *= al0;
+    st.o[nt][1] *= al0;
+    st.o[nt][2] *= al1;
+    st.o[nt][3] *= al1;
+  }
+
+  // V rows outside [lo, hi) may hold anything (NaN canaries): zero them.
+  uint32_t keep_lo[2] = {0xffffffffu, 0xffffffffu}, keep_hi[2] = {0xffffffffu, 0xffffffffu};
+#pragma unroll
+  for (int sl = 0; sl < 2; ++sl) {
+    const int ts = t0 + 16 * sl;
+    if (ts < lo || ts + kSliceTokens > hi) {
+      const int tc = ts + 2 * tq;
+      auto ok = [&](int t) { return t >= lo && t < hi; };
+      keep_lo[sl] = (ok(tc) ? 0x0000ffffu : 0u) | (ok(tc + 1) ? 0xffff0000u : 0u);
+      keep_hi[sl] = (ok(tc + 8) ? 0x0000ffffu : 0u) | (ok(tc + 9) ? 0xffff0000u : 0u);
+    }
+  }
+
+  // ---- O += P V, one k-step per slice ----------------------------------------------------
+  {
+    const int tok = ((mi & 1) << 3) | mj;
+#pragma unroll
+    for (int c = 0; c < D / 16; ++c) {
+      const int chunk = 2 * c + (mi >> 1);
+      const uint32_t off = (chunk >> 3) * kPanelBytes + tok * 128 + ((((chunk & 7) ^ (tok & 7))) << 4);
+#pragma unroll
+      for (int sl = 0; sl < 2; ++sl) {
+        uint32_t v0, v1, v2, v3;
+        ldsm_x4_trans((sl ? vbase1 : vbase0) + off, v0, v1, v2, v3);
+        mma_bf16_16816(st.o[2 * c], a[sl][0], a[sl][1], a[sl][2], a[sl][3], v0 & keep_lo[sl], v1 & keep_hi[sl]);
+        mma_bf16_16816(st.o[2 * c + 1], a[sl][0], a[sl][1], a[sl][2], a[sl][3], v2 & keep_lo[sl],
+                       v3 & keep_hi[sl]);
+      }
+    }
+  }
+}
+
 }  // namespace pa
