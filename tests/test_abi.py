@@ -82,11 +82,22 @@ def _decode(**kw):
 def test_decode_host_checks(kw, status):
     assert _decode(**kw) == status
     assert pa.last_launch_count() == 0
+    assert pa.last_decode_schedule() == "none"  # a refused call ran no schedule
 
 
 def test_empty_batch_is_a_no_op():
     assert _decode(B=0, q=None, out=None) == bnd.PA_OK
     assert pa.last_launch_count() == 0
+    assert pa.last_decode_schedule() == "none"
+
+
+def test_schedule_names_match_the_header():
+    """pa_schedule_t's values as the binding names them."""
+    src = open(HEADER).read()
+    body = src[src.index("typedef enum {\n  PA_SCHEDULE_NONE"):]
+    body = body[:body.index("} pa_schedule_t;")]
+    vals = {int(v): n for n, v in re.findall(r"PA_SCHEDULE_(\w+) = (\d+)", body)}
+    assert {k: v.lower() for k, v in vals.items()} == bnd.SCHEDULES
 
 
 def _splitk(**kw):
