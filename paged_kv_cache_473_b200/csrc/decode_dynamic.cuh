@@ -193,15 +193,14 @@ __device__ __forceinline__ void store_partial_lanes(const WarpAttn<D>& st, const
 // (m, l) come from registers.
 // The loads of kB partials are issued before any is used (one L2 round trip
 // per batch), the first batch together with the (m, l) loads.
-template <int D>
+// Partials per batch (kB): at head_dim 64 with six-stage rings all of them, so
+// that every load of the merge, (m, l) included, is in one L2 round trip (two
+// CTAs per SM are set by shared memory, so the registers cost no occupancy);
+// the configurations sized for three CTAs per SM run at a 168-register cap.
+template <int D, int kB>
 __device__ __forceinline__ void merge_lanes(WarpAttn<D>& st, const DecodeParams& p, size_t row0, int pb, int n,
                                             int own, int G, int lane) {
   constexpr int V = D / 32;                // 16-byte vectors per head per lane
-  // Partials per batch.  At head_dim 64 all of them, so that every load of the
-  // merge, (m, l) included, is in one L2 round trip (the kernel's two CTAs per
-  // SM are set by shared memory, so the registers cost no occupancy); head_dim
-  // 128 runs at a 170-register cap.
-  constexpr int kB = D == 64 ? kMaxMergeParts : 1;
   const int n0 = 2 * (lane & 3), r = lane >> 2;
   const bool h0 = n0 < G, h1 = n0 + 1 < G;
   const size_t slot0 = (row0 + n0) * p.max_parts + pb;
@@ -291,10 +290,16 @@ struct DynCfg {
 // Resident CTAs per SM the configurations are sized for (shared memory allows
 // that many): the register budget ptxas may use follows from it.
 template <int D>
-constexpr int dynamic_min_blocks() { return D == 128 ? 3 : 2; }
+__host__ __device__ constexpr int dynamic_min_blocks() { return D == 128 ? 3 : 2; }
+// The decode kernel's: head_dim 64 with rings of at most four stages (the
+// configuration for steps merged by the combine kernel) runs three CTAs.
+template <int D, int ST>
+__host__ __device__ constexpr int decode_min_blocks() { return D == 64 && ST <= 4 ? 3 : dynamic_min_blocks<D>(); }
+template <int D, int ST>
+__host__ __device__ constexpr int merge_batch() { return D == 64 ? (decode_min_blocks<D, ST>() == 2 ? kMaxMergeParts : 2) : 1; }
 
 template <int D, int NW, int ST, bool APPEND, bool CASCADE = false>
-__global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
+__global__ void __launch_bounds__(NW * 32, decode_min_blocks<D, ST>())
     decode_dynamic_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                           const DecodeParams p) {
   using Cfg = DynCfg<D, NW, ST>;
@@ -593,7 +598,7 @@ __global__ void __launch_bounds__(NW * 32, dynamic_min_blocks<D>())
         if (lane == 0) last = atom_add_acq_rel_gpu(cnt, 1) == ci.parts - 1;
         if (__shfl_sync(FULL, last, 0)) {
           __syncwarp();
-          merge_lanes<D>(st, p, row0, ci.pb, ci.parts, ci.part - ci.pb, G, lane);
+          merge_lanes<D, merge_batch<D, ST>()>(st, p, row0, ci.pb, ci.parts, ci.part - ci.pb, G, lane);
           write_rows = true;
           if (lane == 0) *cnt = 0;  // every partial of the unit has arrived: ready for the next call
         }

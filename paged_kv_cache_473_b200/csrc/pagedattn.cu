@@ -456,8 +456,19 @@ cudaError_t launch_dynamic(DecodeParams& p, cudaStream_t st) {
   switch (p.head_dim) {
     // Warps are independent (one work item each); CTAs of a few warps with a
     // 2-6 stage ring each put ~192 KB of loads in flight per SM.
-    case 64:
-      return launch_dynamic_t<64, 4, 6, APPEND, CASCADE>(p, st, pdl, allow_merge);
+    case 64: {
+      // Steps small enough for the in-kernel merge (bounded on the host as in
+      // launch_dynamic_t, for two resident CTAs of four warps): 8 warps per SM
+      // with six-stage rings, the merge's loads in one L2 round trip.  Larger
+      // steps, merged by the combine kernel: 12 warps per SM (three CTAs,
+      // four-stage rings), so more items stream at once (measured on B200:
+      // TinyLlama shape with 128 sequences 47.2 -> 42.7 us; at 64 sequences,
+      // merged in-kernel, the six-stage configuration is 1.8 us faster).
+      const long long unit_bound = (long long)p.batch * p.hkv * p.max_parts;
+      const bool merge = allow_merge && p.max_parts <= pa::kMaxMergeParts && unit_bound <= 2LL * (2 * 4) * sm_count();
+      if (merge) return launch_dynamic_t<64, 4, 6, APPEND, CASCADE>(p, st, pdl, true);
+      return launch_dynamic_t<64, 4, 4, APPEND, CASCADE>(p, st, pdl, false);
+    }
     case 128:
       return launch_dynamic_t<128, 4, 2, APPEND, CASCADE>(p, st, pdl, allow_merge);
     default:
