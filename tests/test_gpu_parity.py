@@ -508,6 +508,8 @@ def test_dynamic_schedule_counters_return_to_zero():
     ("gemma2_2b", dict(batch=256), None, "dynamic"),
     ("llama3_8b", dict(batch=128, max_len=2048), None, "dynamic"),
     ("tinyllama_1b", dict(batch=256), None, "dynamic"),
+    # head_dim 64 merged by the combine: the 12-warp-per-SM configuration
+    ("tinyllama_1b", dict(batch=128), None, "dynamic"),
 ])
 def test_dynamic_schedule_counter_region_reads_zero_after_each_call(name, kw, max_ctx, schedule):
     """Whichever way the partitions are merged, and whether or not warps claim
